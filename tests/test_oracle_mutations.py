@@ -1,0 +1,103 @@
+"""Planted mistakes in the oracle must trip the pins.
+
+Each mutation below is a plausible slip (a dropped term, a wrong sign or
+index, a mean for a sum, a transposed pairing).  It is applied to a copy of
+``oracle/tri_oracle.c`` in a temporary directory, built on the CPU, swapped in
+for the real oracle, and the pins of ``test_oracle_pins.py`` are run against
+it: at least one must fail.  The real oracle is never modified.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "tri_oracle.c")
+
+# (name, [(old, new), ...]) - every `old` must occur in the source.
+MUTATIONS = [
+    ("norm term dropped",
+     [(" + ((ldbl)mnorm[g * F + f] - qn[g * F + f]) * kn;", ";")]),
+    ("mean over offsets instead of sum",
+     [("sg += qn[g * F + f] * kn * trig", "sg += qn[g * F + f] * kn * trig / n_off")]),
+    ("offset subtracted",
+     [("(p_now + offsets[e] - pos[j])", "(p_now - offsets[e] - pos[j])")]),
+    ("frequency exponent -f/d",
+     [("-2.0L * (ldbl)f / (ldbl)d", "-1.0L * (ldbl)f / (ldbl)d")]),
+    ("de-rotation by +angle",
+     [("*re = xr * c + xi * s;", "*re = xr * c - xi * s;"),
+      ("*im = xi * c - xr * s;", "*im = xi * c + xr * s;")]),
+    ("interleaved pairing",
+     [("ldbl xr = key[f], xi = key[f + F];", "ldbl xr = key[2 * f], xi = key[2 * f + 1];")]),
+    ("phase sign flipped",
+     [("ldbl phi = qa[g * F + f] - atan2l(ki, kr);", "ldbl phi = atan2l(ki, kr) - qa[g * F + f];")]),
+    ("distance uses slot sign reversed",
+     [("cosl(w[f] * (ldbl)(p_now + offsets[e] - pos[j]) + phi)",
+       "cosl(w[f] * (ldbl)(pos[j] - p_now - offsets[e]) + phi)")]),
+    ("GQA sum instead of mean",
+     [("out[j] = (double)(total / (ldbl)G);", "out[j] = (double)total;")]),
+    ("calibration norm of the mean",
+     [("mnorm[f] = (double)(sn / (ldbl)nq);", "mnorm[f] = (double)hypotl(sr / (ldbl)nq, si / (ldbl)nq);")]),
+    ("calibration drops the imaginary half",
+     [("ldbl xr = q[t * d + f], xi = q[t * d + f + F];", "ldbl xr = q[t * d + f], xi = 0.0L * q[t * d + f + F];")]),
+    ("tie-break keeps the older slot",
+     [("if (a->i != b->i) return a->i > b->i ? -1 : 1;", "if (a->i != b->i) return a->i < b->i ? -1 : 1;")]),
+    ("window not protected",
+     [("for (int64_t j = M; j < n; j++) keep[j] = 1;", "for (int64_t j = M; j < n; j++) keep[j] = 0;")]),
+    ("budget excludes the window",
+     [("const int64_t M = n - W, K = B - W;", "const int64_t M = n - W, K = B;")]),
+    ("gather off by one",
+     [("memcpy(dst + t * width, src + idx[t] * width, (size_t)width);",
+       "memcpy(dst + t * width, src + (idx[t] > 0 ? idx[t] - 1 : 0) * width, (size_t)width);")]),
+]
+
+PIN_FUNCS = [
+    lambda: pins.test_omega_is_theta_power(),
+    lambda: pins.test_trig_series_equals_rope_dot_at_every_distance(0),
+    lambda: pins.test_golden_closed_forms(),
+    lambda: pins.test_identical_queries_give_attention_logit_sum(True),
+    lambda: pins.test_identical_queries_give_attention_logit_sum(False),
+    lambda: pins.test_zero_centre_gives_norm_sum(True),
+    lambda: pins.test_two_queries_trig_and_norm_parts(),
+    lambda: pins.test_calib_single_query(),
+    lambda: pins.test_calib_matches_numpy_and_triangle_inequality(),
+    lambda: pins.test_select_brute_force_tiny_rows(),
+    lambda: pins.test_select_matches_lexsort_and_invariants(),
+    lambda: pins.test_select_all_equal_keeps_most_recent(),
+    lambda: pins.test_gather_matches_fancy_indexing(),
+]
+
+
+def _failing_pins():
+    failed = 0
+    for fn in PIN_FUNCS:
+        try:
+            fn()
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    return failed
+
+
+@pytest.mark.parametrize("name,edits", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(tmp_path, name, edits):
+    src = open(SRC).read()
+    for old, new in edits:
+        assert old in src, f"mutation anchor not found: {old!r}"
+        src = src.replace(old, new)
+    mpath = tmp_path / "mut.c"
+    mpath.write_text(src)
+    so = tmp_path / "libmut.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(so),
+                    str(mpath), "-lm"], check=True)
+    saved = oracle.lib()
+    oracle._lib = oracle.load(str(so))
+    try:
+        assert _failing_pins() >= 1, f"no pin caught: {name}"
+    finally:
+        oracle._lib = saved
+
+
+def test_unmutated_oracle_passes_every_pin():
+    assert _failing_pins() == 0
