@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Throughput of TriAttention KV-cache compression on B200: keys scored + selected +
+compacted per second, and the fraction of the HBM roofline.
+
+One step = tri_score + tri_compact over the whole workload (every row of every
+layer), inputs resident in HBM (larger than L2).  Calibration (tri_calib) is
+offline and timed separately.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload qwen3_8b_32k] [--budget B] [--key-mode post|pre]
+
+N > 1 (under torchrun): every rank compacts its own cache of the same shape
+(independent sequences; no collective on the data path), timing is the max
+over ranks, value = keys of all ranks / that time (weak scaling).
+--impl reference times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "keys scored+selected+compacted/sec per B200 and % of HBM roofline"
+UNIT = "keys/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+SCORE_BYTES_PER_KEY = 256 + 4  # read the bf16 key, write its fp32 score
+KEPT_BYTES = 4 * 256 + 8  # read + write K and V of a kept key, read + write its position
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_8b_32k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--key-mode", choices=["post", "pre"], default="post")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def workload_config(wl, B, key_mode):
+    lo, hi = wl.seq_len
+    return {"workload": wl.name, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "rope_theta": wl.theta,
+            "batch": wl.batch, "keys_per_head": lo if lo == hi else [lo, hi], "budget": B,
+            "window": wl.window, "offsets": wl.n_offsets, "key_mode": key_mode + "_rope",
+            "layout": wl.layout,
+            "l2": "inputs larger than L2: K+V %.1f GB read per step, no flush" % (
+                2 * 256 * wl.n_layers * wl.batch * wl.n_kv_heads * np.mean(wl.seq_len) / 1e9)}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def score_kernel_sha():
+    h = hashlib.sha256()
+    for f in ("score.cu", "tri_internal.cuh"):
+        with open(os.path.join(ROOT, "kv_cache_compression_calib_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(total_keys):
+    """DRAM bytes per launch of the score kernel from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "score_kernel_traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except Exception:
+        return None
+    if rec.get("kernel_sha") != score_kernel_sha():
+        return None
+    return float(rec["dram_bytes_per_key"]) * total_keys
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms from before the
+    warm-up until after the timed region; only samples stamped inside the timed
+    region (widened by one interval when it is shorter than that) are reported."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.ident = str(device_index)
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.ident, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t_begin, t_end):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(p[1]), float(p[2]), p[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        pad = 0.0 if t_end - t_begin >= 0.3 else 0.12
+        win = [r for r in rows if t_begin - pad <= r[0] <= t_end + pad]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "timed region shorter than the sampling interval"}
+        reasons = sorted({self.REASONS[i] for r in win for i in range(4) if r[3][i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in win), "sm_max_mhz": max(r[2] for r in win),
+                "reasons": reasons, "samples": len(win)}
+
+
+# ------------------------------------------------------- multi-rank logic
+
+def rank_workload(wl, rank: int, B: int):
+    """Rank r compacts its own independent cache of the same shape (other sequences):
+    same workload, seed offset by the rank.  No rank reads another's rows."""
+    return wl.with_(budget=B, seed=wl.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time (all-reduce MAX; NCCL on GPUs, gloo on CPU)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(keys_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job keys per second: every rank's keys over the slowest rank's step time."""
+    return keys_per_rank * world / (ms_per_step / 1e3)
+
+
+# ----------------------------------------------------------------- ours
+
+def run_ours(a, rank, world, local_rank):
+    import kv_cache_compression_calib_b200 as tri
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl0 = synth.WORKLOADS[a.workload]
+    B = a.budget or wl0.budget
+    wl = rank_workload(wl0, rank, B)
+    key_mode = tri.TRI_KEYS_PRE_ROPE if a.key_mode == "pre" else tri.TRI_KEYS_POST_ROPE
+    if wl.layout != "contig":
+        raise SystemExit("bench.py times the contiguous workloads; the paged one is a parity case")
+    cache = synth.make_contig(wl, dev, rotate=(a.key_mode == "post"))
+    L, S, Hh = wl.n_layers, len(cache.lens), wl.n_kv_heads
+    R, total = cache.n_rows, cache.total
+    m = tri.model(L, wl.n_q_heads, Hh, wl.theta)
+    kv = tri.kv_contig(S, cache.row_off, total)
+    stream = torch.cuda.current_stream(dev)
+
+    # offline calibration (timed separately, not part of a step)
+    centres = torch.empty(L, wl.n_q_heads, 64, 2, dtype=torch.float32, device=dev)
+    mnorm = torch.empty(L, wl.n_q_heads, 64, dtype=torch.float32, device=dev)
+    tri.tri_calib(m, cache.qcal, wl.n_calib, centres, mnorm)
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record()
+    tri.tri_calib(m, cache.qcal, wl.n_calib, centres, mnorm)
+    c1.record()
+    torch.cuda.synchronize()
+    calib_ms = c0.elapsed_time(c1)
+
+    ws = tri.alloc_workspace(m, S, B, device=dev)
+    scores = torch.empty(total, dtype=torch.float32, device=dev)
+    Ko = torch.empty(R, B, 128, dtype=torch.bfloat16, device=dev)
+    Vo = torch.empty_like(Ko)
+    po = torch.empty(R, B, dtype=torch.int32, device=dev)
+    kept = torch.empty(R, B, dtype=torch.int32, device=dev)
+    offsets = wl.offsets
+
+    def step():
+        tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode, scores, ws,
+                      stream)
+        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
+                        kept, None, ws, stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, flags = tri.tri_status_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} after warm-up")
+
+    # ---- device-resident timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t0.record(stream)
+    for i in range(a.steps):
+        ev[i][0].record(stream)
+        tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode, scores, ws,
+                      stream)
+        ev[i][1].record(stream)
+        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
+                        kept, None, ws, stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(wall0, wall1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    score_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    st, flags = tri.tri_status_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} in the timed region")
+
+    lens_rows = np.diff(cache.row_off_np)
+    keys_step = int(total)
+    alg_bytes = float(np.sum(256.0 * lens_rows + np.minimum(lens_rows, B) * KEPT_BYTES))
+    if key_mode == tri.TRI_KEYS_PRE_ROPE:
+        alg_bytes += 4.0 * total
+    ms_step = ms / a.steps
+    value = throughput(keys_step, world, ms_step)
+
+    # ---- end to end through the public API: pinned host inputs, copies in the region
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream,
+                      world, dev)
+
+    peak, peak_kind = measured_peak()
+    score_bytes = SCORE_BYTES_PER_KEY * total
+    achieved = score_bytes / (score_ms / 1e3) / 1e9
+    path_gbs = alg_bytes / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(wl, B, a.key_mode),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(total),
+                     "kernel": "tri_score (prep + score kernels)", "peak_kind": peak_kind,
+                     "bytes_per_launch": score_bytes, "ms_per_launch": score_ms},
+        "path_roofline": {"bytes_per_step": alg_bytes, "achieved_gbs": path_gbs,
+                          "frac_of_measured": path_gbs / peak, "frac_of_8tbs": path_gbs / NOMINAL_HBM_GBS},
+        "calib_ms": calib_ms,
+        "gpu_launches": 4 * a.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, B, cache, a.cpu_seconds)
+    return line
+
+
+def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream, world,
+            dev):
+    try:
+        hK = cache.K.cpu().pin_memory()
+        hV = cache.V.cpu().pin_memory()
+        hpos = cache.pos.cpu().pin_memory()
+        hro = cache.row_off.cpu().pin_memory()
+        hpn = cache.p_now.cpu().pin_memory()
+        hc = centres.cpu().pin_memory()
+        hm = mnorm.cpu().pin_memory()
+        oK = torch.empty(Ko.shape, dtype=Ko.dtype).pin_memory()
+        oV = torch.empty(Vo.shape, dtype=Vo.dtype).pin_memory()
+        op = torch.empty(po.shape, dtype=po.dtype).pin_memory()
+        ok = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
+    except RuntimeError as e:
+        return {"value": None, "unit": UNIT, "skipped": f"pinned host buffers: {e}"[:200]}
+    ins = [(cache.K, hK), (cache.V, hV), (cache.pos, hpos), (cache.row_off, hro), (cache.p_now, hpn),
+           (centres, hc), (mnorm, hm)]
+    outs = [(oK, Ko), (oV, Vo), (op, po), (ok, kept)]
+    h2d = sum(h.numel() * h.element_size() for _, h in ins)
+    d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+    steps = max(3, min(a.steps, 10))
+
+    def step():
+        for d, h in ins:
+            d.copy_(h, non_blocking=True)
+        tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, wl.offsets, key_mode, scores, ws,
+                      stream)
+        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
+                        kept, None, ws, stream)
+        for h, d in outs:
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    return {"value": throughput(cache.total, world, ms / steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps}
+
+
+# ------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs, ms, rows_meta, seconds, max_rows):
+    """Time the oracle (collapsed score + select + gather) on rows until `seconds` pass."""
+    import oracle
+
+    keys = 0
+    n_rows = 0
+    t0 = time.perf_counter()
+    for i in range(max_rows):
+        j = i % len(rows_meta)
+        h, p_now = rows_meta[j]
+        Kf = oracle.bf16_bits_to_f64(K_rows[j])
+        s = oracle.row_scores(wl.theta, cs, ms, h, wl.group, Kf, pos_rows[j], True, p_now, wl.offsets,
+                              "collapsed")
+        kept = oracle.select(s, B, wl.window)
+        oracle.gather(K_rows[j], kept)
+        oracle.gather(V_rows[j], kept)
+        oracle.gather(pos_rows[j], kept)
+        keys += len(s)
+        n_rows += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return keys, n_rows, dt
+
+
+def cpu_baseline(wl, B, cache, seconds):
+    import oracle
+    from tests import harness as H
+
+    Hh = wl.n_kv_heads
+    rows = list(range(min(Hh, cache.n_rows)))  # layer 0, sequence 0, every KV head
+    K_rows, V_rows, pos_rows, meta = [], [], [], []
+    for r in rows:
+        a, b = cache.row_off_np[r], cache.row_off_np[r + 1]
+        K_rows.append(H.bits16(cache.K[a:b]))
+        V_rows.append(H.bits16(cache.V[a:b]))
+        pos_rows.append(cache.pos[a:b].cpu().numpy().astype(np.int64))
+        _, s, h = cache.row_lhs(r)
+        meta.append((h, int(cache.lens[s])))
+    cs, ms = H.oracle_calibration(cache.qcal[:1])
+    keys, n_rows, dt = oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs[0], ms[0], meta, seconds, 64)
+    return {"value": keys / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_rows} rows x {len(K_rows[0])} keys of layer 0 (score collapsed fp64 + select + gather), "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(a, rank, world):
+    import oracle
+    from tests import harness as H
+
+    wl0 = synth.WORKLOADS[a.workload]
+    B = a.budget or wl0.budget
+    wl = wl0.with_(budget=B)
+    cache = synth.make_contig(wl, "cpu", layers=[0], lens=wl.seq_lengths()[:1])
+    Hh = wl.n_kv_heads
+    K_rows, V_rows, pos_rows, meta = [], [], [], []
+    for r in range(Hh):
+        a_, b_ = cache.row_off_np[r], cache.row_off_np[r + 1]
+        K_rows.append(H.bits16(cache.K[a_:b_]))
+        V_rows.append(H.bits16(cache.V[a_:b_]))
+        pos_rows.append(cache.pos[a_:b_].numpy().astype(np.int64))
+        meta.append((r % Hh, int(cache.lens[0])))
+    cs, ms = H.oracle_calibration(cache.qcal)
+    for i in range(a.warmup):
+        oracle_sample(wl, B, K_rows[i % Hh:i % Hh + 1], V_rows[i % Hh:i % Hh + 1], pos_rows[i % Hh:i % Hh + 1],
+                      cs[0], ms[0], meta[i % Hh:i % Hh + 1], 0.0, 1)
+    keys = 0
+    t0 = time.perf_counter()
+    for i in range(a.steps):
+        j = i % Hh
+        k, _, _ = oracle_sample(wl, B, K_rows[j:j + 1], V_rows[j:j + 1], pos_rows[j:j + 1], cs[0], ms[0],
+                                meta[j:j + 1], 0.0, 1)
+        keys += k
+    dt = time.perf_counter() - t0
+    value = keys / dt
+    sample = f"1 row ({len(K_rows[0])} keys) of layer 0 per step (score collapsed fp64 + select + gather)"
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": workload_config(wl, B, "post"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(a, rank, world)), flush=True)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(a, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

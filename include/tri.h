@@ -1,0 +1,213 @@
+/*
+ * tri.h - C ABI of libtri.so: TriAttention KV-cache key scoring, per-head top-B
+ * selection and K/V compaction on NVIDIA B200 (sm_100a).
+ *
+ * The method ("TriAttention：基于三角函数 KV 压缩的高效长推理", whatsmy.fun paper
+ * digest, section 流程详解 steps 1-4; "WeianMao/triattention" project card,
+ * "How it works"): pre-RoPE query centres are calibrated offline (step 1);
+ * every cached key is scored by a trigonometric series in its RoPE distance to
+ * the future positions p_now + delta (step 2) plus a norm term (step 3); each
+ * KV head keeps its B best keys, the W most recent always among them, and the
+ * cache is compacted to those keys (step 4).  The score of the key at position
+ * j in the cache row of KV head h is
+ *
+ *   S_j = (1/G) sum_{g in group(h)} [ sum_f |qbar_f^g| |k_f| sum_delta cos(w_f (p_now + delta - j) + phi_f^g)
+ *                                    + sum_f (E|q_f^g| - |qbar_f^g|) |k_f| ],
+ *   w_f = rope_theta^(-2f/d),  phi_f^g = arg qbar_f^g - arg k_f,
+ *
+ * k the pre-RoPE key, pairs f = dims (f, f + d/2) (rotate-half RoPE, as in
+ * Qwen3/Llama), group(h) = query heads h*G .. h*G+G-1, G = n_q_heads/n_kv_heads.
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers on the current device, allocated
+ *    and owned by the caller; the library allocates nothing and keeps no state
+ *    besides a per-device cache of SM counts.  Every call is asynchronous on
+ *    `stream` (a cudaStream_t; NULL = the legacy default stream) and returns
+ *    after enqueuing its kernels.
+ *  - bf16 tensors are passed as `void*` and hold IEEE bfloat16 bit patterns.
+ *  - Arguments are checked on the host before anything is launched; a failed
+ *    check returns its status and launches nothing.  Kernels never trap and
+ *    never wait on other blocks: data anomalies they detect (see TRI_FLAG_*)
+ *    are OR-ed into a flag word in the workspace, read by tri_status_check.
+ *  - A "row" is one (layer l, sequence s, KV head h), numbered
+ *    r = (l * n_seqs + s) * n_kv_heads + h; R = n_layers * n_seqs * n_kv_heads.
+ */
+#ifndef TRI_H
+#define TRI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *tri_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    TRI_OK = 0,
+    TRI_ERR_INVALID_ARG = 1,         /* null pointer, negative size, inconsistent shapes */
+    TRI_ERR_UNSUPPORTED = 2,         /* head_dim != 128, block size not a power of two, ... */
+    TRI_ERR_ALIGNMENT = 3,           /* a pointer is not aligned as documented */
+    TRI_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < tri_workspace_size(...) */
+    TRI_ERR_CUDA = 5,                /* a CUDA launch or copy failed */
+    TRI_ERR_DEVICE_FLAG = 6          /* tri_status_check found a flag set by a kernel */
+} tri_status;
+
+/* Flag bits that kernels OR into the workspace flag word. */
+#define TRI_FLAG_ROW_OFFSETS 0x1u /* row_off not non-decreasing from 0 to total_keys */
+#define TRI_FLAG_NONFINITE 0x2u   /* a NaN score reached selection (ranked last) */
+#define TRI_FLAG_BLOCK_TABLE 0x4u /* paged: block id out of [0, n_blocks) or row too long for the table; the key is skipped */
+
+#define TRI_MAX_OFFSETS 64
+#define TRI_HEAD_DIM 128
+
+enum { TRI_KV_CONTIG = 0, TRI_KV_PAGED = 1 };
+enum { TRI_KEYS_POST_ROPE = 0, TRI_KEYS_PRE_ROPE = 1 };
+
+typedef struct {
+    int32_t head_dim;   /* d; only 128 is supported */
+    int32_t n_layers;   /* L >= 1 */
+    int32_t n_q_heads;  /* Hq >= 1 */
+    int32_t n_kv_heads; /* H >= 1, Hq % H == 0 */
+    double rope_theta;  /* theta > 1 */
+} tri_model;
+
+/*
+ * Where the cached keys of each row live.
+ *  TRI_KV_CONTIG: K is [total_keys][d] bf16 and pos is [total_keys] int32; row r
+ *    is entries row_off[r] .. row_off[r+1]-1 (rows of any length, in row order).
+ *  TRI_KV_PAGED (vLLM block layout): K is [n_layers][n_blocks][block_size][H][d]
+ *    bf16 and pos is [n_layers][n_blocks][block_size][H] int32; slot j of
+ *    sequence s is slot j % block_size of block block_table[s][j / block_size],
+ *    the same table for every layer.  row_off then only describes the score
+ *    buffer (row r's scores are entries row_off[r] .. row_off[r+1]-1) and the
+ *    row lengths.
+ * In both layouts the score buffer is float [total_keys], indexed like row_off.
+ */
+typedef struct {
+    int32_t layout;         /* TRI_KV_CONTIG or TRI_KV_PAGED */
+    int32_t n_seqs;         /* S >= 1 */
+    int64_t total_keys;     /* must equal row_off[R] */
+    const int64_t *row_off; /* device [R + 1], row_off[0] = 0, non-decreasing */
+    /* TRI_KV_PAGED only (ignored for TRI_KV_CONTIG): */
+    const int32_t *block_table; /* device [n_seqs][max_blocks] */
+    int32_t max_blocks;         /* >= 1 */
+    int32_t block_size;         /* power of two, 1 .. 1024 (vLLM: 16) */
+    int64_t n_blocks;           /* blocks per layer in the pool, >= 1 */
+} tri_kv_desc;
+
+/*
+ * Where tri_compact writes the kept keys.
+ *  TRI_KV_CONTIG: K_out/V_out are [R][B][d], pos_out [R][B]: kept slot i of row
+ *    r goes to entry r * B + i.
+ *  TRI_KV_PAGED: K_out/V_out are [n_layers][n_blocks][block_size][H][d] and
+ *    pos_out [n_layers][n_blocks][block_size][H]; kept slot i of row (l, s, h)
+ *    goes to slot i % block_size of block block_table[s][i / block_size] -
+ *    a fresh table chosen by the caller's block allocator, which needs
+ *    ceil(min(N, B) / block_size) <= max_blocks entries per sequence.
+ */
+typedef struct {
+    int32_t layout;
+    int32_t max_blocks;
+    const int32_t *block_table;
+    int32_t block_size;
+    int32_t pad_;
+    int64_t n_blocks;
+} tri_out_desc;
+
+/* Human-readable name of a status code (static string). */
+const char *tri_status_str(tri_status s);
+
+/* Library version, (major << 16) | minor. */
+uint32_t tri_version(void);
+
+/*
+ * Bytes of workspace that tri_score and tri_compact need for `m` and `n_seqs`
+ * sequences with budget B.  One buffer may serve both calls (they run in
+ * stream order).  The workspace must be 256-byte aligned device memory.
+ */
+size_t tri_workspace_size(const tri_model *m, int32_t n_seqs, int32_t B);
+
+/* Clear the workspace flag word (enqueued on `stream`).  Call once after
+ * allocating a workspace; tri_status_check clears it again after reading. */
+tri_status tri_workspace_init(void *ws, size_t ws_bytes, tri_stream_t stream);
+
+/*
+ * Offline calibration (digest, 流程详解 step 1): for every (layer l, query head g)
+ * and pair f, the complex mean of the pre-RoPE queries and the mean of their
+ * magnitudes,
+ *   centres[l][g][f] = (1/nq) sum_t (q[t][f] + i q[t][f+64])          (re, im)
+ *   mean_norm[l][g][f] = (1/nq) sum_t |q[t][f] + i q[t][f+64]|,
+ * accumulated in fp64, stored fp32.
+ *   qpre:      bf16 [n_layers][n_q_heads][nq][128], 16-byte aligned
+ *   nq:        queries per head, >= 1
+ *   centres:   float [n_layers][n_q_heads][64][2]
+ *   mean_norm: float [n_layers][n_q_heads][64]
+ */
+tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *centres,
+                     float *mean_norm, tri_stream_t stream);
+
+/*
+ * Score every cached key (digest, 流程详解 steps 2-3) with the rule in the
+ * header comment, the GQA mean taken over the query heads of each KV head.
+ *   kv:        layout and row offsets of the cache
+ *   K:         bf16 keys in kv's layout, 16-byte aligned
+ *   pos:       int32 position of every cached slot (kv's layout).  Read only
+ *              for TRI_KEYS_PRE_ROPE; may be NULL for TRI_KEYS_POST_ROPE.
+ *   centres, mean_norm: calibration of tri_calib, [n_layers][n_q_heads][64](x2)
+ *   p_now:     device int64 [n_seqs], the position of each sequence's next token
+ *   offsets:   HOST int32 [n_offsets], the future offsets delta, 1 <= n_offsets
+ *              <= TRI_MAX_OFFSETS (copied into the launch; not kept)
+ *   key_mode:  TRI_KEYS_POST_ROPE: K holds RoPE-rotated keys (as an inference
+ *              cache does): the key's own rotation cancels the -j of the
+ *              distance, so pos is not needed and no per-key sin/cos is taken.
+ *              TRI_KEYS_PRE_ROPE: K holds pre-RoPE keys; one sin/cos per
+ *              (key, pair) of w_f (p_now - pos) is taken, with the phase
+ *              reduced exactly in 64-bit fixed-point turns.
+ *   scores:    float [kv->total_keys], 4-byte aligned
+ *   ws:        workspace of tri_workspace_size bytes
+ * Scores are fp32 with fp32 accumulation; per-row coefficients are formed in
+ * fp64.
+ */
+tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, const int32_t *pos,
+                     const float *centres, const float *mean_norm, const int64_t *p_now,
+                     const int32_t *offsets, int32_t n_offsets, int32_t key_mode, float *scores,
+                     void *ws, size_t ws_bytes, tri_stream_t stream);
+
+/*
+ * Per-row top-B selection and stable compaction (digest, 流程详解 step 4).
+ * For a row of N keys:
+ *   N <= B: every slot is kept (identity compaction);
+ *   N >  B: the last W slots are kept, plus the B - W best of slots
+ *           0 .. N-W-1 under the order (score descending, slot descending),
+ *           so exactly B keys survive and equal scores favour recent slots.
+ *           NaN scores rank last (and set TRI_FLAG_NONFINITE).
+ * Kept slots are emitted in ascending slot order, and K, V and pos of each
+ * kept slot are copied bit for bit to the output.
+ *   scores:     float, as written by tri_score for the same kv
+ *   B, W:       1 <= B, 0 <= W <= B
+ *   K, V, pos:  the cache in kv's layout (pos may be NULL if pos_out is NULL)
+ *   out:        layout of the outputs; K_out/V_out 16-byte aligned, must not
+ *               overlap K/V
+ *   kept_idx:   optional int32 [R][B]: kept slots of row r at r*B .. r*B+cnt-1
+ *   kept_count: optional int32 [R]: min(N, B) per row
+ *   ws:         workspace of tri_workspace_size bytes
+ */
+tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *scores, int32_t B,
+                       int32_t W, const void *K, const void *V, const int32_t *pos,
+                       const tri_out_desc *out, void *K_out, void *V_out, int32_t *pos_out,
+                       int32_t *kept_idx, int32_t *kept_count, void *ws, size_t ws_bytes,
+                       tri_stream_t stream);
+
+/*
+ * Synchronise `stream`, read the workspace flag word into *flags (may be
+ * NULL), clear it, and return TRI_ERR_DEVICE_FLAG if any bit was set.
+ */
+tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_H */

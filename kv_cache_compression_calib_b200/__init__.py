@@ -1,0 +1,144 @@
+"""B200-native TriAttention KV-cache key scoring, top-B selection and compaction.
+
+A thin binding over ``libtri.so`` (C ABI in ``include/tri.h``): the functions
+below only marshal torch tensors into pointers and sizes; every step of the
+computation runs in the library's sm_100a CUDA kernels.  Importing the package
+fails if the library has not been built (``build.py``) - there is no other
+implementation to fall back to.
+
+Method: "TriAttention：基于三角函数 KV 压缩的高效长推理" (whatsmy.fun paper
+digest), section 流程详解 steps 1-4 - calibrate pre-RoPE query centres, score
+each cached key by a trigonometric series in its RoPE distance plus a norm
+term, keep the top keys per KV head, compact the cache.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import (TRI_FLAG_BLOCK_TABLE, TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS,  # noqa: F401
+                   TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
+                   TRI_MAX_OFFSETS, TriKvDesc, TriModel, TriOutDesc)
+
+_L = _abi.load()
+
+
+class TriError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_L.tri_status_str(status).decode()}")
+
+
+def _check(st: int, what: str) -> None:
+    if st != _abi.TRI_OK:
+        raise TriError(st, what)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def version() -> int:
+    return int(_L.tri_version())
+
+
+def library_path() -> str:
+    return _abi.LIB_PATH
+
+
+# ------------------------------------------------------------- descriptors
+
+def model(n_layers: int, n_q_heads: int, n_kv_heads: int, rope_theta: float,
+          head_dim: int = 128) -> TriModel:
+    return TriModel(head_dim, n_layers, n_q_heads, n_kv_heads, float(rope_theta))
+
+
+# A descriptor holds raw device pointers; it also keeps a reference to the tensors
+# they point into, so the memory cannot be freed (and reused) while it is alive.
+
+def kv_contig(n_seqs: int, row_off: torch.Tensor, total_keys: int) -> TriKvDesc:
+    """Rows laid end to end; ``row_off`` int64 [R+1] on the device."""
+    d = TriKvDesc(TRI_KV_CONTIG, n_seqs, int(total_keys), row_off.data_ptr(), None, 0, 0, 0)
+    d._keep = (row_off,)
+    return d
+
+
+def kv_paged(n_seqs: int, row_off: torch.Tensor, total_keys: int, block_table: torch.Tensor,
+             block_size: int, n_blocks: int) -> TriKvDesc:
+    """vLLM block layout; ``block_table`` int32 [S][max_blocks] on the device."""
+    d = TriKvDesc(TRI_KV_PAGED, n_seqs, int(total_keys), row_off.data_ptr(),
+                  block_table.data_ptr(), block_table.shape[1], block_size, int(n_blocks))
+    d._keep = (row_off, block_table)
+    return d
+
+
+def out_contig() -> TriOutDesc:
+    return TriOutDesc(TRI_KV_CONTIG, 0, None, 0, 0, 0)
+
+
+def out_paged(block_table: torch.Tensor, block_size: int, n_blocks: int) -> TriOutDesc:
+    d = TriOutDesc(TRI_KV_PAGED, block_table.shape[1], block_table.data_ptr(), block_size, 0,
+                   int(n_blocks))
+    d._keep = (block_table,)
+    return d
+
+
+# ------------------------------------------------------------------- calls
+
+def tri_workspace_size(m: TriModel, n_seqs: int, B: int) -> int:
+    return int(_L.tri_workspace_size(ctypes.byref(m), n_seqs, B))
+
+
+def tri_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(_L.tri_workspace_init(_p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "tri_workspace_init")
+
+
+def alloc_workspace(m: TriModel, n_seqs: int, B: int, device=None, stream=None) -> torch.Tensor:
+    """Allocate (through torch) and initialise a workspace for ``tri_score``/``tri_compact``."""
+    n = tri_workspace_size(m, n_seqs, B)
+    if n == 0:
+        raise TriError(_abi.TRI_ERR_INVALID_ARG, "tri_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    tri_workspace_init(ws, stream)
+    return ws
+
+
+def tri_calib(m: TriModel, qpre: torch.Tensor, nq: int, centres: torch.Tensor,
+              mean_norm: torch.Tensor, stream=None) -> None:
+    _check(_L.tri_calib(ctypes.byref(m), _p(qpre), int(nq), _p(centres), _p(mean_norm), _s(stream)),
+           "tri_calib")
+
+
+def tri_score(m: TriModel, kv: TriKvDesc, K: torch.Tensor, pos, centres: torch.Tensor,
+              mean_norm: torch.Tensor, p_now: torch.Tensor, offsets, key_mode: int,
+              scores: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    offs = (ctypes.c_int32 * max(len(offsets), 1))(*[int(o) for o in offsets])
+    _check(_L.tri_score(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(pos), _p(centres),
+                        _p(mean_norm), _p(p_now), offs, len(offsets), int(key_mode), _p(scores),
+                        _p(ws), ws.numel() * ws.element_size(), _s(stream)), "tri_score")
+
+
+def tri_compact(m: TriModel, kv: TriKvDesc, scores: torch.Tensor, B: int, W: int,
+                K: torch.Tensor, V: torch.Tensor, pos, out: TriOutDesc, K_out: torch.Tensor,
+                V_out: torch.Tensor, pos_out, kept_idx, kept_count, ws: torch.Tensor,
+                stream=None) -> None:
+    _check(_L.tri_compact(ctypes.byref(m), ctypes.byref(kv), _p(scores), int(B), int(W), _p(K),
+                          _p(V), _p(pos), ctypes.byref(out), _p(K_out), _p(V_out), _p(pos_out),
+                          _p(kept_idx), _p(kept_count), _p(ws), ws.numel() * ws.element_size(),
+                          _s(stream)), "tri_compact")
+
+
+def tri_status_check(ws: torch.Tensor, stream=None):
+    """Synchronise, read and clear the device flag word.  Returns (status, flags)."""
+    flags = ctypes.c_uint32(0)
+    st = _L.tri_status_check(_p(ws), ctypes.byref(flags), _s(stream))
+    return st, int(flags.value)

@@ -1,0 +1,254 @@
+// extern "C" entry points of libtri.so: argument checks, workspace carving and
+// kernel dispatch.  See include/tri.h for the contract of every call.
+#include <cmath>
+#include <cstring>
+
+#include "tri_internal.cuh"
+
+namespace tri {
+
+int sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int &c = cache[dev & 63];
+    if (c == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 1;
+        c = v;
+    }
+    return c;
+}
+
+}  // namespace tri
+
+using namespace tri;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int pow2_shift(int32_t x) {
+    if (x < 1 || x > 1024 || (x & (x - 1))) return -1;
+    int s = 0;
+    while ((1 << s) != x) s++;
+    return s;
+}
+
+tri_status check_model(const tri_model *m) {
+    if (!m) return TRI_ERR_INVALID_ARG;
+    if (m->head_dim != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+    if (m->n_layers < 1 || m->n_q_heads < 1 || m->n_kv_heads < 1) return TRI_ERR_INVALID_ARG;
+    if (m->n_q_heads % m->n_kv_heads) return TRI_ERR_INVALID_ARG;
+    if (!std::isfinite(m->rope_theta) || !(m->rope_theta > 1.0)) return TRI_ERR_INVALID_ARG;
+    return TRI_OK;
+}
+
+int64_t rows_of(const tri_model *m, int32_t S) { return (int64_t)m->n_layers * S * m->n_kv_heads; }
+
+tri_status check_kv(const tri_model *m, const tri_kv_desc *kv, Geometry *geo) {
+    if (!kv || !kv->row_off || kv->n_seqs < 1 || kv->total_keys < 0) return TRI_ERR_INVALID_ARG;
+    if (!aligned(kv->row_off, 8)) return TRI_ERR_ALIGNMENT;
+    const int64_t R = rows_of(m, kv->n_seqs);
+    if (R > 0x7fffffffLL || kv->total_keys > (1LL << 56)) return TRI_ERR_UNSUPPORTED;
+    std::memset(geo, 0, sizeof(*geo));
+    geo->L = m->n_layers;
+    geo->S = kv->n_seqs;
+    geo->H = m->n_kv_heads;
+    geo->Hq = m->n_q_heads;
+    geo->G = m->n_q_heads / m->n_kv_heads;
+    geo->layout = kv->layout;
+    geo->total = kv->total_keys;
+    geo->row_off = kv->row_off;
+    if (kv->layout == TRI_KV_PAGED) {
+        if (!kv->block_table || kv->max_blocks < 1 || kv->n_blocks < 1) return TRI_ERR_INVALID_ARG;
+        if (!aligned(kv->block_table, 4)) return TRI_ERR_ALIGNMENT;
+        const int sh = pow2_shift(kv->block_size);
+        if (sh < 0) return TRI_ERR_UNSUPPORTED;
+        geo->block_table = kv->block_table;
+        geo->max_blocks = kv->max_blocks;
+        geo->block_shift = sh;
+        geo->n_blocks = kv->n_blocks;
+    } else if (kv->layout != TRI_KV_CONTIG) {
+        return TRI_ERR_INVALID_ARG;
+    }
+    return TRI_OK;
+}
+
+tri_status check_ws(const void *ws, size_t have, size_t need) {
+    if (!ws) return TRI_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return TRI_ERR_ALIGNMENT;
+    if (have < need) return TRI_ERR_WORKSPACE_TOO_SMALL;
+    return TRI_OK;
+}
+
+tri_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRI_OK : TRI_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *tri_status_str(tri_status s) {
+    switch (s) {
+        case TRI_OK: return "TRI_OK";
+        case TRI_ERR_INVALID_ARG: return "TRI_ERR_INVALID_ARG";
+        case TRI_ERR_UNSUPPORTED: return "TRI_ERR_UNSUPPORTED";
+        case TRI_ERR_ALIGNMENT: return "TRI_ERR_ALIGNMENT";
+        case TRI_ERR_WORKSPACE_TOO_SMALL: return "TRI_ERR_WORKSPACE_TOO_SMALL";
+        case TRI_ERR_CUDA: return "TRI_ERR_CUDA";
+        case TRI_ERR_DEVICE_FLAG: return "TRI_ERR_DEVICE_FLAG";
+    }
+    return "TRI_ERR_UNKNOWN";
+}
+
+uint32_t tri_version(void) { return (0u << 16) | 1u; }
+
+size_t tri_workspace_size(const tri_model *m, int32_t n_seqs, int32_t B) {
+    if (check_model(m) != TRI_OK || n_seqs < 1 || B < 1) return 0;
+    return ws_total(rows_of(m, n_seqs), B);
+}
+
+tri_status tri_workspace_init(void *ws, size_t ws_bytes, tri_stream_t stream) {
+    tri_status st = check_ws(ws, ws_bytes, 256);
+    if (st != TRI_OK) return st;
+    return cuda_status(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
+}
+
+tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *centres, float *mean_norm,
+                     tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    if (!qpre || !centres || !mean_norm || nq < 1) return TRI_ERR_INVALID_ARG;
+    if (!aligned(qpre, 16) || !aligned(centres, 4) || !aligned(mean_norm, 4)) return TRI_ERR_ALIGNMENT;
+    const int64_t heads = (int64_t)m->n_layers * m->n_q_heads;
+    if (heads > 0x7fffffffLL) return TRI_ERR_UNSUPPORTED;
+    CalibParams p;
+    p.q = (const uint16_t *)qpre;
+    p.nq = nq;
+    p.n_heads = (int32_t)heads;
+    p.centres = centres;
+    p.mean_norm = mean_norm;
+    return cuda_status(launch_calib(p, (cudaStream_t)stream));
+}
+
+tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, const int32_t *pos,
+                     const float *centres, const float *mean_norm, const int64_t *p_now,
+                     const int32_t *offsets, int32_t n_offsets, int32_t key_mode, float *scores, void *ws,
+                     size_t ws_bytes, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    Geometry geo;
+    if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
+    if (!K || !centres || !mean_norm || !p_now || !offsets || !scores) return TRI_ERR_INVALID_ARG;
+    if (n_offsets < 1 || n_offsets > TRI_MAX_OFFSETS) return TRI_ERR_INVALID_ARG;
+    if (key_mode != TRI_KEYS_POST_ROPE && key_mode != TRI_KEYS_PRE_ROPE) return TRI_ERR_INVALID_ARG;
+    if (key_mode == TRI_KEYS_PRE_ROPE && !pos) return TRI_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(scores, 4) || !aligned(centres, 4) || !aligned(mean_norm, 4) ||
+        !aligned(p_now, 8) || (pos && !aligned(pos, 4)))
+        return TRI_ERR_ALIGNMENT;
+    const int64_t R = rows_of(m, kv->n_seqs);
+    if ((st = check_ws(ws, ws_bytes, ws_idx_offset(R))) != TRI_OK) return st;
+    char *w = (char *)ws;
+    cudaStream_t s = (cudaStream_t)stream;
+
+    PrepParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.geo = geo;
+    pp.centres = centres;
+    pp.mean_norm = mean_norm;
+    pp.p_now = p_now;
+    pp.theta = m->rope_theta;
+    pp.n_off = n_offsets;
+    pp.pre_rope = key_mode == TRI_KEYS_PRE_ROPE;
+    for (int i = 0; i < n_offsets; i++) pp.offsets[i] = offsets[i];
+    pp.coef = (float *)(w + kWsCoef);
+    pp.turns = (unsigned long long *)(w + kWsTurns);
+    pp.flags = (unsigned *)(w + kWsFlags);
+    if ((st = cuda_status(launch_prep(pp, s))) != TRI_OK) return st;
+
+    ScoreParams sp;
+    sp.geo = geo;
+    sp.K = (const uint16_t *)K;
+    sp.pos = pos;
+    sp.p_now = p_now;
+    sp.coef = pp.coef;
+    sp.turns = pp.turns;
+    sp.scores = scores;
+    sp.flags = pp.flags;
+    return cuda_status(launch_score(sp, pp.pre_rope, s));
+}
+
+tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *scores, int32_t B, int32_t W,
+                       const void *K, const void *V, const int32_t *pos, const tri_out_desc *out, void *K_out,
+                       void *V_out, int32_t *pos_out, int32_t *kept_idx, int32_t *kept_count, void *ws,
+                       size_t ws_bytes, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    Geometry geo;
+    if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
+    if (B < 1 || W < 0 || W > B) return TRI_ERR_INVALID_ARG;
+    if (!scores || !K || !V || !out || !K_out || !V_out) return TRI_ERR_INVALID_ARG;
+    if (pos_out && !pos) return TRI_ERR_INVALID_ARG;
+    if (K_out == K || V_out == V || K_out == V || V_out == K) return TRI_ERR_INVALID_ARG;
+    if (!aligned(scores, 4) || !aligned(K, 16) || !aligned(V, 16) || !aligned(K_out, 16) || !aligned(V_out, 16) ||
+        (pos && !aligned(pos, 4)) || (pos_out && !aligned(pos_out, 4)) || (kept_idx && !aligned(kept_idx, 4)) ||
+        (kept_count && !aligned(kept_count, 4)))
+        return TRI_ERR_ALIGNMENT;
+    int out_shift = 0;
+    if (out->layout == TRI_KV_PAGED) {
+        if (!out->block_table || out->max_blocks < 1 || out->n_blocks < 1) return TRI_ERR_INVALID_ARG;
+        if (!aligned(out->block_table, 4)) return TRI_ERR_ALIGNMENT;
+        out_shift = pow2_shift(out->block_size);
+        if (out_shift < 0) return TRI_ERR_UNSUPPORTED;
+    } else if (out->layout != TRI_KV_CONTIG) {
+        return TRI_ERR_INVALID_ARG;
+    }
+    const int64_t R = rows_of(m, kv->n_seqs);
+    if ((st = check_ws(ws, ws_bytes, kept_idx ? 256 : ws_total(R, B))) != TRI_OK) return st;
+    char *w = (char *)ws;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t *kept = kept_idx ? kept_idx : (int32_t *)(w + ws_idx_offset(R));
+
+    SelectParams sp;
+    sp.geo = geo;
+    sp.scores = scores;
+    sp.B = B;
+    sp.W = W;
+    sp.kept = kept;
+    sp.kept_count = kept_count;
+    sp.flags = (unsigned *)(w + kWsFlags);
+    if ((st = cuda_status(launch_select(sp, s))) != TRI_OK) return st;
+
+    GatherParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    gp.geo = geo;
+    gp.out_layout = out->layout;
+    gp.out_max_blocks = out->max_blocks;
+    gp.out_block_shift = out_shift;
+    gp.out_n_blocks = out->n_blocks;
+    gp.out_table = out->block_table;
+    gp.B = B;
+    gp.kept = kept;
+    gp.K = (const uint16_t *)K;
+    gp.V = (const uint16_t *)V;
+    gp.pos = pos_out ? pos : nullptr;
+    gp.K_out = (uint16_t *)K_out;
+    gp.V_out = (uint16_t *)V_out;
+    gp.pos_out = pos_out;
+    gp.flags = sp.flags;
+    return cuda_status(launch_gather(gp, s));
+}
+
+tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream) {
+    tri_status st = check_ws(ws, 256, 256);
+    if (st != TRI_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t host = 0;
+    if (cudaMemcpyAsync(&host, ws, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return TRI_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TRI_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(host), s) != cudaSuccess) return TRI_ERR_CUDA;
+    if (flags) *flags = host;
+    return host ? TRI_ERR_DEVICE_FLAG : TRI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// Stable compaction: copy K, V (and pos) of every kept slot, in ascending slot
+// order, into the output cache ("TriAttention：基于三角函数 KV 压缩的高效长推理",
+// 流程详解 step 4: later attention reads only the compressed cache).
+//
+// Flat grid over (row, 64-slot chunk).  A half-warp moves one 256-byte key
+// record as 16 x 16-byte vectors, so each warp instruction copies two whole
+// records; every thread keeps 4 K and 4 V vectors in flight.  Source reads
+// bypass L1; destination writes are streaming stores (not re-read here).
+// Paged input and/or output addresses go through the block tables.
+#include "tri_internal.cuh"
+
+namespace tri {
+
+constexpr int kGatherThreads = 256;
+constexpr int kSlotsPerCta = 64;  // 8 warps x 4 iterations x 2 records
+
+__global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherParams p) {
+    const Geometry &geo = p.geo;
+    const int64_t chunks = (p.B + kSlotsPerCta - 1) / kSlotsPerCta;
+    const int64_t r = blockIdx.x / chunks;
+    const int base = (int)(blockIdx.x % chunks) * kSlotsPerCta;
+    const int64_t row_lo = geo.row_off[r];
+    const int64_t N = geo.row_off[r + 1] - row_lo;
+    if (N < 0 || N > 0x7fffffffLL || row_lo < 0 || row_lo + N > geo.total) return;  // flagged by the selection
+    const int cnt = (int)min(N, (int64_t)p.B);
+    if (base >= cnt) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = lane >> 4, c = lane & 15;
+    const int h = (int)(r % geo.H);
+    const int s = (int)((r / geo.H) % geo.S);
+    const int l = (int)(r / ((int64_t)geo.H * geo.S));
+
+    uint4 kv[4], vv[4];
+    int64_t dst[4];
+    int32_t pv[4];
+#pragma unroll
+    for (int it = 0; it < 4; it++) {
+        const int i = base + warp * 8 + it * 2 + half;
+        dst[it] = -1;
+        pv[it] = 0;
+        if (i >= cnt) continue;
+        const int64_t j = p.kept[r * p.B + i];
+        int64_t src = -1;
+        if (j >= 0 && j < N) {
+            if (geo.layout == TRI_KV_PAGED) {
+                const int64_t bi = j >> geo.block_shift;
+                const int32_t blk = bi < geo.max_blocks ? __ldg(geo.block_table + (int64_t)s * geo.max_blocks + bi) : -1;
+                if (blk >= 0 && blk < geo.n_blocks)
+                    src = ((((int64_t)l * geo.n_blocks + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) * geo.H + h;
+            } else {
+                src = row_lo + j;
+            }
+        }
+        int64_t d = -1;
+        if (p.out_layout == TRI_KV_PAGED) {
+            const int64_t bi = (int64_t)i >> p.out_block_shift;
+            const int32_t blk = bi < p.out_max_blocks ? __ldg(p.out_table + (int64_t)s * p.out_max_blocks + bi) : -1;
+            if (blk >= 0 && blk < p.out_n_blocks)
+                d = ((((int64_t)l * p.out_n_blocks + blk) << p.out_block_shift) | (i & ((1 << p.out_block_shift) - 1))) * geo.H + h;
+        } else {
+            d = r * p.B + i;
+        }
+        if (src < 0 || d < 0) {
+            if (c == 0) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
+            continue;
+        }
+        dst[it] = d;
+        kv[it] = ld_nc16(p.K + src * kD + 8 * c);
+        vv[it] = ld_nc16(p.V + src * kD + 8 * c);
+        if (p.pos && c == 0) pv[it] = __ldg(p.pos + src);
+    }
+#pragma unroll
+    for (int it = 0; it < 4; it++) {
+        if (dst[it] < 0) continue;
+        st_stream16(p.K_out + dst[it] * kD + 8 * c, kv[it]);
+        st_stream16(p.V_out + dst[it] * kD + 8 * c, vv[it]);
+        if (p.pos_out && c == 0) p.pos_out[dst[it]] = pv[it];
+    }
+}
+
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t s) {
+    const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
+    if (R <= 0) return cudaSuccess;
+    const int64_t chunks = (p.B + kSlotsPerCta - 1) / kSlotsPerCta;
+    const int64_t grid = R * chunks;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    gather_kernel<<<(unsigned)grid, kGatherThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace tri

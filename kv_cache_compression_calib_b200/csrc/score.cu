@@ -1,0 +1,346 @@
+// Key scoring ("TriAttention：基于三角函数 KV 压缩的高效长推理", 流程详解 steps 2-3;
+// "WeianMao/triattention", How it works).
+//
+// For the row of KV head h the score of a cached key is
+//   S_j = (1/G) sum_g sum_f [ |qbar_f^g||k_f| sum_delta cos(w_f (p_now + delta - j) + phi_f^g)
+//                             + (E|q_f^g| - |qbar_f^g|) |k_f| ].
+// With q.conj(k) written as complex pairs, each cosine term is
+// Re(qbar_f conj(k_f^pre) e^{i w_f (p_now + delta - j)}), and a RoPE cache holds
+// k_f^post = k_f^pre e^{i w_f j}, so the key's own rotation cancels the -j:
+//   S_j = sum_f Re(A_f conj(k_f^post)) + c_f |k_f|,
+//   A_f = (1/G) sum_g qbar_f^g * e^{i w_f p_now} * sum_delta e^{i w_f delta},
+//   c_f = (1/G) sum_g (E|q_f^g| - |qbar_f^g|).
+// The delta sum collapses by angle addition into one complex constant per f,
+// and the GQA mean into A_f (the score is linear in the per-head terms).  The
+// per-key work is then a 64-pair dot product plus 64 magnitudes: 256 B of
+// bf16 read per key, ~6 FP32 ops per pair - bound by HBM, not arithmetic, so
+// no tensor cores (no dense contraction here).
+//
+// For a cache of pre-RoPE keys, the literal one-(sin, cos)-per-(key, pair)
+// form is used instead: A'_f = (1/G) sum_g qbar_f^g sum_delta e^{i w_f delta}
+// and S_j = sum_f Re(A'_f e^{i w_f (p_now - j)} conj(k_f)) + c_f |k_f|, with the
+// phase w_f (p_now - j) reduced exactly as a 64-bit fixed-point fraction of a
+// turn (integer multiply mod 2^64), so fp32 never holds a large angle.
+//
+// prep_kernel forms A_f, c_f per row in fp64 and stores fp32.  score_kernel
+// streams the keys: each warp owns a contiguous span of the concatenated key
+// space (all rows end to end, so ragged rows balance across the whole grid);
+// per batch of 32 keys, lane (q, g) loads the 16-byte real and imaginary
+// halves of pairs 8g..8g+7 for keys 4u+q, u = 0..7 (two full 128-byte lines
+// per key per instruction), accumulates 8 pairs in fp32, and a butterfly
+// reduce-scatter over the 8 lanes of a key leaves lane i holding key i's
+// score for one coalesced 128-byte store.
+#include "tri_internal.cuh"
+
+namespace tri {
+
+constexpr int kPrepThreads = 64;
+constexpr int kScoreThreads = 256;
+constexpr double kTurnScale = 2.9358905032820014e+18;  // 2^64 / (2 pi)
+constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
+
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) {
+    const Geometry &geo = p.geo;
+    const int r = blockIdx.x;
+    const int f = threadIdx.x;
+    const int h = r % geo.H;
+    const int s = (r / geo.H) % geo.S;
+    const int l = r / (geo.H * geo.S);
+    const double w = pow(p.theta, -2.0 * (double)f / (double)kD);
+    double sr = 0.0, si = 0.0;
+    for (int e = 0; e < p.n_off; e++) {
+        double sn, cs;
+        sincos(w * (double)p.offsets[e], &sn, &cs);
+        sr += cs;
+        si += sn;
+    }
+    double mr = 0.0, mi = 0.0, cf = 0.0;
+    for (int g = 0; g < geo.G; g++) {
+        const int64_t qh = (int64_t)l * geo.Hq + (int64_t)h * geo.G + g;
+        const double qr = p.centres[(qh * kF + f) * 2];
+        const double qi = p.centres[(qh * kF + f) * 2 + 1];
+        mr += qr;
+        mi += qi;
+        cf += (double)p.mean_norm[qh * kF + f] - hypot(qr, qi);
+    }
+    mr /= (double)geo.G;
+    mi /= (double)geo.G;
+    cf /= (double)geo.G;
+    const double tr = mr * sr - mi * si, ti = mr * si + mi * sr;
+    double ar = tr, ai = ti;
+    if (!p.pre_rope) {
+        double sn, cs;
+        sincos(w * (double)p.p_now[s], &sn, &cs);
+        ar = tr * cs - ti * sn;
+        ai = tr * sn + ti * cs;
+    }
+    float *c = p.coef + (int64_t)r * kCoefPerRow + (f >> 3) * kCoefPerGroup;
+    c[f & 7] = (float)ar;
+    c[8 + (f & 7)] = (float)ai;
+    c[16 + (f & 7)] = (float)cf;
+    if (r == 0) {
+        p.turns[f] = __double2ull_rn(w * kTurnScale);
+        if (f == 0) {
+            const int64_t R = (int64_t)geo.L * geo.S * geo.H;
+            if (geo.row_off[0] != 0 || geo.row_off[R] != geo.total) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
+        }
+    }
+}
+
+struct RowCtx {
+    int r;
+    int64_t lo, hi;
+    // paged addressing
+    const int32_t *table;
+    int64_t layer_blk;  // l * n_blocks
+    int h;
+    int64_t p_now;
+    float ar[8], ai[8], cc[8];
+};
+
+__device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, int g) {
+    const Geometry &geo = p.geo;
+    c.r = r;
+    c.lo = geo.row_off[r];
+    c.hi = geo.row_off[r + 1];
+    const int h = r % geo.H;
+    const int s = (r / geo.H) % geo.S;
+    const int l = r / (geo.H * geo.S);
+    c.h = h;
+    c.table = geo.block_table + (int64_t)s * geo.max_blocks;
+    c.layer_blk = (int64_t)l * geo.n_blocks;
+    c.p_now = p.p_now[s];
+    const float4 *cp = reinterpret_cast<const float4 *>(p.coef + (int64_t)r * kCoefPerRow + g * kCoefPerGroup);
+    const float4 v0 = cp[0], v1 = cp[1], v2 = cp[2], v3 = cp[3], v4 = cp[4], v5 = cp[5];
+    c.ar[0] = v0.x; c.ar[1] = v0.y; c.ar[2] = v0.z; c.ar[3] = v0.w;
+    c.ar[4] = v1.x; c.ar[5] = v1.y; c.ar[6] = v1.z; c.ar[7] = v1.w;
+    c.ai[0] = v2.x; c.ai[1] = v2.y; c.ai[2] = v2.z; c.ai[3] = v2.w;
+    c.ai[4] = v3.x; c.ai[5] = v3.y; c.ai[6] = v3.z; c.ai[7] = v3.w;
+    c.cc[0] = v4.x; c.cc[1] = v4.y; c.cc[2] = v4.z; c.cc[3] = v4.w;
+    c.cc[4] = v5.x; c.cc[5] = v5.y; c.cc[6] = v5.z; c.cc[7] = v5.w;
+}
+
+// Slot index (in units of one (slot, head) record) of global key k in row c,
+// or -1 if the paged table cannot place it.
+template <bool PAGED>
+__device__ __forceinline__ int64_t key_slot(const ScoreParams &p, const RowCtx &c, int64_t k) {
+    if (!PAGED) return k;
+    const Geometry &geo = p.geo;
+    const int64_t j = k - c.lo;
+    const int64_t bi = j >> geo.block_shift;
+    if (j < 0 || bi >= geo.max_blocks) return -1;
+    const int32_t blk = __ldg(c.table + bi);
+    if (blk < 0 || blk >= geo.n_blocks) return -1;
+    return ((((c.layer_blk + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) * geo.H) + c.h;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 v, float (&x)[8]) {
+    x[0] = bf16lo(v.x); x[1] = bf16hi(v.x); x[2] = bf16lo(v.y); x[3] = bf16hi(v.y);
+    x[4] = bf16lo(v.z); x[5] = bf16hi(v.z); x[6] = bf16lo(v.w); x[7] = bf16hi(v.w);
+}
+
+// Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|.
+__device__ __forceinline__ float partial_post(const uint4 re, const uint4 im, const RowCtx &c) {
+    float x[8], y[8];
+    unpack8(re, x);
+    unpack8(im, y);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        a0 = fmaf(c.ar[i], x[i], a0);
+        a1 = fmaf(c.ai[i], y[i], a1);
+        a2 = fmaf(c.cc[i], sqrt_approx(fmaf(x[i], x[i], y[i] * y[i])), a2);
+    }
+    return (a0 + a1) + a2;
+}
+
+// Pre-RoPE cache: rotate A'_i by w_i (p_now - pos) first.  The phase in turns
+// is (delta * T_i) mod 2^64 with T_i = w_i / 2pi in 0.64 fixed point; its top
+// 32 bits as a signed integer are the angle in [-pi, pi).
+__device__ __forceinline__ float partial_pre(const uint4 re, const uint4 im, const RowCtx &c,
+                                             const unsigned long long (&T)[8], int64_t delta) {
+    float x[8], y[8];
+    unpack8(re, x);
+    unpack8(im, y);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const unsigned long long t = (unsigned long long)delta * T[i];
+        const float ang = (float)(int)(t >> 32) * kTurnToRad;
+        float sn, cs;
+        __sincosf(ang, &sn, &cs);
+        const float br = c.ar[i] * cs - c.ai[i] * sn;
+        const float bi = c.ar[i] * sn + c.ai[i] * cs;
+        a0 = fmaf(br, x[i], a0);
+        a1 = fmaf(bi, y[i], a1);
+        a2 = fmaf(c.cc[i], sqrt_approx(fmaf(x[i], x[i], y[i] * y[i])), a2);
+    }
+    return (a0 + a1) + a2;
+}
+
+template <bool PAGED, bool PRE>
+__device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx &c, int64_t k, int g,
+                                             unsigned long long pol, const unsigned long long (&T)[8]) {
+    const int64_t slot = key_slot<PAGED>(p, c, k);
+    if (slot < 0) {
+        atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
+        return 0.f;
+    }
+    const uint16_t *kp = p.K + slot * kD + 8 * g;
+    const uint4 re = ld_stream16(kp, pol);
+    const uint4 im = ld_stream16(kp + kF, pol);
+    if (PRE) return partial_pre(re, im, c, T, c.p_now - (int64_t)__ldg(p.pos + slot));
+    return partial_post(re, im, c);
+}
+
+template <bool PAGED, bool PRE>
+__global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const ScoreParams p) {
+    const Geometry &geo = p.geo;
+    const int lane = threadIdx.x & 31;
+    const int q = lane >> 3;  // key of the 4-key group
+    const int g = lane & 7;   // pairs 8g .. 8g+7
+    const int64_t nwarps = (int64_t)gridDim.x * (kScoreThreads / 32);
+    const int64_t wid = (int64_t)blockIdx.x * (kScoreThreads / 32) + (threadIdx.x >> 5);
+    const int64_t total = geo.total;
+    int64_t per = (total + nwarps - 1) / nwarps;
+    per = (per + 31) & ~int64_t(31);
+    const int64_t beg = wid * per;
+    const int64_t end = min(total, beg + per);
+    if (beg >= end) return;
+    const int R = geo.L * geo.S * geo.H;
+
+    unsigned long long T[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * g + i] : 0ull;
+    const unsigned long long pol = policy_evict_first();
+
+    // Row holding key `beg`: the last r with row_off[r] <= beg.
+    int rl = 0, rh = R;
+    while (rh - rl > 1) {
+        const int mid = (rl + rh) >> 1;
+        if (geo.row_off[mid] <= beg) rl = mid;
+        else rh = mid;
+    }
+    int r0 = rl;
+    while (r0 < R - 1 && geo.row_off[r0 + 1] <= beg) r0++;
+    RowCtx c;
+    set_row(c, p, r0, g);
+
+    for (int64_t b0 = beg; b0 < end; b0 += 32) {
+        const int64_t bend = min(b0 + 32, end);
+        float part[8];
+        if (bend == b0 + 32 && b0 >= c.lo && bend <= c.hi) {
+            // Whole batch inside the current row: issue all 16 loads, then compute.
+            uint4 re[8], im[8];
+            int64_t slot[8];
+            int32_t kpos[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                slot[u] = key_slot<PAGED>(p, c, b0 + 4 * u + q);
+                if (slot[u] >= 0) {
+                    const uint16_t *kp = p.K + slot[u] * kD + 8 * g;
+                    re[u] = ld_stream16(kp, pol);
+                    im[u] = ld_stream16(kp + kF, pol);
+                    kpos[u] = PRE ? __ldg(p.pos + slot[u]) : 0;
+                } else {
+                    re[u] = make_uint4(0, 0, 0, 0);
+                    im[u] = re[u];
+                    kpos[u] = 0;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                if (PAGED && slot[u] < 0) {
+                    atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
+                    part[u] = 0.f;
+                } else if (PRE) {
+                    part[u] = partial_pre(re[u], im[u], c, T, c.p_now - (int64_t)kpos[u]);
+                } else {
+                    part[u] = partial_post(re[u], im[u], c);
+                }
+            }
+        } else {
+            // Batch crosses a row boundary or the span end: one segment per row.
+#pragma unroll
+            for (int u = 0; u < 8; u++) part[u] = 0.f;
+            int64_t k0 = b0;
+            for (;;) {
+                const int64_t seg_end = min(bend, c.hi);
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    const int64_t k = b0 + 4 * u + q;
+                    if (k >= k0 && k < seg_end) part[u] += key_partial<PAGED, PRE>(p, c, k, g, pol, T);
+                }
+                if (bend <= c.hi) break;
+                k0 = max(k0, c.hi);
+                int r = c.r + 1;
+                while (r < R && geo.row_off[r + 1] <= k0) r++;
+                if (r >= R) {
+                    atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
+                    break;
+                }
+                set_row(c, p, r, g);
+                if (c.lo != k0) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
+            }
+        }
+        // Butterfly reduce-scatter over the 8 lanes (bits of g) sharing a key:
+        // afterwards lane (q, g) holds the full score of key 4g + q.
+        {
+            const bool h2 = (g >> 2) & 1;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float send = h2 ? part[i] : part[i + 4];
+                const float keep = h2 ? part[i + 4] : part[i];
+                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+            }
+            const bool h1 = (g >> 1) & 1;
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+                const float send = h1 ? part[i] : part[i + 2];
+                const float keep = h1 ? part[i + 2] : part[i];
+                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            }
+            const bool h0 = g & 1;
+            const float send = h0 ? part[0] : part[1];
+            const float keep = h0 ? part[1] : part[0];
+            part[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+        }
+        const float v = __shfl_sync(0xffffffffu, part[0], 8 * (lane & 3) + (lane >> 2));
+        if (b0 + lane < bend) p.scores[b0 + lane] = v;
+    }
+}
+
+cudaError_t launch_prep(const PrepParams &p, cudaStream_t s) {
+    const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
+    if (R <= 0) return cudaSuccess;
+    prep_kernel<<<(unsigned)R, kPrepThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool PAGED, bool PRE>
+static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
+    static int occ[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int &o = occ[dev & 63];
+    if (o == 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_kernel<PAGED, PRE>, kScoreThreads, 0);
+        if (e != cudaSuccess) return e;
+        if (o < 1) o = 1;
+    }
+    const int64_t want = (p.geo.total + 32 * (kScoreThreads / 32) - 1) / (32 * (kScoreThreads / 32));
+    int64_t grid = (int64_t)sm_count() * o;
+    if (want < grid) grid = want;
+    if (grid < 1) grid = 1;
+    score_kernel<PAGED, PRE><<<(unsigned)grid, kScoreThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s) {
+    if (p.geo.total <= 0) return cudaSuccess;
+    const bool paged = p.geo.layout == TRI_KV_PAGED;
+    if (paged) return pre_rope ? launch_score_t<true, true>(p, s) : launch_score_t<true, false>(p, s);
+    return pre_rope ? launch_score_t<false, true>(p, s) : launch_score_t<false, false>(p, s);
+}
+
+}  // namespace tri

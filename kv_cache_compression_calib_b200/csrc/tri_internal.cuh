@@ -1,0 +1,150 @@
+// Internal launch interface and device helpers of libtri.so (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tri.h"
+
+namespace tri {
+
+constexpr int kD = TRI_HEAD_DIM;  // head dim
+constexpr int kF = kD / 2;        // frequency pairs
+constexpr int kCoefPerGroup = 24; // 8 pairs x (Re A, Im A, c)
+constexpr int kCoefPerRow = 8 * kCoefPerGroup;
+
+// Workspace layout (byte offsets from the 256-byte aligned base).
+constexpr size_t kWsFlags = 0;       // uint32 flag word
+constexpr size_t kWsTurns = 256;     // uint64 [64]: w_f / 2pi in 0.64 fixed point
+constexpr size_t kWsCoef = 1024;     // float [R][8][24]
+inline size_t ws_coef_bytes(int64_t R) { return ((size_t)R * kCoefPerRow * 4 + 255) & ~size_t(255); }
+inline size_t ws_idx_offset(int64_t R) { return kWsCoef + ws_coef_bytes(R); }
+inline size_t ws_total(int64_t R, int64_t B) {
+    return ws_idx_offset(R) + (((size_t)R * (size_t)B * 4 + 255) & ~size_t(255));
+}
+
+struct Geometry {  // row numbering and cache addressing
+    int32_t L, S, H, Hq, G;
+    int32_t layout;
+    int32_t max_blocks, block_shift;  // paged: block_size = 1 << block_shift
+    int64_t n_blocks;
+    int64_t total;
+    const int64_t *row_off;
+    const int32_t *block_table;
+};
+
+struct PrepParams {
+    Geometry geo;
+    const float *centres;
+    const float *mean_norm;
+    const int64_t *p_now;
+    double theta;
+    int32_t n_off;
+    int32_t pre_rope;
+    int32_t offsets[TRI_MAX_OFFSETS];
+    float *coef;
+    unsigned long long *turns;
+    unsigned *flags;
+};
+
+struct ScoreParams {
+    Geometry geo;
+    const uint16_t *K;
+    const int32_t *pos;
+    const int64_t *p_now;
+    const float *coef;
+    const unsigned long long *turns;
+    float *scores;
+    unsigned *flags;
+};
+
+struct SelectParams {
+    Geometry geo;
+    const float *scores;
+    int32_t B, W;
+    int32_t *kept;        // [R][B]
+    int32_t *kept_count;  // [R] or null
+    unsigned *flags;
+};
+
+struct GatherParams {
+    Geometry geo;
+    // output paging (layout TRI_KV_PAGED) or contiguous [R][B]
+    int32_t out_layout, out_max_blocks, out_block_shift;
+    int64_t out_n_blocks;
+    const int32_t *out_table;
+    int32_t B;
+    const int32_t *kept;
+    const uint16_t *K, *V;
+    const int32_t *pos;
+    uint16_t *K_out, *V_out;
+    int32_t *pos_out;
+    unsigned *flags;
+};
+
+struct CalibParams {
+    const uint16_t *q;
+    int64_t nq;
+    int32_t n_heads;  // L * Hq
+    float *centres, *mean_norm;
+};
+
+cudaError_t launch_calib(const CalibParams &p, cudaStream_t s);
+cudaError_t launch_prep(const PrepParams &p, cudaStream_t s);
+cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s);
+cudaError_t launch_select(const SelectParams &p, cudaStream_t s);
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t s);
+
+int sm_count();  // SMs of the current device (cached per device)
+
+// ------------------------------------------------------------ device helpers
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// L2 policy that marks lines for early eviction: streamed-once data.
+__device__ __forceinline__ unsigned long long policy_evict_first() {
+    unsigned long long pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 16-byte read-only load that bypasses L1 and carries an L2 eviction policy.
+__device__ __forceinline__ uint4 ld_stream16(const void *ptr, unsigned long long pol) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ld_nc16(const void *ptr) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream16(void *ptr, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Order-preserving map of fp32 scores to uint32: larger score -> larger key.
+// -0 is folded onto +0 (they compare equal); NaN maps to 0, below -inf.
+__device__ __forceinline__ uint32_t order_key(float s) {
+    uint32_t u = __float_as_uint(s);
+    if (s != s) return 0u;
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+}  // namespace tri

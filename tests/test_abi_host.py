@@ -1,0 +1,141 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/tri.h declares, and rejects bad arguments on the host before any
+CUDA call (these calls never reach the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kv_cache_compression_calib_b200 as tri
+from kv_cache_compression_calib_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tri.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tri_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    names = header_functions()
+    assert names == sorted(_abi.EXPORTS)
+    assert {"tri_calib", "tri_score", "tri_compact"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(tri.library_path())
+    for name in header_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version():
+    L = _abi.load()
+    for code, name in [(0, "TRI_OK"), (1, "TRI_ERR_INVALID_ARG"), (2, "TRI_ERR_UNSUPPORTED"),
+                       (3, "TRI_ERR_ALIGNMENT"), (4, "TRI_ERR_WORKSPACE_TOO_SMALL"),
+                       (5, "TRI_ERR_CUDA"), (6, "TRI_ERR_DEVICE_FLAG")]:
+        assert L.tri_status_str(code).decode() == name
+    assert tri.version() >= 1
+
+
+def test_workspace_size():
+    m = tri.model(36, 32, 8, 1e6)
+    n = tri.tri_workspace_size(m, 1, 2048)
+    R = 36 * 8
+    assert n >= R * 768 + R * 2048 * 4 and n % 256 == 0
+    assert tri.tri_workspace_size(m, 0, 2048) == 0
+    assert tri.tri_workspace_size(m, 1, 0) == 0
+    assert tri.tri_workspace_size(tri.model(1, 32, 8, 1e6, head_dim=64), 1, 16) == 0
+
+
+# Fake (never dereferenced) device addresses: the host checks run first.
+A = 1 << 20  # 1 MiB: aligned for every check
+
+
+def _kv(layout=0, n_seqs=1, total=4096, row_off=A, table=None, max_blocks=0, bs=0, nb=0):
+    return _abi.TriKvDesc(layout, n_seqs, total, row_off, table, max_blocks, bs, nb)
+
+
+def _score(m, kv, K=A, pos=None, c=A, mn=A, pnow=A, offs=(1, 2, 4), mode=0, scores=A, ws=A,
+           ws_bytes=1 << 30):
+    L = _abi.load()
+    arr = (ctypes.c_int32 * max(len(offs), 1))(*offs)
+    return L.tri_score(ctypes.byref(m), ctypes.byref(kv) if kv is not None else None, K, pos, c, mn,
+                       pnow, arr, len(offs), mode, scores, ws, ws_bytes, None)
+
+
+def _compact(m, kv, B=64, W=8, scores=A, K=A, V=2 * A, pos=None, out=None, Ko=3 * A, Vo=4 * A,
+             poso=None, kept=None, cnt=None, ws=A, ws_bytes=1 << 30):
+    L = _abi.load()
+    out = out or _abi.TriOutDesc(0, 0, None, 0, 0, 0)
+    return L.tri_compact(ctypes.byref(m), ctypes.byref(kv), scores, B, W, K, V, pos, ctypes.byref(out),
+                         Ko, Vo, poso, kept, cnt, ws, ws_bytes, None)
+
+
+M = tri.model(1, 32, 8, 1e6)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(K=None), _abi.TRI_ERR_INVALID_ARG),
+    (dict(scores=None), _abi.TRI_ERR_INVALID_ARG),
+    (dict(offs=()), _abi.TRI_ERR_INVALID_ARG),
+    (dict(offs=tuple(range(65))), _abi.TRI_ERR_INVALID_ARG),
+    (dict(mode=7), _abi.TRI_ERR_INVALID_ARG),
+    (dict(mode=1, pos=None), _abi.TRI_ERR_INVALID_ARG),
+    (dict(K=A + 8), _abi.TRI_ERR_ALIGNMENT),
+    (dict(scores=A + 2), _abi.TRI_ERR_ALIGNMENT),
+    (dict(ws=A + 64), _abi.TRI_ERR_ALIGNMENT),
+    (dict(ws_bytes=100), _abi.TRI_ERR_WORKSPACE_TOO_SMALL),
+    (dict(ws=None), _abi.TRI_ERR_INVALID_ARG),
+])
+def test_score_rejects_bad_arguments(kwargs, status):
+    assert _score(M, _kv(), **kwargs) == status
+
+
+def test_score_rejects_bad_model_and_layout():
+    assert _score(tri.model(1, 32, 8, 1e6, head_dim=64), _kv()) == _abi.TRI_ERR_UNSUPPORTED
+    assert _score(tri.model(1, 30, 8, 1e6), _kv()) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(tri.model(1, 32, 8, 0.5), _kv()) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(tri.model(0, 32, 8, 1e6), _kv()) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(M, None) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(M, _kv(layout=5)) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(M, _kv(n_seqs=0)) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(M, _kv(total=-1)) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(M, _kv(row_off=A + 4)) == _abi.TRI_ERR_ALIGNMENT
+    # paged: table required, block size must be a power of two
+    assert _score(M, _kv(layout=1)) == _abi.TRI_ERR_INVALID_ARG
+    assert _score(M, _kv(layout=1, table=A, max_blocks=4, bs=12, nb=8)) == _abi.TRI_ERR_UNSUPPORTED
+    assert _score(M, _kv(layout=1, table=A, max_blocks=0, bs=16, nb=8)) == _abi.TRI_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(B=0), _abi.TRI_ERR_INVALID_ARG),
+    (dict(W=-1), _abi.TRI_ERR_INVALID_ARG),
+    (dict(B=8, W=9), _abi.TRI_ERR_INVALID_ARG),
+    (dict(Ko=A), _abi.TRI_ERR_INVALID_ARG),          # output aliases the input
+    (dict(poso=5 * A, pos=None), _abi.TRI_ERR_INVALID_ARG),
+    (dict(V=2 * A + 8), _abi.TRI_ERR_ALIGNMENT),
+    (dict(Vo=4 * A + 4), _abi.TRI_ERR_ALIGNMENT),
+    (dict(ws_bytes=1024), _abi.TRI_ERR_WORKSPACE_TOO_SMALL),
+    (dict(out=_abi.TriOutDesc(1, 0, None, 16, 0, 4)), _abi.TRI_ERR_INVALID_ARG),
+    (dict(out=_abi.TriOutDesc(1, 4, A, 24, 0, 4)), _abi.TRI_ERR_UNSUPPORTED),
+])
+def test_compact_rejects_bad_arguments(kwargs, status):
+    assert _compact(M, _kv(), **kwargs) == status
+
+
+def test_calib_rejects_bad_arguments():
+    L = _abi.load()
+    assert L.tri_calib(ctypes.byref(M), None, 1024, A, A, None) == _abi.TRI_ERR_INVALID_ARG
+    assert L.tri_calib(ctypes.byref(M), A, 0, A, A, None) == _abi.TRI_ERR_INVALID_ARG
+    assert L.tri_calib(ctypes.byref(M), A + 2, 8, A, A, None) == _abi.TRI_ERR_ALIGNMENT
+    assert L.tri_calib(None, A, 8, A, A, None) == _abi.TRI_ERR_INVALID_ARG
+
+
+def test_status_check_rejects_bad_workspace():
+    L = _abi.load()
+    assert L.tri_status_check(None, None, None) == _abi.TRI_ERR_INVALID_ARG
+    assert L.tri_status_check(A + 16, None, None) == _abi.TRI_ERR_ALIGNMENT
