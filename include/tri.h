@@ -21,7 +21,8 @@
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers on the current device, allocated
  *    and owned by the caller; the library allocates nothing and keeps no state
- *    besides a per-device cache of SM counts.  Every call is asynchronous on
+ *    besides per-device caches (SM counts, and the fixed scratch array of
+ *    tri_score_noalloc with its address).  Every call is asynchronous on
  *    `stream` (a cudaStream_t; NULL = the legacy default stream) and returns
  *    after enqueuing its kernels.
  *  - bf16 tensors are passed as `void*` and hold IEEE bfloat16 bit patterns.
@@ -205,6 +206,35 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
  * NULL), clear it, and return TRI_ERR_DEVICE_FLAG if any bit was set.
  */
 tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream);
+
+/*
+ * tri_score without a workspace argument, for callers that cannot allocate
+ * device memory where they score: code running inside another framework's
+ * memory pool that forbids foreign allocations, plugins whose host process
+ * owns every device allocation, and serving loops that allocate everything
+ * once at start-up.  The method pages have no counterpart to this call; it is
+ * an interface convenience.
+ *
+ * Same arguments and results as tri_score, minus ws/ws_bytes.  The scratch is
+ * a fixed array inside the library (about 3 MiB on every GPU that loads it,
+ * held until the process exits), enough for at most TRI_NOALLOC_MAX_ROWS rows
+ * (n_layers * n_seqs * n_kv_heads); more rows return
+ * TRI_ERR_WORKSPACE_TOO_SMALL before anything is launched.  The call
+ * allocates nothing.
+ *  - The first call on each device looks up the scratch's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.
+ *  - All calls on a device share the one scratch array: calls whose kernels
+ *    can overlap on the GPU (other streams, other threads) race and must be
+ *    serialised by the caller.
+ *  - Data anomalies detected by the kernels are not reported (there is no
+ *    workspace flag word to read); use tri_score with a workspace for those.
+ */
+#define TRI_NOALLOC_MAX_ROWS 4096
+tri_status tri_score_noalloc(const tri_model *m, const tri_kv_desc *kv, const void *K, const int32_t *pos,
+                             const float *centres, const float *mean_norm, const int64_t *p_now,
+                             const int32_t *offsets, int32_t n_offsets, int32_t key_mode, float *scores,
+                             tri_stream_t stream);
 
 #ifdef __cplusplus
 }

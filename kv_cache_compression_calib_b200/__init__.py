@@ -142,3 +142,15 @@ def tri_status_check(ws: torch.Tensor, stream=None):
     flags = ctypes.c_uint32(0)
     st = _L.tri_status_check(_p(ws), ctypes.byref(flags), _s(stream))
     return st, int(flags.value)
+
+
+def tri_score_noalloc(m: TriModel, kv: TriKvDesc, K: torch.Tensor, pos, centres: torch.Tensor,
+                      mean_norm: torch.Tensor, p_now: torch.Tensor, offsets, key_mode: int,
+                      scores: torch.Tensor, stream=None) -> None:
+    """``tri_score`` for callers that cannot allocate device memory: the scratch is a
+    fixed array inside the library (at most TRI_NOALLOC_MAX_ROWS rows; calls on a
+    device share it, so calls that overlap on the GPU race)."""
+    offs = (ctypes.c_int32 * max(len(offsets), 1))(*[int(o) for o in offsets])
+    _check(_L.tri_score_noalloc(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(pos), _p(centres),
+                                _p(mean_norm), _p(p_now), offs, len(offsets), int(key_mode),
+                                _p(scores), _s(stream)), "tri_score_noalloc")

@@ -28,7 +28,8 @@ TRI_KEYS_PRE_ROPE = 1
 
 # Every symbol include/tri.h declares.
 EXPORTS = ("tri_status_str", "tri_version", "tri_workspace_size", "tri_workspace_init", "tri_calib",
-           "tri_score", "tri_compact", "tri_status_check")
+           "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc")
+TRI_NOALLOC_MAX_ROWS = 4096
 
 
 class TriModel(ctypes.Structure):
@@ -82,5 +83,9 @@ def load(path: str = LIB_PATH):
                               _P, _P, ctypes.c_size_t, _P]
     L.tri_status_check.restype = ctypes.c_int
     L.tri_status_check.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), _P]
+    L.tri_score_noalloc.restype = ctypes.c_int
+    L.tri_score_noalloc.argtypes = [ctypes.POINTER(TriModel), ctypes.POINTER(TriKvDesc), _P, _P, _P, _P,
+                                    _P, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, ctypes.c_int32,
+                                    _P, _P]
     _lib = L
     return L
