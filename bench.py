@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_8b_32k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="first N layers only (small cases for profiling; not a bench line)")
     ap.add_argument("--key-mode", choices=["post", "pre"], default="post")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -193,6 +195,8 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.set_device(dev)
     wl0 = synth.WORKLOADS[a.workload]
     B = a.budget or wl0.budget
+    if a.layers:
+        wl0 = wl0.with_(n_layers=min(a.layers, wl0.n_layers))
     wl = rank_workload(wl0, rank, B)
     key_mode = tri.TRI_KEYS_PRE_ROPE if a.key_mode == "pre" else tri.TRI_KEYS_POST_ROPE
     if wl.layout != "contig":

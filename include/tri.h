@@ -156,7 +156,8 @@ tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *ce
  *   K:         bf16 keys in kv's layout, 16-byte aligned
  *   pos:       int32 position of every cached slot (kv's layout).  Read only
  *              for TRI_KEYS_PRE_ROPE; may be NULL for TRI_KEYS_POST_ROPE.
- *   centres, mean_norm: calibration of tri_calib, [n_layers][n_q_heads][64](x2)
+ *   centres, mean_norm: calibration of tri_calib, [n_layers][n_q_heads][64](x2);
+ *              centres 8-byte aligned, mean_norm 4-byte aligned
  *   p_now:     device int64 [n_seqs], the position of each sequence's next token
  *   offsets:   HOST int32 [n_offsets], the future offsets delta, 1 <= n_offsets
  *              <= TRI_MAX_OFFSETS (copied into the launch; not kept)

@@ -143,7 +143,7 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
     if (n_offsets < 1 || n_offsets > TRI_MAX_OFFSETS) return TRI_ERR_INVALID_ARG;
     if (key_mode != TRI_KEYS_POST_ROPE && key_mode != TRI_KEYS_PRE_ROPE) return TRI_ERR_INVALID_ARG;
     if (key_mode == TRI_KEYS_PRE_ROPE && !pos) return TRI_ERR_INVALID_ARG;
-    if (!aligned(K, 16) || !aligned(scores, 4) || !aligned(centres, 4) || !aligned(mean_norm, 4) ||
+    if (!aligned(K, 16) || !aligned(scores, 4) || !aligned(centres, 8) || !aligned(mean_norm, 4) ||
         !aligned(p_now, 8) || (pos && !aligned(pos, 4)))
         return TRI_ERR_ALIGNMENT;
     const int64_t R = rows_of(m, kv->n_seqs);

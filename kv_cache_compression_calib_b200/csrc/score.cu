@@ -22,7 +22,8 @@
 // phase w_f (p_now - j) reduced exactly as a 64-bit fixed-point fraction of a
 // turn (integer multiply mod 2^64), so fp32 never holds a large angle.
 //
-// prep_kernel forms A_f, c_f per row in fp64 and stores fp32.  score_kernel
+// prep_kernel (prep.cu) forms A_f, c_f per row in fp64 and stores fp32.
+// score_kernel
 // streams the keys: each warp owns a contiguous span of the concatenated key
 // space (all rows end to end, so ragged rows balance across the whole grid);
 // per batch of 32 keys, lane (q, g) loads the 16-byte real and imaginary
@@ -34,58 +35,8 @@
 
 namespace tri {
 
-constexpr int kPrepThreads = 64;
 constexpr int kScoreThreads = 256;
-constexpr double kTurnScale = 2.9358905032820014e+18;  // 2^64 / (2 pi)
 constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
-
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) {
-    const Geometry &geo = p.geo;
-    const int r = blockIdx.x;
-    const int f = threadIdx.x;
-    const int h = r % geo.H;
-    const int s = (r / geo.H) % geo.S;
-    const int l = r / (geo.H * geo.S);
-    const double w = pow(p.theta, -2.0 * (double)f / (double)kD);
-    double sr = 0.0, si = 0.0;
-    for (int e = 0; e < p.n_off; e++) {
-        double sn, cs;
-        sincos(w * (double)p.offsets[e], &sn, &cs);
-        sr += cs;
-        si += sn;
-    }
-    double mr = 0.0, mi = 0.0, cf = 0.0;
-    for (int g = 0; g < geo.G; g++) {
-        const int64_t qh = (int64_t)l * geo.Hq + (int64_t)h * geo.G + g;
-        const double qr = p.centres[(qh * kF + f) * 2];
-        const double qi = p.centres[(qh * kF + f) * 2 + 1];
-        mr += qr;
-        mi += qi;
-        cf += (double)p.mean_norm[qh * kF + f] - hypot(qr, qi);
-    }
-    mr /= (double)geo.G;
-    mi /= (double)geo.G;
-    cf /= (double)geo.G;
-    const double tr = mr * sr - mi * si, ti = mr * si + mi * sr;
-    double ar = tr, ai = ti;
-    if (!p.pre_rope) {
-        double sn, cs;
-        sincos(w * (double)p.p_now[s], &sn, &cs);
-        ar = tr * cs - ti * sn;
-        ai = tr * sn + ti * cs;
-    }
-    float *c = p.coef + (int64_t)r * kCoefPerRow + (f >> 3) * kCoefPerGroup;
-    c[f & 7] = (float)ar;
-    c[8 + (f & 7)] = (float)ai;
-    c[16 + (f & 7)] = (float)cf;
-    if (r == 0) {
-        p.turns[f] = __double2ull_rn(w * kTurnScale);
-        if (f == 0) {
-            const int64_t R = (int64_t)geo.L * geo.S * geo.H;
-            if (geo.row_off[0] != 0 || geo.row_off[R] != geo.total) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
-        }
-    }
-}
 
 struct RowCtx {
     int r;
@@ -308,13 +259,6 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
         const float v = __shfl_sync(0xffffffffu, part[0], 8 * (lane & 3) + (lane >> 2));
         if (b0 + lane < bend) p.scores[b0 + lane] = v;
     }
-}
-
-cudaError_t launch_prep(const PrepParams &p, cudaStream_t s) {
-    const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
-    if (R <= 0) return cudaSuccess;
-    prep_kernel<<<(unsigned)R, kPrepThreads, 0, s>>>(p);
-    return cudaGetLastError();
 }
 
 template <bool PAGED, bool PRE>

@@ -87,6 +87,7 @@ M = tri.model(1, 32, 8, 1e6)
     (dict(mode=1, pos=None), _abi.TRI_ERR_INVALID_ARG),
     (dict(K=A + 8), _abi.TRI_ERR_ALIGNMENT),
     (dict(scores=A + 2), _abi.TRI_ERR_ALIGNMENT),
+    (dict(c=A + 4), _abi.TRI_ERR_ALIGNMENT),
     (dict(ws=A + 64), _abi.TRI_ERR_ALIGNMENT),
     (dict(ws_bytes=100), _abi.TRI_ERR_WORKSPACE_TOO_SMALL),
     (dict(ws=None), _abi.TRI_ERR_INVALID_ARG),

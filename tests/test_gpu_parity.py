@@ -227,6 +227,19 @@ def _scores_case(kind, n, rng):
         return s
     if kind == "wide":
         return rng.standard_normal(n) * np.exp(rng.standard_normal(n) * 20)
+    if kind == "subnormal":
+        return rng.standard_normal(n) * 1e-42
+    if kind == "huge":
+        s = rng.standard_normal(n)
+        s[::5] = 3.0e38
+        s[1::7] = -3.0e38
+        return s
+    if kind == "straddle":
+        return rng.standard_normal(n) * 50 + 10
+    if kind == "outlier":
+        s = rng.standard_normal(n)
+        s[::1000] = 1e6
+        return s
     if kind == "inf":
         s = rng.standard_normal(n)
         s[::97] = np.inf
@@ -235,7 +248,8 @@ def _scores_case(kind, n, rng):
     raise ValueError(kind)
 
 
-@pytest.mark.parametrize("kind", ["all_equal", "quantized", "signed_zero", "nan", "wide", "inf"])
+@pytest.mark.parametrize("kind", ["all_equal", "quantized", "signed_zero", "nan", "wide", "inf",
+                                  "subnormal", "huge", "straddle", "outlier"])
 def test_selection_special_scores(ragged, kind):
     wl, host, dev, cs, ms, ref, bound = ragged
     rng = np.random.default_rng(5)
