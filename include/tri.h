@@ -123,6 +123,10 @@ const char *tri_status_str(tri_status s);
 /* Library version, (major << 16) | minor. */
 uint32_t tri_version(void);
 
+/* After a call returned TRI_ERR_CUDA: which CUDA call failed on this thread,
+ * with the CUDA error name and text (a thread-local string, "" if none). */
+const char *tri_last_error(void);
+
 /*
  * Bytes of workspace that tri_score and tri_compact need for `m` and `n_seqs`
  * sequences with budget B.  One buffer may serve both calls (they run in

@@ -28,7 +28,10 @@ _L = _abi.load()
 class TriError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {_L.tri_status_str(status).decode()}")
+        msg = f"{what}: {_L.tri_status_str(status).decode()}"
+        if status == _abi.TRI_ERR_CUDA:
+            msg += f" [{_L.tri_last_error().decode()}]"
+        super().__init__(msg)
 
 
 def _check(st: int, what: str) -> None:

@@ -27,7 +27,7 @@ TRI_KEYS_POST_ROPE = 0
 TRI_KEYS_PRE_ROPE = 1
 
 # Every symbol include/tri.h declares.
-EXPORTS = ("tri_status_str", "tri_version", "tri_workspace_size", "tri_workspace_init", "tri_calib",
+EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_size", "tri_workspace_init", "tri_calib",
            "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc")
 TRI_NOALLOC_MAX_ROWS = 4096
 
@@ -67,6 +67,8 @@ def load(path: str = LIB_PATH):
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_version.restype = ctypes.c_uint32
     L.tri_version.argtypes = []
+    L.tri_last_error.restype = ctypes.c_char_p
+    L.tri_last_error.argtypes = []
     L.tri_workspace_size.restype = ctypes.c_size_t
     L.tri_workspace_size.argtypes = [ctypes.POINTER(TriModel), ctypes.c_int32, ctypes.c_int32]
     L.tri_workspace_init.restype = ctypes.c_int

@@ -1,6 +1,7 @@
 // extern "C" entry points of libtri.so: argument checks, workspace carving and
 // kernel dispatch.  See include/tri.h for the contract of every call.
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 
 #include "tri_internal.cuh"
@@ -82,7 +83,14 @@ tri_status check_ws(const void *ws, size_t have, size_t need) {
     return TRI_OK;
 }
 
-tri_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRI_OK : TRI_ERR_CUDA; }
+thread_local char g_last_error[256] = "";
+
+// Maps a CUDA result to a status, recording the failing call for tri_last_error.
+tri_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return TRI_OK;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+    return TRI_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -103,6 +111,8 @@ const char *tri_status_str(tri_status s) {
 
 uint32_t tri_version(void) { return (0u << 16) | 1u; }
 
+const char *tri_last_error(void) { return g_last_error; }
+
 size_t tri_workspace_size(const tri_model *m, int32_t n_seqs, int32_t B) {
     if (check_model(m) != TRI_OK || n_seqs < 1 || B < 1) return 0;
     return ws_total(rows_of(m, n_seqs), B);
@@ -111,7 +121,7 @@ size_t tri_workspace_size(const tri_model *m, int32_t n_seqs, int32_t B) {
 tri_status tri_workspace_init(void *ws, size_t ws_bytes, tri_stream_t stream) {
     tri_status st = check_ws(ws, ws_bytes, 256);
     if (st != TRI_OK) return st;
-    return cuda_status(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
+    return cuda_status(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream), "tri_workspace_init");
 }
 
 tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *centres, float *mean_norm,
@@ -128,7 +138,7 @@ tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *ce
     p.n_heads = (int32_t)heads;
     p.centres = centres;
     p.mean_norm = mean_norm;
-    return cuda_status(launch_calib(p, (cudaStream_t)stream));
+    return cuda_status(launch_calib(p, (cudaStream_t)stream), "calib_kernel launch");
 }
 
 tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, const int32_t *pos,
@@ -164,7 +174,7 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
     pp.coef = (float *)(w + kWsCoef);
     pp.turns = (unsigned long long *)(w + kWsTurns);
     pp.flags = (unsigned *)(w + kWsFlags);
-    if ((st = cuda_status(launch_prep(pp, s))) != TRI_OK) return st;
+    if ((st = cuda_status(launch_prep(pp, s), "prep_kernel launch")) != TRI_OK) return st;
 
     ScoreParams sp;
     sp.geo = geo;
@@ -175,7 +185,7 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
     sp.turns = pp.turns;
     sp.scores = scores;
     sp.flags = pp.flags;
-    return cuda_status(launch_score(sp, pp.pre_rope, s));
+    return cuda_status(launch_score(sp, pp.pre_rope, s), "score_kernel launch");
 }
 
 tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *scores, int32_t B, int32_t W,
@@ -217,7 +227,7 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
     sp.kept = kept;
     sp.kept_count = kept_count;
     sp.flags = (unsigned *)(w + kWsFlags);
-    if ((st = cuda_status(launch_select(sp, s))) != TRI_OK) return st;
+    if ((st = cuda_status(launch_select(sp, s), "select_kernel launch")) != TRI_OK) return st;
 
     GatherParams gp;
     std::memset(&gp, 0, sizeof(gp));
@@ -236,7 +246,7 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
     gp.V_out = (uint16_t *)V_out;
     gp.pos_out = pos_out;
     gp.flags = sp.flags;
-    return cuda_status(launch_gather(gp, s));
+    return cuda_status(launch_gather(gp, s), "gather_kernel launch");
 }
 
 tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream) {
@@ -244,9 +254,10 @@ tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream) {
     if (st != TRI_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     uint32_t host = 0;
-    if (cudaMemcpyAsync(&host, ws, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return TRI_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return TRI_ERR_CUDA;
-    if (cudaMemsetAsync(ws, 0, sizeof(host), s) != cudaSuccess) return TRI_ERR_CUDA;
+    if ((st = cuda_status(cudaMemcpyAsync(&host, ws, sizeof(host), cudaMemcpyDeviceToHost, s), "flag read")) != TRI_OK)
+        return st;
+    if ((st = cuda_status(cudaStreamSynchronize(s), "stream synchronize")) != TRI_OK) return st;
+    if ((st = cuda_status(cudaMemsetAsync(ws, 0, sizeof(host), s), "flag clear")) != TRI_OK) return st;
     if (flags) *flags = host;
     return host ? TRI_ERR_DEVICE_FLAG : TRI_OK;
 }

@@ -6,33 +6,33 @@
 //   N >  B: keep slots N-W .. N-1, plus the K = B-W best of slots 0 .. M-1
 //           (M = N-W) under (score desc, slot desc); emit slots ascending.
 //
-// One CTA of 512 threads per row, in 32768-slot chunks (one chunk covers rows
-// up to 32K keys).  Streaming passes read the scores coalesced (a warp reads
-// 512 contiguous bytes per instruction); the passes that must walk slots in
-// order give thread t the range 64t .. 64t+63 and read its bins from shared
-// memory.  Scores are compared
-// through order-preserving uint32 keys (-0 folded onto +0, NaN lowest).
-// Exact threshold search:
-//  0. one streaming pass takes the row's finite min/max (and whether a NaN or
-//     an infinity is present);
-//  1. a second pass maps every score to one of 2048 bins by a monotone map -
-//     linear in value over [min, max] when all scores are finite, else the
-//     adaptive key-space map (u - min) >> shift - keeps the bin index (2 B per
-//     slot, shared memory) and histograms it; one block scan finds the bin
-//     holding the K-th best score (higher bins outrank it entirely, lower bins
-//     are outranked entirely);
-//  2. that bin's members (typically a few dozen) are gathered and the K-th
-//     best key value thr is found by counting, per candidate, how many others
-//     are greater / not smaller; a crowded bin instead narrows in key space
-//     with further 2048-bin passes over its members until one value remains;
-//  3. a last pass in slot order keeps the higher bins, the bin's keys above
-//     thr and the most recent of the ties at thr: one block scan of packed
-//     (greater, equal) counts gives every thread its output offset and its
-//     ties' ranks, so kept slots are written ascending with no sort.
-// Only bin indices live in shared memory (64 KB), so two rows share an SM;
-// scores are re-read from global memory (L2) by the streaming passes and by
-// the candidate lookups.  Rows longer than one chunk recompute the bins of
-// non-resident chunks.  Blocks never wait on other blocks.
+// One CTA of 512 threads per row, walking the row in 32768-slot chunks (one
+// chunk covers rows up to 32K keys).  Scores are compared through
+// order-preserving uint32 keys (-0 folded onto +0, NaN lowest).  Streaming
+// passes read the scores coalesced (a warp reads 512 contiguous bytes per
+// instruction, from L2 while the scores are resident there):
+//  0. the value range of an evenly spaced 1024-slot sample, widened by 1/16 of
+//     its span on each side;
+//  1. a monotone map of every score to one of 2048 bins - linear in value over
+//     that range and clamped at both ends (NaN to the lowest bin, as it ranks
+//     lowest), or, when the sample is constant or non-finite, the adaptive
+//     key-space map (u - min) >> shift over the row's key range - is
+//     histogrammed; one block scan finds the bin b* holding the K-th best
+//     score.  Any monotone map keeps the search exact: higher bins are kept
+//     whole, lower bins dropped whole; the spread only decides how many keys
+//     share b*;
+//  2. each chunk's keep-bitmap (1 bit per slot, shared memory) gets the slots
+//     of higher bins, assembled with warp shuffles, and b*'s members (a few
+//     dozen at the workloads' score spreads) are gathered;
+//  3. the members are ranked exactly by (key desc, slot desc) by counting, and
+//     the best ones needed set their bits;
+//  4. the kept slots are emitted ascending from the bitmap: one block scan of
+//     per-thread popcounts gives every thread its output offset.
+// A crowded b* (many ties, outliers, constant rows) instead narrows in key
+// space with further 2048-bin passes over its members to the single key value
+// thr of the K-th best, then an in-order pass with one block scan of packed
+// (greater, equal) counts marks the keys above thr and the most recent ties.
+// Blocks never wait on other blocks.
 #include "tri_internal.cuh"
 
 namespace tri {
@@ -41,10 +41,10 @@ constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kItems = 64;  // slots per thread per chunk
 constexpr int64_t kChunk = (int64_t)kSelThreads * kItems;
+constexpr int kWords = (int)(kChunk / 32);  // bitmap words per chunk
 constexpr int kBins = 2048;
 constexpr int kBinsPerThread = kBins / kSelThreads;
-constexpr int kCandMax = kSelThreads / 4;  // candidates resolved by counting
-constexpr size_t kSelDynSmem = (size_t)kItems * kSelThreads * sizeof(uint16_t);  // 64 KiB
+constexpr int kCandMax = kSelThreads / 4;  // members of b* resolved by counting
 
 // Exclusive scan over the block in thread order; *total receives the sum.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *sm, uint32_t *total) {
@@ -87,8 +87,8 @@ __device__ __forceinline__ void block_minmax(T &mn, T &mx, T *red_min, T *red_ma
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-        T a = threadIdx.x < kSelWarps ? red_min[threadIdx.x] : red_min[0];
-        T b = threadIdx.x < kSelWarps ? red_max[threadIdx.x] : red_max[0];
+        T a = red_min[threadIdx.x < kSelWarps ? threadIdx.x : 0];
+        T b = red_max[threadIdx.x < kSelWarps ? threadIdx.x : 0];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -105,17 +105,35 @@ __device__ __forceinline__ void block_minmax(T &mn, T &mx, T *red_min, T *red_ma
     mx = red_max[0];
 }
 
-// Calls fn(j, score) for the chunk's valid slots j (relative to c0) in a
-// coalesced order: 16-byte vector v = k*512 + t covers slots 4v .. 4v+3, so a
-// warp reads 512 contiguous bytes per instruction (4-byte loads, slot
-// k*512 + t, when the row is not 16-byte aligned).
-template <typename Fn>
-__device__ __forceinline__ void for_each_score(const float *sc, int64_t M, int64_t c0, bool vec, Fn &&fn) {
-    const int t = threadIdx.x;
+// Monotone map of a score to one of kBins bins (uniform over the row).
+struct BinMap {
+    int by_value;  // 1: linear in value from vmin; 0: key space from lo
+    float vmin, scale;
+    uint32_t lo;
+    int shift;
+    __device__ __forceinline__ int operator()(float s) const {
+        // Clamped at both ends: values outside [vmin, vmin + kBins/scale) go to
+        // the end bins and NaN (fmaxf returns the non-NaN operand) to bin 0, where
+        // it ranks lowest; subtract, multiply and clamps all keep the order.
+        if (by_value) return (int)fminf(fmaxf((s - vmin) * scale, 0.f), (float)(kBins - 1));
+        return (int)((order_key(s) - lo) >> shift);
+    }
+};
+
+// Number of slots of the chunk starting at c0 (at most kChunk).
+__device__ __forceinline__ int chunk_len(int64_t M, int64_t c0) {
     const int64_t rem = M - c0;
-    const int n = rem >= kChunk ? (int)kChunk : (int)rem;
+    return rem >= kChunk ? (int)kChunk : (int)rem;
+}
+
+// Calls fn(j, score) for every slot j < n of the chunk at `base`, coalesced:
+// 16-byte vector v = k*512 + t covers slots 4v .. 4v+3 (4-byte loads of slot
+// k*512 + t when the row is not 16-byte aligned).
+template <typename Fn>
+__device__ __forceinline__ void for_each_score(const float *base, int n, bool vec, Fn &&fn) {
+    const int t = threadIdx.x;
     if (vec) {
-        const float4 *q = reinterpret_cast<const float4 *>(sc + c0);
+        const float4 *q = reinterpret_cast<const float4 *>(base);
         const int nvec = n >> 2;
 #pragma unroll 4
         for (int k = 0; k < kItems / 4; k++) {
@@ -129,42 +147,53 @@ __device__ __forceinline__ void for_each_score(const float *sc, int64_t M, int64
             }
         }
         const int j = 4 * nvec + t;  // ragged tail: at most 3 slots
-        if (j < n) fn(j, __ldg(sc + c0 + j));
+        if (j < n) fn(j, __ldg(base + j));
     } else {
 #pragma unroll 4
         for (int k = 0; k < kItems; k++) {
             const int j = k * kSelThreads + t;
-            if (j < n) fn(j, __ldg(sc + c0 + j));
+            if (j < n) fn(j, __ldg(base + j));
         }
     }
 }
 
-// Shared-memory position (in uint16 units) of the bin of chunk slot j.  Slot
-// j = 64t + e belongs to thread t's range; its 32 words are stored XOR-swizzled
-// (word w at w ^ (t mod 32)), so a warp reading word w of each lane's range
-// touches 32 distinct banks.
-__device__ __forceinline__ int bin_pos(int j) {
-    const int t = j >> 6, e = j & 63;
-    return (((t << 5) | ((e >> 1) ^ (t & 31))) << 1) | (e & 1);
-}
-
-// Number of valid slots of chunk c0 in this thread's range 64t .. 64t+63.
-__device__ __forceinline__ int range_count(int64_t M, int64_t c0) {
-    const int64_t rem = M - c0 - (int64_t)threadIdx.x * kItems;
-    return rem <= 0 ? 0 : (rem >= kItems ? kItems : (int)rem);
-}
-
-// Monotone map of a score to one of kBins bins (uniform over the row).
-struct BinMap {
-    int by_value;  // 1: linear in value from vmin; 0: key space from lo
-    float vmin, scale;
-    uint32_t lo;
-    int shift;
-    __device__ __forceinline__ int operator()(float s) const {
-        if (by_value) return min((int)((s - vmin) * scale), kBins - 1);
-        return (int)((order_key(s) - lo) >> shift);
+// Writes the chunk's bitmap words with bit j = pred(j, score of slot j), j < n
+// (bits past n are 0).  Every word is written once, without atomics: in the
+// vector layout lane l holds slots 4l .. 4l+3 of its warp's 128-slot span, so
+// the 8 lanes of a word OR their nibbles together with shuffles.
+template <typename Pred>
+__device__ __forceinline__ void build_bitmap(const float *base, int n, bool vec, uint32_t *bm_words, Pred &&pred) {
+    const int t = threadIdx.x, lane = t & 31;
+    if (vec) {
+        const float4 *q = reinterpret_cast<const float4 *>(base);
+#pragma unroll 4
+        for (int k = 0; k < kItems / 4; k++) {
+            const int v = k * kSelThreads + t;
+            uint32_t nib = 0;
+            if (4 * v + 3 < n) {
+                const float4 x = __ldg(q + v);
+                nib = (uint32_t)pred(4 * v, x.x) | ((uint32_t)pred(4 * v + 1, x.y) << 1) |
+                      ((uint32_t)pred(4 * v + 2, x.z) << 2) | ((uint32_t)pred(4 * v + 3, x.w) << 3);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    if (4 * v + i < n) nib |= (uint32_t)pred(4 * v + i, __ldg(base + 4 * v + i)) << i;
+            }
+            uint32_t w = nib << (4 * (lane & 7));
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            w |= __shfl_xor_sync(0xffffffffu, w, 4);
+            if ((lane & 7) == 0) bm_words[(4 * v) >> 5] = w;
+        }
+    } else {
+#pragma unroll 4
+        for (int k = 0; k < kItems; k++) {
+            const int j = k * kSelThreads + t;
+            const uint32_t w = __ballot_sync(0xffffffffu, j < n && pred(j, __ldg(base + j)));
+            if (lane == 0) bm_words[j >> 5] = w;
+        }
     }
-};
+}
 
 // After a histogram pass: the bin (top first) holding the need-th best key and
 // the number of keys in higher bins.
@@ -193,14 +222,34 @@ __device__ __forceinline__ void find_bin(const uint32_t *hist, uint32_t need, ui
     above = *sh_above;
 }
 
+// Emits the set bits of a chunk's bitmap as ascending slots c0 + j into
+// out[*base ...] (positions >= K are never written).
+__device__ __forceinline__ void emit_bitmap(const uint32_t *bm_words, int64_t c0, int32_t *out, uint32_t K,
+                                            uint32_t &base, uint32_t *scan_sm) {
+    const int t = threadIdx.x;
+    const uint32_t w0 = bm_words[2 * t], w1 = bm_words[2 * t + 1];
+    uint32_t tot;
+    uint32_t o = base + block_exclusive_scan((uint32_t)(__popc(w0) + __popc(w1)), scan_sm, &tot);
+    unsigned long long bits = ((unsigned long long)w1 << 32) | w0;
+    while (bits) {
+        const int e = __ffsll((long long)bits) - 1;
+        bits &= bits - 1;
+        if (o < K) out[o] = (int32_t)(c0 + 64 * t + e);
+        o++;
+    }
+    base += tot;
+}
+
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectParams p) {
-    extern __shared__ __align__(16) uint16_t bins[];  // [kChunk], bin of each slot of the resident chunk
     __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t bmw[kWords];  // keep-bitmap of the current chunk
     __shared__ uint32_t scan_sm[kSelWarps];
     __shared__ uint32_t red_a[kSelWarps], red_b[kSelWarps];
     __shared__ float red_fa[kSelWarps], red_fb[kSelWarps];
     __shared__ uint32_t cand_key[kCandMax];
-    __shared__ uint32_t sh_bin, sh_above, sh_count, sh_thr, sh_ge;
+    __shared__ int64_t cand_slot[kCandMax];
+    __shared__ uint8_t cand_keep[kCandMax];
+    __shared__ uint32_t sh_bin, sh_above, sh_count;
 
     const int tid = threadIdx.x;
     const int r = blockIdx.x;
@@ -232,39 +281,39 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
         sh_bin = 0;
         sh_above = 0;
         sh_count = 0;
-        sh_thr = 0;
-        sh_ge = 0;
     }
 
-    // Pass 0: finite value range; NaN / infinity present.
+    // Value range of an evenly spaced 1024-slot sample of the row, widened by
+    // 1/16 of its span on each side (two 4-byte loads per thread).
     float fmn = INFINITY, fmx = -INFINITY;
-    int nan = 0, inf = 0;
-    for (int c = 0; c < nchunks; c++) {
-        for_each_score(sc, M, (int64_t)c * kChunk, vec, [&](int, float s) {
-            fmn = fminf(fmn, s);
-            fmx = fmaxf(fmx, s);
-            nan |= s != s;
-            inf |= fabsf(s) == INFINITY;
-        });
+    int snan = 0;
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+        const int64_t j = ((int64_t)(2 * tid + k) * M) / (2 * kSelThreads);  // < M
+        const float s = __ldg(sc + j);
+        fmn = fminf(fmn, s);
+        fmx = fmaxf(fmx, s);
+        snan |= s != s;
     }
-    if (__syncthreads_or(nan) && tid == 0) atomicOr(p.flags, TRI_FLAG_NONFINITE);
-    const int any_nonfinite = __syncthreads_or(nan | inf);
+    const int any_snan = __syncthreads_or(snan);
     block_minmax(fmn, fmx, red_fa, red_fb);
 
     BinMap bm;
-    bm.vmin = fmn;
     const float vspan = fmx - fmn;
-    bm.scale = vspan > 0.f ? (float)kBins / vspan : 0.f;
-    bm.by_value = !any_nonfinite && isfinite(vspan) && vspan > 0.f && isfinite(bm.scale);
-    uint32_t umn = 0u, umx = 0xffffffffu;
+    const float vlo = fmn - 0.0625f * vspan, vhi = fmx + 0.0625f * vspan;
+    bm.vmin = vlo;
+    bm.scale = vhi > vlo ? (float)kBins / (vhi - vlo) : 0.f;
+    bm.by_value = !any_snan && isfinite(vspan) && vspan > 0.f && isfinite(vlo) && isfinite(vhi) &&
+                  isfinite(bm.scale) && bm.scale > 0.f;
+    uint32_t umx = 0xffffffffu;
     bm.lo = 0u;
     bm.shift = 21;
-    if (!bm.by_value) {
-        // key-space bins over the row's key range
-        umn = 0xffffffffu;
+    if (!bm.by_value) {  // key-space bins over the row's key range
+        uint32_t umn = 0xffffffffu;
         umx = 0u;
         for (int c = 0; c < nchunks; c++) {
-            for_each_score(sc, M, (int64_t)c * kChunk, vec, [&](int, float s) {
+            const int64_t c0 = (int64_t)c * kChunk;
+            for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
                 const uint32_t u = order_key(s);
                 umn = min(umn, u);
                 umx = max(umx, u);
@@ -277,198 +326,185 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
         bm.shift = nbits > 11 ? nbits - 11 : 0;
     }
 
-    // Pass 1: bin every score (kept in shared memory) and histogram the bins.
+    // Pass 1: histogram of the bins; b* and the keys above it.
     for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
     __syncthreads();
-    int resident = 0;
+    int nan = 0;
     for (int c = 0; c < nchunks; c++) {
-        __syncthreads();  // bins of the previous chunk are no longer read
-        for_each_score(sc, M, (int64_t)c * kChunk, vec, [&](int j, float s) {
-            const int b = bm(s);
-            bins[bin_pos(j)] = (uint16_t)b;
-            atomicAdd(&hist[b], 1u);
+        const int64_t c0 = (int64_t)c * kChunk;
+        for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
+            atomicAdd(&hist[bm(s)], 1u);
+            nan |= s != s;
         });
-        resident = c;
     }
-    __syncthreads();
+    if (__syncthreads_or(nan) && tid == 0) atomicOr(p.flags, TRI_FLAG_NONFINITE);
     uint32_t bin, above;
     find_bin(hist, K, scan_sm, &sh_bin, &sh_above, bin, above);
-    uint32_t need = K - above;  // keys still to keep from `bin`
-    uint32_t cand = hist[bin];  // keys in `bin`
-    uint32_t thr, tie_skip;
-
-    // Make chunk c's bins resident (recomputed from the scores if needed); nv is
-    // then this thread's count in its slot range 64t .. 64t+63 of the chunk.
-    int nv = range_count(M, (int64_t)resident * kChunk);
-    auto ensure = [&](int c) {
-        if (c != resident) {
-            __syncthreads();
-            for_each_score(sc, M, (int64_t)c * kChunk, vec, [&](int j, float s) { bins[bin_pos(j)] = (uint16_t)bm(s); });
-            __syncthreads();
-            resident = c;
-        }
-        nv = range_count(M, (int64_t)c * kChunk);
-    };
-
-    // Calls fn(e, bin) for this thread's valid range slots 64t + e, e < nv.
-    const uint32_t *bins32 = reinterpret_cast<const uint32_t *>(bins);
-    auto for_range = [&](auto &&fn) {
-#pragma unroll 4
-        for (int w = 0; w < kItems / 2; w++) {
-            if (2 * w < nv) {
-                const uint32_t pair = bins32[(tid << 5) | (w ^ (tid & 31))];
-                fn(2 * w, pair & 0xffffu);
-                if (2 * w + 1 < nv) fn(2 * w + 1, pair >> 16);
-            }
-        }
-    };
+    const uint32_t need = K - above;  // keys to keep from b*
+    const uint32_t cand = hist[bin];  // keys in b*
+    const int ibin = (int)bin;
+    uint32_t out_base = 0;
 
     if (cand <= (uint32_t)kCandMax) {
-        // Gather the bin's keys; the need-th largest is thr.
-        for (int k = 0; k < nchunks; k++) {
-            const int c = (resident + k) % nchunks;
-            ensure(c);
-            const int64_t s0 = (int64_t)c * kChunk + (int64_t)tid * kItems;
-            for_range([&](int e, uint32_t b) {
-                if (b == bin) {
-                    const uint32_t slot = atomicAdd(&sh_count, 1u);
-                    if (slot < (uint32_t)kCandMax) cand_key[slot] = order_key(__ldg(sc + s0 + e));
+        // Pass 2: gather b*'s members (and, for a one-chunk row, the bitmap of
+        // the higher bins on the same read).
+        for (int c = 0; c < nchunks; c++) {
+            const int64_t c0 = (int64_t)c * kChunk;
+            const int n = chunk_len(M, c0);
+            if (nchunks == 1) {
+                build_bitmap(sc, n, vec, bmw, [&](int j, float s) {
+                    const int b = bm(s);
+                    if (b == ibin) {
+                        const uint32_t i = atomicAdd(&sh_count, 1u);
+                        if (i < (uint32_t)kCandMax) {
+                            cand_key[i] = order_key(s);
+                            cand_slot[i] = j;
+                        }
+                    }
+                    return b > ibin;
+                });
+            } else {
+                for_each_score(sc + c0, n, vec, [&](int j, float s) {
+                    if (bm(s) == ibin) {
+                        const uint32_t i = atomicAdd(&sh_count, 1u);
+                        if (i < (uint32_t)kCandMax) {
+                            cand_key[i] = order_key(s);
+                            cand_slot[i] = c0 + j;
+                        }
+                    }
+                });
+            }
+        }
+        __syncthreads();
+        // Rank each member by (key desc, slot desc), 4 threads per member.
+        const int i = tid >> 2, q = tid & 3;
+        uint32_t rank = 0;
+        uint32_t ui = 0;
+        int64_t si = 0;
+        if (i < (int)cand) {
+            ui = cand_key[i];
+            si = cand_slot[i];
+            for (int j = q; j < (int)cand; j += 4) {
+                const uint32_t uj = cand_key[j];
+                rank += (uj > ui) | ((uj == ui) & (cand_slot[j] > si));
+            }
+        }
+        rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+        rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+        if (i < (int)cand && q == 0) cand_keep[i] = rank < need;
+        __syncthreads();
+        for (int c = 0; c < nchunks; c++) {
+            const int64_t c0 = (int64_t)c * kChunk;
+            const int n = chunk_len(M, c0);
+            if (nchunks > 1) build_bitmap(sc + c0, n, vec, bmw, [&](int, float s) { return bm(s) > ibin; });
+            __syncthreads();
+            if (tid < (int)cand && cand_keep[tid] && cand_slot[tid] >= c0 && cand_slot[tid] < c0 + n) {
+                const int j = (int)(cand_slot[tid] - c0);
+                atomicOr(&bmw[j >> 5], 1u << (j & 31));
+            }
+            __syncthreads();
+            emit_bitmap(bmw, c0, out, K, out_base, scan_sm);
+        }
+        return;
+    }
+
+    // Crowded b*: narrow in key space over its members, whose keys form the
+    // contiguous range [lo, hi], to the single key value thr.
+    uint32_t lo, hi;
+    if (bm.by_value) {
+        uint32_t cmn = 0xffffffffu, cmx = 0u;
+        for (int c = 0; c < nchunks; c++) {
+            const int64_t c0 = (int64_t)c * kChunk;
+            for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
+                if (bm(s) == ibin) {
+                    const uint32_t u = order_key(s);
+                    cmn = min(cmn, u);
+                    cmx = max(cmx, u);
+                }
+            });
+        }
+        block_minmax(cmn, cmx, red_a, red_b);
+        lo = cmn;
+        hi = cmx;
+    } else {
+        lo = bm.lo + (bin << bm.shift);
+        const unsigned long long h = (unsigned long long)lo + ((1ull << bm.shift) - 1ull);
+        hi = h < (unsigned long long)umx ? (uint32_t)h : umx;
+    }
+    uint32_t need2 = need, cand2 = cand;
+    for (;;) {
+        const uint32_t range = hi - lo;
+        if (range == 0) break;
+        const int nbits = 32 - __clz(range);
+        const int shift = nbits > 11 ? nbits - 11 : 0;
+        for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
+        __syncthreads();
+        for (int c = 0; c < nchunks; c++) {
+            const int64_t c0 = (int64_t)c * kChunk;
+            for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
+                if (bm(s) == ibin) {
+                    const uint32_t u = order_key(s);
+                    if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> shift], 1u);
                 }
             });
         }
         __syncthreads();
-        // 4 threads per candidate count the candidates greater / not smaller.
-        const int i = tid >> 2, q = tid & 3;
-        uint32_t gt = 0, ge = 0, ui = 0;
-        if (i < (int)cand) {
-            ui = cand_key[i];
-            for (int j = q; j < (int)cand; j += 4) {
-                const uint32_t uj = cand_key[j];
-                gt += uj > ui;
-                ge += uj >= ui;
-            }
-        }
-        gt += __shfl_xor_sync(0xffffffffu, gt, 1);
-        gt += __shfl_xor_sync(0xffffffffu, gt, 2);
-        ge += __shfl_xor_sync(0xffffffffu, ge, 1);
-        ge += __shfl_xor_sync(0xffffffffu, ge, 2);
-        if (i < (int)cand && q == 0 && gt < need && ge >= need) {
-            sh_thr = ui;  // every such candidate holds the same key value
-            sh_ge = ge;
-        }
+        uint32_t b2, ab2;
+        find_bin(hist, need2, scan_sm, &sh_bin, &sh_above, b2, ab2);
+        need2 -= ab2;
+        cand2 = hist[b2];
+        const uint32_t nlo = lo + (b2 << shift);
+        const unsigned long long nhi = (unsigned long long)nlo + ((1ull << shift) - 1ull);
+        hi = nhi < (unsigned long long)hi ? (uint32_t)nhi : hi;
+        lo = nlo;
         __syncthreads();
-        thr = sh_thr;
-        tie_skip = sh_ge - need;
-    } else {
-        // Crowded bin: narrow in key space over its members, whose keys form the
-        // contiguous range [lo, hi].
-        uint32_t lo, hi;
-        if (bm.by_value) {
-            uint32_t cmn = 0xffffffffu, cmx = 0u;
-            for (int k = 0; k < nchunks; k++) {
-                const int c = (resident + k) % nchunks;
-                ensure(c);
-                const int64_t s0 = (int64_t)c * kChunk + (int64_t)tid * kItems;
-                for_range([&](int e, uint32_t b) {
-                    if (b == bin) {
-                        const uint32_t u = order_key(__ldg(sc + s0 + e));
-                        cmn = min(cmn, u);
-                        cmx = max(cmx, u);
-                    }
-                });
-            }
-            block_minmax(cmn, cmx, red_a, red_b);
-            lo = cmn;
-            hi = cmx;
-        } else {
-            lo = bm.lo + (bin << bm.shift);
-            const unsigned long long h = (unsigned long long)lo + ((1ull << bm.shift) - 1ull);
-            hi = h < (unsigned long long)umx ? (uint32_t)h : umx;
-        }
-        for (;;) {
-            const uint32_t range = hi - lo;
-            if (range == 0) break;
-            const int nbits = 32 - __clz(range);
-            const int shift = nbits > 11 ? nbits - 11 : 0;
-            for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
-            __syncthreads();
-            for (int k = 0; k < nchunks; k++) {
-                const int c = (resident + k) % nchunks;
-                ensure(c);
-                const int64_t s0 = (int64_t)c * kChunk + (int64_t)tid * kItems;
-                for_range([&](int e, uint32_t b) {
-                    if (b == bin) {
-                        const uint32_t u = order_key(__ldg(sc + s0 + e));
-                        if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> shift], 1u);
-                    }
-                });
-            }
-            __syncthreads();
-            uint32_t b2, ab2;
-            find_bin(hist, need, scan_sm, &sh_bin, &sh_above, b2, ab2);
-            need -= ab2;
-            cand = hist[b2];
-            const uint32_t nlo = lo + (b2 << shift);
-            const unsigned long long nhi = (unsigned long long)nlo + ((1ull << shift) - 1ull);
-            hi = nhi < (unsigned long long)hi ? (uint32_t)nhi : hi;
-            lo = nlo;
-            __syncthreads();
-            if (shift == 0) break;
-        }
-        thr = lo;
-        tie_skip = cand - need;
+        if (shift == 0) break;
     }
-
-    // Last pass: emit kept slots of [0, M) in ascending order, chunk by chunk.
-    uint32_t gt_base = 0, tie_base = 0;
+    const uint32_t thr = lo;
+    const uint32_t tie_skip = cand2 - need2;  // ties at thr in the oldest slots are dropped
+    // In slot order (thread t: slots 64t .. 64t+63), mark the keys above thr and
+    // the ties whose rank from the oldest is at least tie_skip.
+    uint32_t tie_base = 0;
     for (int c = 0; c < nchunks; c++) {
-        ensure(c);
-        const int64_t s0 = (int64_t)c * kChunk + (int64_t)tid * kItems;
+        const int64_t c0 = (int64_t)c * kChunk;
+        const int n = chunk_len(M, c0);
+        const int j0 = tid * kItems;
         unsigned long long gt_bits = 0, eq_bits = 0;
-        for_range([&](int e, uint32_t b) {
-            if (b > bin) {
-                gt_bits |= 1ull << e;
-            } else if (b == bin) {
-                const uint32_t u = order_key(__ldg(sc + s0 + e));
-                gt_bits |= (unsigned long long)(u > thr) << e;
-                eq_bits |= (unsigned long long)(u == thr) << e;
-            }
-        });
-        const uint32_t packed = ((uint32_t)__popcll(gt_bits) << 16) | (uint32_t)__popcll(eq_bits);
-        uint32_t tot;
-        const uint32_t ex = block_exclusive_scan(packed, scan_sm, &tot);
-        uint32_t tie_rank = tie_base + (ex & 0xffffu);
-        uint32_t o = gt_base + (ex >> 16) + (tie_rank > tie_skip ? tie_rank - tie_skip : 0u);
-        unsigned long long any = gt_bits | eq_bits;
-        while (any) {
-            const int e = __ffsll((long long)any) - 1;
-            any &= any - 1;
-            const bool eq = (eq_bits >> e) & 1ull;
-            const bool keep = !eq || tie_rank >= tie_skip;
-            tie_rank += eq;
-            if (keep) {
-                if (o < K) out[o] = (int32_t)(s0 + e);
-                o++;
+        for (int e = 0; e < kItems; e++) {
+            const int j = j0 + e;
+            if (j < n) {
+                const float s = __ldg(sc + c0 + j);
+                const int b = bm(s);
+                if (b > ibin) {
+                    gt_bits |= 1ull << e;
+                } else if (b == ibin) {
+                    const uint32_t u = order_key(s);
+                    gt_bits |= (unsigned long long)(u > thr) << e;
+                    eq_bits |= (unsigned long long)(u == thr) << e;
+                }
             }
         }
-        gt_base += tot >> 16;
-        tie_base += tot & 0xffffu;
+        uint32_t tot;
+        uint32_t rank = tie_base + block_exclusive_scan((uint32_t)__popcll(eq_bits), scan_sm, &tot);
+        unsigned long long keep = gt_bits, eqs = eq_bits;
+        while (eqs) {
+            const int e = __ffsll((long long)eqs) - 1;
+            eqs &= eqs - 1;
+            if (rank >= tie_skip) keep |= 1ull << e;
+            rank++;
+        }
+        tie_base += tot;
+        bmw[2 * tid] = (uint32_t)keep;
+        bmw[2 * tid + 1] = (uint32_t)(keep >> 32);
+        __syncthreads();
+        emit_bitmap(bmw, c0, out, K, out_base, scan_sm);
     }
 }
 
 cudaError_t launch_select(const SelectParams &p, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
-    static bool configured[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!configured[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSelDynSmem);
-        if (e != cudaSuccess) return e;
-        configured[dev & 63] = true;
-    }
-    select_kernel<<<(unsigned)R, kSelThreads, kSelDynSmem, s>>>(p);
+    select_kernel<<<(unsigned)R, kSelThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 
