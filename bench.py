@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=None,
                     help="first N layers only (small cases for profiling; not a bench line)")
     ap.add_argument("--key-mode", choices=["post", "pre"], default="post")
+    ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
+                    help="timed steps replay CUDA graphs of the calls (default) or call eagerly")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -62,12 +64,13 @@ def parse():
     return a
 
 
-def workload_config(wl, B, key_mode):
+def workload_config(wl, B, key_mode, launch="eager"):
     lo, hi = wl.seq_len
     return {"workload": wl.name, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "rope_theta": wl.theta,
             "batch": wl.batch, "keys_per_head": lo if lo == hi else [lo, hi], "budget": B,
             "window": wl.window, "offsets": wl.n_offsets, "key_mode": key_mode + "_rope",
+            "launch": launch,
             "layout": wl.layout,
             "l2": "inputs larger than L2: K+V %.1f GB read per step, no flush" % (
                 2 * 256 * wl.n_layers * wl.batch * wl.n_kv_heads * np.mean(wl.seq_len) / 1e9)}
@@ -228,20 +231,38 @@ def run_ours(a, rank, world, local_rank):
     kept = torch.empty(R, B, dtype=torch.int32, device=dev)
     offsets = wl.offsets
 
-    def step():
+    out_desc = tri.out_contig()
+
+    def score_call():  # on the current stream (the capture stream while capturing)
         tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode, scores, ws,
-                      stream)
-        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
-                        kept, None, ws, stream)
+                      torch.cuda.current_stream(dev))
+
+    def compact_call():
+        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, out_desc, Ko, Vo, po, kept, None,
+                        ws, torch.cuda.current_stream(dev))
 
     sampler = ClockSampler(local_rank)
     sampler.start()
     for _ in range(a.warmup):
-        step()
+        score_call()
+        compact_call()
     torch.cuda.synchronize()
     st, flags = tri.tri_status_check(ws, stream)
     if st != 0:
         raise RuntimeError(f"device flags {flags:#x} after warm-up")
+    if a.launch == "graph":
+        g_score, g_compact = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_score):
+            score_call()
+        with torch.cuda.graph(g_compact):
+            compact_call()
+        do_score, do_compact = g_score.replay, g_compact.replay
+        for _ in range(a.warmup):
+            do_score()
+            do_compact()
+        torch.cuda.synchronize()
+    else:
+        do_score, do_compact = score_call, compact_call
 
     # ---- device-resident timed region
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
@@ -253,11 +274,9 @@ def run_ours(a, rank, world, local_rank):
     t0.record(stream)
     for i in range(a.steps):
         ev[i][0].record(stream)
-        tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode, scores, ws,
-                      stream)
+        do_score()
         ev[i][1].record(stream)
-        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
-                        kept, None, ws, stream)
+        do_compact()
     t1.record(stream)
     torch.cuda.synchronize()
     wall1 = time.time()
@@ -292,7 +311,7 @@ def run_ours(a, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(wl, B, a.key_mode),
+        "config": workload_config(wl, B, a.key_mode, "cuda_graph" if a.launch == "graph" else "eager"),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(total),
                      "kernel": "tri_score (prep + score kernels)", "peak_kind": peak_kind,
@@ -439,7 +458,7 @@ def run_reference(a, rank, world):
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": workload_config(wl, B, "post"),
+            "config": workload_config(wl, B, "post", "cuda_graph" if a.launch == "graph" else "eager"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

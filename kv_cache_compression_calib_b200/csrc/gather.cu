@@ -15,6 +15,8 @@ constexpr int kGatherThreads = 256;
 constexpr int kSlotsPerCta = 64;  // 8 warps x 4 iterations x 2 records
 
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherParams p) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     const Geometry &geo = p.geo;
     const int64_t chunks = (p.B + kSlotsPerCta - 1) / kSlotsPerCta;
     const int64_t r = blockIdx.x / chunks;
@@ -84,8 +86,7 @@ cudaError_t launch_gather(const GatherParams &p, cudaStream_t s) {
     const int64_t chunks = (p.B + kSlotsPerCta - 1) / kSlotsPerCta;
     const int64_t grid = R * chunks;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    gather_kernel<<<(unsigned)grid, kGatherThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(gather_kernel, dim3((unsigned)grid), dim3(kGatherThreads), 0, s, p);
 }
 
 }  // namespace tri

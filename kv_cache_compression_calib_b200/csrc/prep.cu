@@ -36,8 +36,19 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
     const int s = (r / geo.H) % geo.S;
     const int l = r / (geo.H * geo.S);
     const int64_t qh0 = (int64_t)l * geo.Hq + (int64_t)h * geo.G;
-    // Issue the loads the part-0 threads need first, so their latency overlaps
-    // the fp64 math below (the first 8 query heads of the group).
+    // The offsets' phasor sums depend on kernel parameters only: form them before
+    // waiting for the preceding kernel on the stream.
+    const double w = pow(p.theta, -2.0 * (double)f / (double)kD);
+    const unsigned long long T = __double2ull_rn(w * kTurnScale);
+    double sr = 0.0, si = 0.0;
+    for (int e = part; e < p.n_off; e += kPrepParts) {
+        double sn, cs;
+        sincos_turns((unsigned long long)(long long)p.offsets[e] * T, &sn, &cs);
+        sr += cs;
+        si += sn;
+    }
+    grid_dependency_wait();
+    grid_dependents_launch();
     float2 qv[8];
     float mv[8];
     long long pnow = 0;
@@ -50,15 +61,6 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
             }
         }
         pnow = p.p_now[s];
-    }
-    const double w = pow(p.theta, -2.0 * (double)f / (double)kD);
-    const unsigned long long T = __double2ull_rn(w * kTurnScale);
-    double sr = 0.0, si = 0.0;
-    for (int e = part; e < p.n_off; e += kPrepParts) {
-        double sn, cs;
-        sincos_turns((unsigned long long)(long long)p.offsets[e] * T, &sn, &cs);
-        sr += cs;
-        si += sn;
     }
     part_re[part][f] = sr;
     part_im[part][f] = si;
@@ -119,8 +121,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
 cudaError_t launch_prep(const PrepParams &p, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
-    prep_kernel<<<(unsigned)R, kPrepThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(prep_kernel, dim3((unsigned)R), dim3(kPrepThreads), 0, s, p);
 }
 
 }  // namespace tri

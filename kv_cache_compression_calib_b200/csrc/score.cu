@@ -146,6 +146,8 @@ __device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx 
 
 template <bool PAGED, bool PRE>
 __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const ScoreParams p) {
+    grid_dependency_wait();
+    grid_dependents_launch();
     const Geometry &geo = p.geo;
     const int lane = threadIdx.x & 31;
     const int q = lane >> 3;  // key of the 4-key group
@@ -276,8 +278,7 @@ static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
     int64_t grid = (int64_t)sm_count() * o;
     if (want < grid) grid = want;
     if (grid < 1) grid = 1;
-    score_kernel<PAGED, PRE><<<(unsigned)grid, kScoreThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(score_kernel<PAGED, PRE>, dim3((unsigned)grid), dim3(kScoreThreads), 0, s, p);
 }
 
 cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s) {

@@ -115,7 +115,11 @@ struct BinMap {
         // Clamped at both ends: values outside [vmin, vmin + kBins/scale) go to
         // the end bins and NaN (fmaxf returns the non-NaN operand) to bin 0, where
         // it ranks lowest; subtract, multiply and clamps all keep the order.
-        if (by_value) return (int)fminf(fmaxf((s - vmin) * scale, 0.f), (float)(kBins - 1));
+        // Adding 2^23 to a value in [0, 2047] rounds it to an integer held in the
+        // low mantissa bits: a monotone float-to-bin step on the FMA/ALU pipes.
+        if (by_value)
+            return __float_as_int(fminf(fmaxf((s - vmin) * scale, 0.f), (float)(kBins - 1)) + 8388608.f) -
+                   0x4B000000;
         return (int)((order_key(s) - lo) >> shift);
     }
 };
@@ -251,6 +255,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
     __shared__ uint8_t cand_keep[kCandMax];
     __shared__ uint32_t sh_bin, sh_above, sh_count;
 
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int tid = threadIdx.x;
     const int r = blockIdx.x;
     const int64_t row_lo = p.geo.row_off[r];
@@ -504,8 +510,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
 cudaError_t launch_select(const SelectParams &p, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
-    select_kernel<<<(unsigned)R, kSelThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(select_kernel, dim3((unsigned)R), dim3(kSelThreads), 0, s, p);
 }
 
 }  // namespace tri

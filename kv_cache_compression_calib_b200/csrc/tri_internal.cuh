@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "tri.h"
 
 namespace tri {
@@ -96,6 +98,34 @@ cudaError_t launch_select(const SelectParams &p, cudaStream_t s);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t s);
 
 int sm_count();  // SMs of the current device (cached per device)
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while its predecessor on the stream finishes.  Every kernel launched this
+// way calls grid_dependency_wait() before its first access to global memory
+// and grid_dependents_launch() only after that wait, so each kernel still
+// starts its memory work after every earlier kernel on the stream completed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Wait until the grids this one depends on have completed and their memory is
+// visible (returns at once when launched without programmatic serialization).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel on the stream to be scheduled.
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 // ------------------------------------------------------------ device helpers
 
