@@ -8,6 +8,7 @@ offline and timed separately.  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload qwen3_8b_32k] [--budget B] [--key-mode post|pre]
+                  [--elem bf16|fp8]
 
 N > 1 (under torchrun): every rank compacts its own cache of the same shape
 (independent sequences; no collective on the data path), timing is the max
@@ -39,8 +40,15 @@ METRIC = "keys scored+selected+compacted/sec per B200 and % of HBM roofline"
 UNIT = "keys/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-SCORE_BYTES_PER_KEY = 256 + 4  # read the bf16 key, write its fp32 score
-KEPT_BYTES = 4 * 256 + 8  # read + write K and V of a kept key, read + write its position
+ELEM_BYTES = {"bf16": 2, "fp8": 1}
+
+
+def score_bytes_per_key(eb: int) -> int:
+    return 128 * eb + 4  # read the key, write its fp32 score
+
+
+def kept_bytes(eb: int) -> int:
+    return 4 * 128 * eb + 8  # read + write K and V of a kept key, read + write its position
 
 
 def parse():
@@ -54,6 +62,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=None,
                     help="first N layers only (small cases for profiling; not a bench line)")
     ap.add_argument("--key-mode", choices=["post", "pre"], default="post")
+    ap.add_argument("--elem", choices=sorted(ELEM_BYTES), default="bf16",
+                    help="K/V cache element type (fp8 = OCP e4m3, converted from the bf16 cache)")
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="timed steps replay CUDA graphs of the calls (default) or call eagerly")
     ap.add_argument("--no-e2e", action="store_true")
@@ -64,16 +74,17 @@ def parse():
     return a
 
 
-def workload_config(wl, B, key_mode, launch="eager"):
+def workload_config(wl, B, key_mode, launch="eager", elem="bf16"):
     lo, hi = wl.seq_len
+    eb = ELEM_BYTES[elem]
     return {"workload": wl.name, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "rope_theta": wl.theta,
             "batch": wl.batch, "keys_per_head": lo if lo == hi else [lo, hi], "budget": B,
             "window": wl.window, "offsets": wl.n_offsets, "key_mode": key_mode + "_rope",
             "launch": launch,
-            "layout": wl.layout,
+            "layout": wl.layout, "kv_elem": elem,
             "l2": "inputs larger than L2: K+V %.1f GB read per step, no flush" % (
-                2 * 256 * wl.n_layers * wl.batch * wl.n_kv_heads * np.mean(wl.seq_len) / 1e9)}
+                2 * 128 * eb * wl.n_layers * wl.batch * wl.n_kv_heads * np.mean(wl.seq_len) / 1e9)}
 
 
 def measured_peak():
@@ -93,18 +104,19 @@ def score_kernel_sha():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(total_keys):
+def recorded_traffic(total_keys, elem="bf16"):
     """DRAM bytes per launch of the score kernel from the committed ncu summary, if it
-    was taken on the current kernel source; else None."""
+    was taken on the current kernel source for this element type; else None."""
     path = os.path.join(ROOT, "profiles", "score_kernel_traffic.json")
     try:
         with open(path) as fh:
             rec = json.load(fh)
     except Exception:
         return None
-    if rec.get("kernel_sha") != score_kernel_sha():
+    per = rec.get("by_elem", {}).get(elem)
+    if rec.get("kernel_sha") != score_kernel_sha() or per is None:
         return None
-    return float(rec["dram_bytes_per_key"]) * total_keys
+    return float(per["dram_bytes_per_key"]) * total_keys
 
 
 class ClockSampler:
@@ -205,10 +217,15 @@ def run_ours(a, rank, world, local_rank):
     if wl.layout != "contig":
         raise SystemExit("bench.py times the contiguous workloads; the paged one is a parity case")
     cache = synth.make_contig(wl, dev, rotate=(a.key_mode == "post"))
+    eb = ELEM_BYTES[a.elem]
+    if a.elem == "fp8":
+        cache.K = synth.to_fp8(cache.K)
+        cache.V = synth.to_fp8(cache.V)
+        torch.cuda.empty_cache()
     L, S, Hh = wl.n_layers, len(cache.lens), wl.n_kv_heads
     R, total = cache.n_rows, cache.total
     m = tri.model(L, wl.n_q_heads, Hh, wl.theta)
-    kv = tri.kv_contig(S, cache.row_off, total)
+    kv = tri.kv_contig(S, cache.row_off, total, tri.elem_type_of(cache.K))
     stream = torch.cuda.current_stream(dev)
 
     # offline calibration (timed separately, not part of a step)
@@ -225,7 +242,7 @@ def run_ours(a, rank, world, local_rank):
 
     ws = tri.alloc_workspace(m, S, B, device=dev)
     scores = torch.empty(total, dtype=torch.float32, device=dev)
-    Ko = torch.empty(R, B, 128, dtype=torch.bfloat16, device=dev)
+    Ko = torch.empty(R, B, 128, dtype=cache.K.dtype, device=dev)
     Vo = torch.empty_like(Ko)
     po = torch.empty(R, B, dtype=torch.int32, device=dev)
     kept = torch.empty(R, B, dtype=torch.int32, device=dev)
@@ -291,7 +308,7 @@ def run_ours(a, rank, world, local_rank):
 
     lens_rows = np.diff(cache.row_off_np)
     keys_step = int(total)
-    alg_bytes = float(np.sum(256.0 * lens_rows + np.minimum(lens_rows, B) * KEPT_BYTES))
+    alg_bytes = float(np.sum(128.0 * eb * lens_rows + np.minimum(lens_rows, B) * kept_bytes(eb)))
     if key_mode == tri.TRI_KEYS_PRE_ROPE:
         alg_bytes += 4.0 * total
     ms_step = ms / a.steps
@@ -304,16 +321,16 @@ def run_ours(a, rank, world, local_rank):
                       world, dev)
 
     peak, peak_kind = measured_peak()
-    score_bytes = SCORE_BYTES_PER_KEY * total
+    score_bytes = score_bytes_per_key(eb) * total
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     path_gbs = alg_bytes / (ms_step / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(wl, B, a.key_mode, "cuda_graph" if a.launch == "graph" else "eager"),
+        "config": workload_config(wl, B, a.key_mode, "cuda_graph" if a.launch == "graph" else "eager", a.elem),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(total),
+                     "frac": achieved / peak, "traffic": recorded_traffic(total, a.elem),
                      "kernel": "tri_score (prep + score kernels)", "peak_kind": peak_kind,
                      "bytes_per_launch": score_bytes, "ms_per_launch": score_ms},
         "path_roofline": {"bytes_per_step": alg_bytes, "achieved_gbs": path_gbs,
@@ -380,6 +397,7 @@ def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, 
 # ------------------------------------------------------- CPU oracle leg
 
 def oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs, ms, rows_meta, seconds, max_rows):
+    """K_rows/V_rows hold the stored bits (int16 for bf16, uint8 for fp8)."""
     """Time the oracle (collapsed score + select + gather) on rows until `seconds` pass."""
     import oracle
 
@@ -389,7 +407,8 @@ def oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs, ms, rows_meta, seconds, m
     for i in range(max_rows):
         j = i % len(rows_meta)
         h, p_now = rows_meta[j]
-        Kf = oracle.bf16_bits_to_f64(K_rows[j])
+        Kb = K_rows[j]
+        Kf = oracle.e4m3_bits_to_f64(Kb) if Kb.dtype == np.uint8 else oracle.bf16_bits_to_f64(Kb)
         s = oracle.row_scores(wl.theta, cs, ms, h, wl.group, Kf, pos_rows[j], True, p_now, wl.offsets,
                               "collapsed")
         kept = oracle.select(s, B, wl.window)
@@ -413,8 +432,8 @@ def cpu_baseline(wl, B, cache, seconds):
     K_rows, V_rows, pos_rows, meta = [], [], [], []
     for r in rows:
         a, b = cache.row_off_np[r], cache.row_off_np[r + 1]
-        K_rows.append(H.bits16(cache.K[a:b]))
-        V_rows.append(H.bits16(cache.V[a:b]))
+        K_rows.append(H.raw_bits(cache.K[a:b]))
+        V_rows.append(H.raw_bits(cache.V[a:b]))
         pos_rows.append(cache.pos[a:b].cpu().numpy().astype(np.int64))
         _, s, h = cache.row_lhs(r)
         meta.append((h, int(cache.lens[s])))
@@ -433,12 +452,15 @@ def run_reference(a, rank, world):
     B = a.budget or wl0.budget
     wl = wl0.with_(budget=B)
     cache = synth.make_contig(wl, "cpu", layers=[0], lens=wl.seq_lengths()[:1])
+    if a.elem == "fp8":
+        cache.K = synth.to_fp8(cache.K)
+        cache.V = synth.to_fp8(cache.V)
     Hh = wl.n_kv_heads
     K_rows, V_rows, pos_rows, meta = [], [], [], []
     for r in range(Hh):
         a_, b_ = cache.row_off_np[r], cache.row_off_np[r + 1]
-        K_rows.append(H.bits16(cache.K[a_:b_]))
-        V_rows.append(H.bits16(cache.V[a_:b_]))
+        K_rows.append(H.raw_bits(cache.K[a_:b_]))
+        V_rows.append(H.raw_bits(cache.V[a_:b_]))
         pos_rows.append(cache.pos[a_:b_].numpy().astype(np.int64))
         meta.append((r % Hh, int(cache.lens[0])))
     cs, ms = H.oracle_calibration(cache.qcal)
@@ -458,7 +480,7 @@ def run_reference(a, rank, world):
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": workload_config(wl, B, "post", "cuda_graph" if a.launch == "graph" else "eager"),
+            "config": workload_config(wl, B, "post", "cuda_graph" if a.launch == "graph" else "eager", a.elem),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -64,6 +64,7 @@ typedef enum {
 #define TRI_HEAD_DIM 128
 
 enum { TRI_KV_CONTIG = 0, TRI_KV_PAGED = 1 };
+enum { TRI_ELEM_BF16 = 0, TRI_ELEM_FP8_E4M3 = 1 }; /* K/V element type */
 enum { TRI_KEYS_POST_ROPE = 0, TRI_KEYS_PRE_ROPE = 1 };
 
 typedef struct {
@@ -76,10 +77,10 @@ typedef struct {
 
 /*
  * Where the cached keys of each row live.
- *  TRI_KV_CONTIG: K is [total_keys][d] bf16 and pos is [total_keys] int32; row r
+ *  TRI_KV_CONTIG: K is [total_keys][d] (elem_type) and pos is [total_keys] int32; row r
  *    is entries row_off[r] .. row_off[r+1]-1 (rows of any length, in row order).
  *  TRI_KV_PAGED (vLLM block layout): K is [n_layers][n_blocks][block_size][H][d]
- *    bf16 and pos is [n_layers][n_blocks][block_size][H] int32; slot j of
+ *    (elem_type) and pos is [n_layers][n_blocks][block_size][H] int32; slot j of
  *    sequence s is slot j % block_size of block block_table[s][j / block_size],
  *    the same table for every layer.  row_off then only describes the score
  *    buffer (row r's scores are entries row_off[r] .. row_off[r+1]-1) and the
@@ -96,6 +97,13 @@ typedef struct {
     int32_t max_blocks;         /* >= 1 */
     int32_t block_size;         /* power of two, 1 .. 1024 (vLLM: 16) */
     int64_t n_blocks;           /* blocks per layer in the pool, >= 1 */
+    /* Element type of K and V (and of the compacted outputs): TRI_ELEM_BF16
+     * (2 bytes, the default of a zeroed descriptor) or TRI_ELEM_FP8_E4M3 (1 byte,
+     * OCP e4m3 "fn": no infinities, 0x7f/0xff are NaN).  fp8 values are scored as
+     * stored: a per-tensor dequantisation scale multiplies every score of a row
+     * equally and leaves the selection unchanged. */
+    int32_t elem_type;
+    int32_t pad_;
 } tri_kv_desc;
 
 /*
@@ -157,7 +165,7 @@ tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *ce
  * Score every cached key (digest, 流程详解 steps 2-3) with the rule in the
  * header comment, the GQA mean taken over the query heads of each KV head.
  *   kv:        layout and row offsets of the cache
- *   K:         bf16 keys in kv's layout, 16-byte aligned
+ *   K:         keys (kv->elem_type) in kv's layout, 16-byte aligned
  *   pos:       int32 position of every cached slot (kv's layout).  Read only
  *              for TRI_KEYS_PRE_ROPE; may be NULL for TRI_KEYS_POST_ROPE.
  *   centres, mean_norm: calibration of tri_calib, [n_layers][n_q_heads][64](x2);

@@ -18,8 +18,8 @@ import ctypes
 import torch
 
 from . import _abi
-from ._abi import (TRI_FLAG_BLOCK_TABLE, TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS,  # noqa: F401
-                   TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
+from ._abi import (TRI_ELEM_BF16, TRI_ELEM_FP8_E4M3, TRI_FLAG_BLOCK_TABLE,  # noqa: F401
+                   TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS, TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
                    TRI_MAX_OFFSETS, TriKvDesc, TriModel, TriOutDesc)
 
 _L = _abi.load()
@@ -67,18 +67,30 @@ def model(n_layers: int, n_q_heads: int, n_kv_heads: int, rope_theta: float,
 # A descriptor holds raw device pointers; it also keeps a reference to the tensors
 # they point into, so the memory cannot be freed (and reused) while it is alive.
 
-def kv_contig(n_seqs: int, row_off: torch.Tensor, total_keys: int) -> TriKvDesc:
+def elem_type_of(t: torch.Tensor) -> int:
+    """TRI_ELEM_* of a K/V tensor (bf16 or float8_e4m3fn)."""
+    if t.dtype == torch.bfloat16:
+        return TRI_ELEM_BF16
+    if t.dtype == torch.float8_e4m3fn:
+        return TRI_ELEM_FP8_E4M3
+    raise TypeError(f"unsupported K/V dtype {t.dtype}")
+
+
+def kv_contig(n_seqs: int, row_off: torch.Tensor, total_keys: int,
+              elem_type: int = TRI_ELEM_BF16) -> TriKvDesc:
     """Rows laid end to end; ``row_off`` int64 [R+1] on the device."""
-    d = TriKvDesc(TRI_KV_CONTIG, n_seqs, int(total_keys), row_off.data_ptr(), None, 0, 0, 0)
+    d = TriKvDesc(TRI_KV_CONTIG, n_seqs, int(total_keys), row_off.data_ptr(), None, 0, 0, 0,
+                  int(elem_type), 0)
     d._keep = (row_off,)
     return d
 
 
 def kv_paged(n_seqs: int, row_off: torch.Tensor, total_keys: int, block_table: torch.Tensor,
-             block_size: int, n_blocks: int) -> TriKvDesc:
+             block_size: int, n_blocks: int, elem_type: int = TRI_ELEM_BF16) -> TriKvDesc:
     """vLLM block layout; ``block_table`` int32 [S][max_blocks] on the device."""
     d = TriKvDesc(TRI_KV_PAGED, n_seqs, int(total_keys), row_off.data_ptr(),
-                  block_table.data_ptr(), block_table.shape[1], block_size, int(n_blocks))
+                  block_table.data_ptr(), block_table.shape[1], block_size, int(n_blocks),
+                  int(elem_type), 0)
     d._keep = (row_off, block_table)
     return d
 

@@ -23,6 +23,8 @@ TRI_MAX_OFFSETS = 64
 TRI_HEAD_DIM = 128
 TRI_KV_CONTIG = 0
 TRI_KV_PAGED = 1
+TRI_ELEM_BF16 = 0
+TRI_ELEM_FP8_E4M3 = 1
 TRI_KEYS_POST_ROPE = 0
 TRI_KEYS_PRE_ROPE = 1
 
@@ -42,7 +44,8 @@ class TriKvDesc(ctypes.Structure):
     _fields_ = [("layout", ctypes.c_int32), ("n_seqs", ctypes.c_int32),
                 ("total_keys", ctypes.c_int64), ("row_off", ctypes.c_void_p),
                 ("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int32),
-                ("block_size", ctypes.c_int32), ("n_blocks", ctypes.c_int64)]
+                ("block_size", ctypes.c_int32), ("n_blocks", ctypes.c_int64),
+                ("elem_type", ctypes.c_int32), ("pad_", ctypes.c_int32)]
 
 
 class TriOutDesc(ctypes.Structure):

@@ -61,6 +61,9 @@ tri_status check_kv(const tri_model *m, const tri_kv_desc *kv, Geometry *geo) {
     geo->layout = kv->layout;
     geo->total = kv->total_keys;
     geo->row_off = kv->row_off;
+    if (kv->elem_type == TRI_ELEM_BF16) geo->elem_bytes = 2;
+    else if (kv->elem_type == TRI_ELEM_FP8_E4M3) geo->elem_bytes = 1;
+    else return TRI_ERR_INVALID_ARG;
     if (kv->layout == TRI_KV_PAGED) {
         if (!kv->block_table || kv->max_blocks < 1 || kv->n_blocks < 1) return TRI_ERR_INVALID_ARG;
         if (!aligned(kv->block_table, 4)) return TRI_ERR_ALIGNMENT;
@@ -178,7 +181,7 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
 
     ScoreParams sp;
     sp.geo = geo;
-    sp.K = (const uint16_t *)K;
+    sp.K = (const char *)K;
     sp.pos = pos;
     sp.p_now = p_now;
     sp.coef = pp.coef;
@@ -239,11 +242,11 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
     gp.out_table = out->block_table;
     gp.B = B;
     gp.kept = kept;
-    gp.K = (const uint16_t *)K;
-    gp.V = (const uint16_t *)V;
+    gp.K = (const char *)K;
+    gp.V = (const char *)V;
     gp.pos = pos_out ? pos : nullptr;
-    gp.K_out = (uint16_t *)K_out;
-    gp.V_out = (uint16_t *)V_out;
+    gp.K_out = (char *)K_out;
+    gp.V_out = (char *)V_out;
     gp.pos_out = pos_out;
     gp.flags = sp.flags;
     return cuda_status(launch_gather(gp, s), "gather_kernel launch");

@@ -2,9 +2,10 @@
 // order, into the output cache ("TriAttention：基于三角函数 KV 压缩的高效长推理",
 // 流程详解 step 4: later attention reads only the compressed cache).
 //
-// Flat grid over (row, 64-slot chunk).  A half-warp moves one 256-byte key
-// record as 16 x 16-byte vectors, so each warp instruction copies two whole
-// records; every thread keeps 4 K and 4 V vectors in flight.  Source reads
+// Flat grid over (row, chunk of kept slots).  A record (one key or value: 256
+// bytes in bf16, 128 in fp8) is moved as 16-byte vectors by 16 (8) lanes, so
+// each warp instruction copies two (four) whole records; every thread keeps 4
+// K and 4 V vectors in flight.  Source reads
 // bypass L1; destination writes are streaming stores (not re-read here).
 // Paged input and/or output addresses go through the block tables.
 #include "tri_internal.cuh"
@@ -12,9 +13,15 @@
 namespace tri {
 
 constexpr int kGatherThreads = 256;
-constexpr int kSlotsPerCta = 64;  // 8 warps x 4 iterations x 2 records
+constexpr int kGatherIters = 4;
 
+// RB: record bytes (128 dims x element size).  A record is moved as RB/16
+// 16-byte vectors by RB/16 lanes, so a warp instruction moves 512 bytes.
+template <int RB>
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherParams p) {
+    constexpr int kLanes = RB / 16;                                       // lanes per record
+    constexpr int kPerWarp = 32 / kLanes;                                 // records per instruction
+    constexpr int kSlotsPerCta = (kGatherThreads / 32) * kGatherIters * kPerWarp;
     grid_dependency_wait();
     grid_dependents_launch();
     const Geometry &geo = p.geo;
@@ -27,17 +34,17 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     const int cnt = (int)min(N, (int64_t)p.B);
     if (base >= cnt) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half = lane >> 4, c = lane & 15;
+    const int sub = lane / kLanes, c = lane % kLanes;
     const int h = (int)(r % geo.H);
     const int s = (int)((r / geo.H) % geo.S);
     const int l = (int)(r / ((int64_t)geo.H * geo.S));
 
-    uint4 kv[4], vv[4];
-    int64_t dst[4];
-    int32_t pv[4];
+    uint4 kv[kGatherIters], vv[kGatherIters];
+    int64_t dst[kGatherIters];
+    int32_t pv[kGatherIters];
 #pragma unroll
-    for (int it = 0; it < 4; it++) {
-        const int i = base + warp * 8 + it * 2 + half;
+    for (int it = 0; it < kGatherIters; it++) {
+        const int i = base + (warp * kGatherIters + it) * kPerWarp + sub;
         dst[it] = -1;
         pv[it] = 0;
         if (i >= cnt) continue;
@@ -67,26 +74,32 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
             continue;
         }
         dst[it] = d;
-        kv[it] = ld_nc16(p.K + src * kD + 8 * c);
-        vv[it] = ld_nc16(p.V + src * kD + 8 * c);
+        kv[it] = ld_nc16(p.K + src * RB + 16 * c);
+        vv[it] = ld_nc16(p.V + src * RB + 16 * c);
         if (p.pos && c == 0) pv[it] = __ldg(p.pos + src);
     }
 #pragma unroll
-    for (int it = 0; it < 4; it++) {
+    for (int it = 0; it < kGatherIters; it++) {
         if (dst[it] < 0) continue;
-        st_stream16(p.K_out + dst[it] * kD + 8 * c, kv[it]);
-        st_stream16(p.V_out + dst[it] * kD + 8 * c, vv[it]);
+        st_stream16(p.K_out + dst[it] * RB + 16 * c, kv[it]);
+        st_stream16(p.V_out + dst[it] * RB + 16 * c, vv[it]);
         if (p.pos_out && c == 0) p.pos_out[dst[it]] = pv[it];
     }
 }
 
-cudaError_t launch_gather(const GatherParams &p, cudaStream_t s) {
+template <int RB>
+static cudaError_t launch_gather_t(const GatherParams &p, cudaStream_t s) {
+    constexpr int kSlotsPerCta = (kGatherThreads / 32) * kGatherIters * (32 / (RB / 16));
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
     const int64_t chunks = (p.B + kSlotsPerCta - 1) / kSlotsPerCta;
     const int64_t grid = R * chunks;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    return launch_pdl(gather_kernel, dim3((unsigned)grid), dim3(kGatherThreads), 0, s, p);
+    return launch_pdl(gather_kernel<RB>, dim3((unsigned)grid), dim3(kGatherThreads), 0, s, p);
+}
+
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t s) {
+    return p.geo.elem_bytes == 1 ? launch_gather_t<kD>(p, s) : launch_gather_t<2 * kD>(p, s);
 }
 
 }  // namespace tri

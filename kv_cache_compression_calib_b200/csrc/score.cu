@@ -85,16 +85,61 @@ __device__ __forceinline__ int64_t key_slot(const ScoreParams &p, const RowCtx &
     return ((((c.layer_blk + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) * geo.H) + c.h;
 }
 
-__device__ __forceinline__ void unpack8(const uint4 v, float (&x)[8]) {
+__device__ __forceinline__ void unpack_bf16x8(const uint4 v, float (&x)[8]) {
     x[0] = bf16lo(v.x); x[1] = bf16hi(v.x); x[2] = bf16lo(v.y); x[3] = bf16hi(v.y);
     x[4] = bf16lo(v.z); x[5] = bf16hi(v.z); x[6] = bf16lo(v.w); x[7] = bf16hi(v.w);
 }
 
+// Two packed e4m3 values (low byte first) to floats: exact via f16.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return __half22float2(__half2(h));
+}
+
+__device__ __forceinline__ void unpack_e4m3x8(const uint2 v, float (&x)[8]) {
+    const float2 a = e4m3x2_to_float2(v.x), b = e4m3x2_to_float2(v.x >> 16);
+    const float2 c = e4m3x2_to_float2(v.y), d = e4m3x2_to_float2(v.y >> 16);
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
+}
+
+// Lane g's share of one key record: the real parts (dims 8g..8g+7) and the
+// imaginary parts (dims 64+8g..64+8g+7) of pairs 8g..8g+7, as stored - 2 x 16
+// bytes for bf16, 2 x 8 bytes for fp8 e4m3.  A warp instruction covers four
+// keys' halves, each a contiguous 128 (bf16) or 64 (fp8) bytes.
+template <int ELEM>
+struct KeyChunk;
+
+template <>
+struct KeyChunk<2> {
+    uint4 re, im;
+    __device__ __forceinline__ void load(const char *key, int g, unsigned long long pol) {
+        re = ld_stream16(key + 16 * g, pol);
+        im = ld_stream16(key + 2 * kF + 16 * g, pol);
+    }
+    __device__ __forceinline__ void zero() { re = im = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
+        unpack_bf16x8(re, x);
+        unpack_bf16x8(im, y);
+    }
+};
+
+template <>
+struct KeyChunk<1> {
+    uint2 re, im;
+    __device__ __forceinline__ void load(const char *key, int g, unsigned long long pol) {
+        re = ld_stream8(key + 8 * g, pol);
+        im = ld_stream8(key + kF + 8 * g, pol);
+    }
+    __device__ __forceinline__ void zero() { re = im = make_uint2(0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
+        unpack_e4m3x8(re, x);
+        unpack_e4m3x8(im, y);
+    }
+};
+
 // Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|.
-__device__ __forceinline__ float partial_post(const uint4 re, const uint4 im, const RowCtx &c) {
-    float x[8], y[8];
-    unpack8(re, x);
-    unpack8(im, y);
+__device__ __forceinline__ float partial_post(const float (&x)[8], const float (&y)[8], const RowCtx &c) {
     float a0 = 0.f, a1 = 0.f, a2 = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; i++) {
@@ -108,11 +153,8 @@ __device__ __forceinline__ float partial_post(const uint4 re, const uint4 im, co
 // Pre-RoPE cache: rotate A'_i by w_i (p_now - pos) first.  The phase in turns
 // is (delta * T_i) mod 2^64 with T_i = w_i / 2pi in 0.64 fixed point; its top
 // 32 bits as a signed integer are the angle in [-pi, pi).
-__device__ __forceinline__ float partial_pre(const uint4 re, const uint4 im, const RowCtx &c,
+__device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&y)[8], const RowCtx &c,
                                              const unsigned long long (&T)[8], int64_t delta) {
-    float x[8], y[8];
-    unpack8(re, x);
-    unpack8(im, y);
     float a0 = 0.f, a1 = 0.f, a2 = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; i++) {
@@ -129,7 +171,15 @@ __device__ __forceinline__ float partial_pre(const uint4 re, const uint4 im, con
     return (a0 + a1) + a2;
 }
 
-template <bool PAGED, bool PRE>
+template <bool PRE, int ELEM>
+__device__ __forceinline__ float chunk_partial(const KeyChunk<ELEM> &kc, const RowCtx &c,
+                                               const unsigned long long (&T)[8], int64_t delta) {
+    float x[8], y[8];
+    kc.unpack(x, y);
+    return PRE ? partial_pre(x, y, c, T, delta) : partial_post(x, y, c);
+}
+
+template <bool PAGED, bool PRE, int ELEM>
 __device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx &c, int64_t k, int g,
                                              unsigned long long pol, const unsigned long long (&T)[8]) {
     const int64_t slot = key_slot<PAGED>(p, c, k);
@@ -137,14 +187,13 @@ __device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx 
         atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
         return 0.f;
     }
-    const uint16_t *kp = p.K + slot * kD + 8 * g;
-    const uint4 re = ld_stream16(kp, pol);
-    const uint4 im = ld_stream16(kp + kF, pol);
-    if (PRE) return partial_pre(re, im, c, T, c.p_now - (int64_t)__ldg(p.pos + slot));
-    return partial_post(re, im, c);
+    KeyChunk<ELEM> kc;
+    kc.load(p.K + slot * (kD * ELEM), g, pol);
+    const int64_t delta = PRE ? c.p_now - (int64_t)__ldg(p.pos + slot) : 0;
+    return chunk_partial<PRE, ELEM>(kc, c, T, delta);
 }
 
-template <bool PAGED, bool PRE>
+template <bool PAGED, bool PRE, int ELEM>
 __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const ScoreParams p) {
     grid_dependency_wait();
     grid_dependents_launch();
@@ -184,20 +233,17 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
         float part[8];
         if (bend == b0 + 32 && b0 >= c.lo && bend <= c.hi) {
             // Whole batch inside the current row: issue all 16 loads, then compute.
-            uint4 re[8], im[8];
+            KeyChunk<ELEM> kc[8];
             int64_t slot[8];
             int32_t kpos[8];
 #pragma unroll
             for (int u = 0; u < 8; u++) {
                 slot[u] = key_slot<PAGED>(p, c, b0 + 4 * u + q);
                 if (slot[u] >= 0) {
-                    const uint16_t *kp = p.K + slot[u] * kD + 8 * g;
-                    re[u] = ld_stream16(kp, pol);
-                    im[u] = ld_stream16(kp + kF, pol);
+                    kc[u].load(p.K + slot[u] * (kD * ELEM), g, pol);
                     kpos[u] = PRE ? __ldg(p.pos + slot[u]) : 0;
                 } else {
-                    re[u] = make_uint4(0, 0, 0, 0);
-                    im[u] = re[u];
+                    kc[u].zero();
                     kpos[u] = 0;
                 }
             }
@@ -206,10 +252,8 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
                 if (PAGED && slot[u] < 0) {
                     atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
                     part[u] = 0.f;
-                } else if (PRE) {
-                    part[u] = partial_pre(re[u], im[u], c, T, c.p_now - (int64_t)kpos[u]);
                 } else {
-                    part[u] = partial_post(re[u], im[u], c);
+                    part[u] = chunk_partial<PRE, ELEM>(kc[u], c, T, c.p_now - (int64_t)kpos[u]);
                 }
             }
         } else {
@@ -222,7 +266,7 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
 #pragma unroll
                 for (int u = 0; u < 8; u++) {
                     const int64_t k = b0 + 4 * u + q;
-                    if (k >= k0 && k < seg_end) part[u] += key_partial<PAGED, PRE>(p, c, k, g, pol, T);
+                    if (k >= k0 && k < seg_end) part[u] += key_partial<PAGED, PRE, ELEM>(p, c, k, g, pol, T);
                 }
                 if (bend <= c.hi) break;
                 k0 = max(k0, c.hi);
@@ -263,14 +307,15 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
     }
 }
 
-template <bool PAGED, bool PRE>
+template <bool PAGED, bool PRE, int ELEM>
 static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
     static int occ[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     int &o = occ[dev & 63];
     if (o == 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_kernel<PAGED, PRE>, kScoreThreads, 0);
+        cudaError_t e =
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_kernel<PAGED, PRE, ELEM>, kScoreThreads, 0);
         if (e != cudaSuccess) return e;
         if (o < 1) o = 1;
     }
@@ -278,14 +323,19 @@ static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
     int64_t grid = (int64_t)sm_count() * o;
     if (want < grid) grid = want;
     if (grid < 1) grid = 1;
-    return launch_pdl(score_kernel<PAGED, PRE>, dim3((unsigned)grid), dim3(kScoreThreads), 0, s, p);
+    return launch_pdl(score_kernel<PAGED, PRE, ELEM>, dim3((unsigned)grid), dim3(kScoreThreads), 0, s, p);
+}
+
+template <int ELEM>
+static cudaError_t launch_score_e(const ScoreParams &p, int pre_rope, cudaStream_t s) {
+    const bool paged = p.geo.layout == TRI_KV_PAGED;
+    if (paged) return pre_rope ? launch_score_t<true, true, ELEM>(p, s) : launch_score_t<true, false, ELEM>(p, s);
+    return pre_rope ? launch_score_t<false, true, ELEM>(p, s) : launch_score_t<false, false, ELEM>(p, s);
 }
 
 cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s) {
     if (p.geo.total <= 0) return cudaSuccess;
-    const bool paged = p.geo.layout == TRI_KV_PAGED;
-    if (paged) return pre_rope ? launch_score_t<true, true>(p, s) : launch_score_t<true, false>(p, s);
-    return pre_rope ? launch_score_t<false, true>(p, s) : launch_score_t<false, false>(p, s);
+    return p.geo.elem_bytes == 1 ? launch_score_e<1>(p, pre_rope, s) : launch_score_e<2>(p, pre_rope, s);
 }
 
 }  // namespace tri

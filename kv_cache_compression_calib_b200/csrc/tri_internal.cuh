@@ -4,6 +4,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include <utility>
 
 #include "tri.h"
@@ -28,6 +31,7 @@ inline size_t ws_total(int64_t R, int64_t B) {
 struct Geometry {  // row numbering and cache addressing
     int32_t L, S, H, Hq, G;
     int32_t layout;
+    int32_t elem_bytes;  // 2: bf16, 1: fp8 e4m3
     int32_t max_blocks, block_shift;  // paged: block_size = 1 << block_shift
     int64_t n_blocks;
     int64_t total;
@@ -51,7 +55,7 @@ struct PrepParams {
 
 struct ScoreParams {
     Geometry geo;
-    const uint16_t *K;
+    const char *K;
     const int32_t *pos;
     const int64_t *p_now;
     const float *coef;
@@ -77,9 +81,9 @@ struct GatherParams {
     const int32_t *out_table;
     int32_t B;
     const int32_t *kept;
-    const uint16_t *K, *V;
+    const char *K, *V;
     const int32_t *pos;
-    uint16_t *K_out, *V_out;
+    char *K_out, *V_out;
     int32_t *pos_out;
     unsigned *flags;
 };
@@ -150,6 +154,15 @@ __device__ __forceinline__ uint4 ld_stream16(const void *ptr, unsigned long long
     uint4 v;
     asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr), "l"(pol));
+    return v;
+}
+
+// 8-byte variant of ld_stream16.
+__device__ __forceinline__ uint2 ld_stream8(const void *ptr, unsigned long long pol) {
+    uint2 v;
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
+        : "=r"(v.x), "=r"(v.y)
         : "l"(ptr), "l"(pol));
     return v;
 }

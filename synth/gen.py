@@ -272,3 +272,11 @@ def decode_keys(wl: Workload, layer: int, round_idx: int, start: np.ndarray, cou
             Kn[s, :, h] = head_keys(heads, h, p, g, wl.theta, d, True)
             Vn[s, :, h] = torch.randn(count, d, generator=g, device=device).to(torch.bfloat16)
     return Kn, Vn
+
+
+FP8_MAX = 448.0  # largest finite OCP e4m3 value
+
+
+def to_fp8(t: torch.Tensor) -> torch.Tensor:
+    """The cache as an fp8 e4m3 cache would store it: clamp to +-448, round to nearest."""
+    return t.float().clamp_(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn)

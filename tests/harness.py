@@ -16,8 +16,17 @@ def bits16(t: torch.Tensor) -> np.ndarray:
     return t.detach().contiguous().view(torch.int16).cpu().numpy()
 
 
+def raw_bits(t: torch.Tensor) -> np.ndarray:
+    """Stored bits of a K/V tensor: int16 per bf16 element, uint8 per fp8 element."""
+    if t.dtype == torch.float8_e4m3fn:
+        return t.detach().contiguous().view(torch.uint8).cpu().numpy()
+    return bits16(t)
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
-    """Exact widening of a bf16 tensor's bits to float64 (host)."""
+    """Exact widening of a bf16 or fp8 e4m3 tensor's bits to float64 (host)."""
+    if t.dtype == torch.float8_e4m3fn:
+        return oracle.e4m3_bits_to_f64(raw_bits(t))
     return oracle.bf16_bits_to_f64(bits16(t))
 
 

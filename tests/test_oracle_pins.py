@@ -369,3 +369,14 @@ def test_bf16_widening_is_exact():
     assert got[4] == float(np.float32(3.3895313892515355e38))
     assert got[5] == 2.0 ** -133
     assert got[6] == 3.140625
+
+
+def test_e4m3_decoding_matches_definition_and_torch():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_bits_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref)) and np.isnan(got).sum() == 2
+    np.testing.assert_array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+    # hand-checked codes: 1.0, the largest finite 448, the smallest subnormal 2^-9, -2
+    assert got[0x38] == 1.0 and got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0xC0] == -2.0
