@@ -61,10 +61,10 @@ def _declare(L) -> None:
     L.ora_num_threads.restype = ctypes.c_int
     L.ora_num_threads.argtypes = []
     L.ora_trig_series.restype = ctypes.c_double
-    L.ora_trig_series.argtypes = [ctypes.c_int, ctypes.c_double, _f64p, _f64p, ctypes.c_int64]
+    L.ora_trig_series.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double, _f64p, _f64p, ctypes.c_int64]
     L.ora_calib.restype = None
-    L.ora_calib.argtypes = [ctypes.c_int, ctypes.c_int64, _f64p, _f64p, _f64p]
-    score_args = [ctypes.c_int, ctypes.c_double, ctypes.c_int, _f64p, _f64p, ctypes.c_int64,
+    L.ora_calib.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, _f64p, _f64p, _f64p]
+    score_args = [ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, _f64p, _f64p, ctypes.c_int64,
                   _f64p, _i64p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, _i64p, _f64p]
     for name in ("ora_score_literal", "ora_score_collapsed", "ora_score_absorbed"):
         fn = getattr(L, name)
@@ -115,13 +115,17 @@ def omega(theta: float, d: int) -> np.ndarray:
     return np.array([lib().ora_omega(theta, d, f) for f in range(d // 2)])
 
 
-def trig_series(theta: float, qbar: np.ndarray, k_pre: np.ndarray, dist: int) -> float:
-    """sum_f |qbar_f||k_f| cos(w_f dist + arg qbar_f - arg k_f); qbar [F][2], k_pre [d]."""
+def trig_series(theta: float, qbar: np.ndarray, k_pre: np.ndarray, dist: int,
+                interleaved: bool = False) -> float:
+    """sum_f |qbar_f||k_f| cos(w_f dist + arg qbar_f - arg k_f); qbar [F][2], k_pre [d].
+
+    Pair f is dims (f, f+d/2) (rotate-half), or (2f, 2f+1) when ``interleaved``."""
     k_pre = _f64(k_pre)
-    return float(lib().ora_trig_series(k_pre.shape[0], theta, _f64(qbar), k_pre, int(dist)))
+    return float(lib().ora_trig_series(k_pre.shape[0], int(bool(interleaved)), theta, _f64(qbar), k_pre,
+                                       int(dist)))
 
 
-def calib(q: np.ndarray):
+def calib(q: np.ndarray, interleaved: bool = False):
     """Per-pair complex centre and mean magnitude of pre-RoPE queries q [nq][d].
 
     Returns (centre [F][2], mnorm [F])."""
@@ -129,11 +133,11 @@ def calib(q: np.ndarray):
     nq, d = q.shape
     centre = np.empty((d // 2, 2))
     mnorm = np.empty(d // 2)
-    lib().ora_calib(d, nq, q, centre, mnorm)
+    lib().ora_calib(d, int(bool(interleaved)), nq, q, centre, mnorm)
     return centre, mnorm
 
 
-def _score(fn, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets):
+def _score(fn, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets, interleaved=False):
     qbar = _f64(qbar)
     mnorm = _f64(mnorm)
     keys = _f64(keys)
@@ -144,26 +148,30 @@ def _score(fn, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets):
     assert pos.shape == (n,)
     offs = _i64(offsets)
     out = np.empty(n)
-    fn(d, float(theta), G, qbar, mnorm, n, keys, pos, 1 if post_rope else 0, int(p_now),
-       offs.shape[0], offs, out)
+    fn(d, int(bool(interleaved)), float(theta), G, qbar, mnorm, n, keys, pos, 1 if post_rope else 0,
+       int(p_now), offs.shape[0], offs, out)
     return out
 
 
-def score_literal(theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets) -> np.ndarray:
+def score_literal(theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets,
+                  interleaved=False) -> np.ndarray:
     """Literal triple sum (g, f, delta).  qbar [G][F][2], mnorm [G][F], keys [n][d]."""
-    return _score(lib().ora_score_literal, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets)
+    return _score(lib().ora_score_literal, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets,
+                  interleaved)
 
 
-def score_collapsed(theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets) -> np.ndarray:
+def score_collapsed(theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets,
+                    interleaved=False) -> np.ndarray:
     """Delta sum folded by angle addition: one (cos, sin) per (key, g, f)."""
     return _score(lib().ora_score_collapsed, theta, qbar, mnorm, keys, pos, post_rope, p_now,
-                  offsets)
+                  offsets, interleaved)
 
 
-def score_absorbed(theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets) -> np.ndarray:
+def score_absorbed(theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets,
+                   interleaved=False) -> np.ndarray:
     """Linear form sum_f Re(A_f conj k_f) + c_f |k_f| (identity cross-check only)."""
     return _score(lib().ora_score_absorbed, theta, qbar, mnorm, keys, pos, post_rope, p_now,
-                  offsets)
+                  offsets, interleaved)
 
 
 def select(score: np.ndarray, B: int, W: int) -> np.ndarray:
@@ -191,7 +199,7 @@ def gather(src: np.ndarray, idx: np.ndarray) -> np.ndarray:
 
 
 def row_scores(theta, centres, mnorms, h, G, keys, pos, post_rope, p_now, offsets,
-               tier: str = "collapsed") -> np.ndarray:
+               tier: str = "collapsed", interleaved: bool = False) -> np.ndarray:
     """Scores of one cache row of KV head ``h``: query heads h*G .. h*G+G-1 of one layer.
 
     centres [Hq][F][2], mnorms [Hq][F] (one layer); keys [n][d] float64.
@@ -200,4 +208,4 @@ def row_scores(theta, centres, mnorms, h, G, keys, pos, post_rope, p_now, offset
     qb = _f64(centres)[h * G:(h + 1) * G]
     mn = _f64(mnorms)[h * G:(h + 1) * G]
     fn = {"literal": score_literal, "collapsed": score_collapsed, "absorbed": score_absorbed}[tier]
-    return fn(theta, qb, mn, keys, pos, post_rope, p_now, offsets)
+    return fn(theta, qb, mn, keys, pos, post_rope, p_now, offsets, interleaved)

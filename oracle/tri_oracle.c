@@ -31,8 +31,8 @@
  *    w_f = theta^(-2f/d),  phi_f^g = arg qbar_f^g - arg k_f,
  *
  *  with k the pre-RoPE key at position j, pairs (f, f + d/2) (rotate-half
- *  RoPE), g over the G query heads of one KV head, and delta over the offset
- *  set.  Selection keeps the last W slots plus the top (B - W) of the rest,
+ *  RoPE) or (2f, 2f + 1) (interleaved RoPE), g over the G query heads of one
+ *  KV head, and delta over the offset set.  Selection keeps the last W slots plus the top (B - W) of the rest,
  *  ordered by (score descending, slot descending); compaction is a stable
  *  gather by the kept slots.
  */
@@ -64,13 +64,28 @@ int ora_num_threads(void)
 #endif
 }
 
+/* The two dimensions of frequency pair f: (f, f + d/2) for rotate-half RoPE
+ * (GPT-NeoX / Llama-HF / Qwen layout), (2f, 2f + 1) for interleaved RoPE
+ * (GPT-J / Meta-Llama complex layout).  The first is the real part. */
+static void pair_dims(int d, int interleaved, int f, int *ire, int *iim)
+{
+    if (interleaved) {
+        *ire = 2 * f;
+        *iim = 2 * f + 1;
+    } else {
+        *ire = f;
+        *iim = f + d / 2;
+    }
+}
+
 /* Pre-RoPE pair f of a cached key.  post_rope != 0: the cache holds
  * k_post_f = k_pre_f * e^{i w_f pos}, so multiply by e^{-i w_f pos}. */
-static void key_pair(int d, const double *key, int f, int post_rope, ldbl w,
+static void key_pair(int d, int il, const double *key, int f, int post_rope, ldbl w,
                      int64_t pos, ldbl *re, ldbl *im)
 {
-    const int F = d / 2;
-    ldbl xr = key[f], xi = key[f + F];
+    int ire, iim;
+    pair_dims(d, il, f, &ire, &iim);
+    ldbl xr = key[ire], xi = key[iim];
     if (post_rope) {
         ldbl a = w * (ldbl)pos;
         ldbl c = cosl(a), s = sinl(a);
@@ -85,18 +100,20 @@ static void key_pair(int d, const double *key, int f, int post_rope, ldbl w,
 /*
  * One term of the trigonometric series, for one query centre and one key:
  *   T = sum_f |qbar_f| |k_f| cos(w_f * dist + arg qbar_f - arg k_f)
- * qbar: [F][2] (re, im); k: [d] pre-RoPE key in rotate-half layout.
+ * qbar: [F][2] (re, im); k: [d] pre-RoPE key, pairs as pair_dims(il).
  * This is the pre-RoPE form of the q.k logit at token distance `dist`
  * (digest, 流程详解 step 2).
  */
-double ora_trig_series(int d, double theta, const double *qbar, const double *k, int64_t dist)
+double ora_trig_series(int d, int il, double theta, const double *qbar, const double *k, int64_t dist)
 {
     const int F = d / 2;
     ldbl s = 0.0L;
     for (int f = 0; f < F; f++) {
         ldbl w = omega_l(theta, d, f);
         ldbl qr = qbar[2 * f], qi = qbar[2 * f + 1];
-        ldbl kr = k[f], ki = k[f + F];
+        int ire, iim;
+        pair_dims(d, il, f, &ire, &iim);
+        ldbl kr = k[ire], ki = k[iim];
         ldbl phi = atan2l(qi, qr) - atan2l(ki, kr);
         s += hypotl(qr, qi) * hypotl(kr, ki) * cosl(w * (ldbl)dist + phi);
     }
@@ -107,15 +124,18 @@ double ora_trig_series(int d, double theta, const double *qbar, const double *k,
  * Calibration (digest, 流程详解 step 1): per frequency pair f of one query
  * head, the complex mean of the pre-RoPE queries and the mean of their
  * magnitudes.
- *   q: [nq][d] pre-RoPE queries; centre: [F][2]; mnorm: [F].
+ *   q: [nq][d] pre-RoPE queries (pairs as pair_dims(il)); centre: [F][2];
+ *   mnorm: [F].
  */
-void ora_calib(int d, int64_t nq, const double *q, double *centre, double *mnorm)
+void ora_calib(int d, int il, int64_t nq, const double *q, double *centre, double *mnorm)
 {
     const int F = d / 2;
     for (int f = 0; f < F; f++) {
         ldbl sr = 0.0L, si = 0.0L, sn = 0.0L;
+        int ire, iim;
+        pair_dims(d, il, f, &ire, &iim);
         for (int64_t t = 0; t < nq; t++) {
-            ldbl xr = q[t * d + f], xi = q[t * d + f + F];
+            ldbl xr = q[t * d + ire], xi = q[t * d + iim];
             sr += xr;
             si += xi;
             sn += hypotl(xr, xi);
@@ -135,9 +155,10 @@ void ora_calib(int d, int64_t nq, const double *q, double *centre, double *mnorm
  *   post_rope: 1 if the cache holds RoPE-rotated keys (they are de-rotated
  *         by their own position first), 0 if it holds pre-RoPE keys.
  *   offsets: [n_off] future offsets delta.
+ *   il: 1 for interleaved RoPE pairs, 0 for rotate-half (pair_dims).
  *   out: [n] scores.
  */
-void ora_score_literal(int d, double theta, int G, const double *qbar, const double *mnorm,
+void ora_score_literal(int d, int il, double theta, int G, const double *qbar, const double *mnorm,
                        int64_t n, const double *keys, const int64_t *pos, int post_rope,
                        int64_t p_now, int n_off, const int64_t *offsets, double *out)
 {
@@ -159,7 +180,7 @@ void ora_score_literal(int d, double theta, int G, const double *qbar, const dou
             ldbl sg = 0.0L;
             for (int f = 0; f < F; f++) {
                 ldbl kr, ki;
-                key_pair(d, keys + j * d, f, post_rope, w[f], pos[j], &kr, &ki);
+                key_pair(d, il, keys + j * d, f, post_rope, w[f], pos[j], &kr, &ki);
                 ldbl kn = hypotl(kr, ki);
                 ldbl phi = qa[g * F + f] - atan2l(ki, kr);
                 ldbl trig = 0.0L;
@@ -182,7 +203,7 @@ void ora_score_literal(int d, double theta, int G, const double *qbar, const dou
  * so there is one (cos, sin) per (key, g, f) of x = w_f (p_now - j) + phi.
  * Arguments as for ora_score_literal.
  */
-void ora_score_collapsed(int d, double theta, int G, const double *qbar, const double *mnorm,
+void ora_score_collapsed(int d, int il, double theta, int G, const double *qbar, const double *mnorm,
                          int64_t n, const double *keys, const int64_t *pos, int post_rope,
                          int64_t p_now, int n_off, const int64_t *offsets, double *out)
 {
@@ -214,7 +235,7 @@ void ora_score_collapsed(int d, double theta, int G, const double *qbar, const d
             ldbl sg = 0.0L;
             for (int f = 0; f < F; f++) {
                 ldbl kr, ki;
-                key_pair(d, keys + j * d, f, post_rope, w[f], pos[j], &kr, &ki);
+                key_pair(d, il, keys + j * d, f, post_rope, w[f], pos[j], &kr, &ki);
                 ldbl kn = hypotl(kr, ki);
                 ldbl x = w[f] * (ldbl)(p_now - pos[j]) + qa[g * F + f] - atan2l(ki, kr);
                 ldbl trig = cosl(x) * sr[f] - sinl(x) * si[f];
@@ -243,7 +264,7 @@ void ora_score_collapsed(int d, double theta, int G, const double *qbar, const d
  *   c_f = (1/G) sum_g (E|q_f^g| - |qbar_f^g|).
  * Kept only to cross-check that identity against the literal form.
  */
-void ora_score_absorbed(int d, double theta, int G, const double *qbar, const double *mnorm,
+void ora_score_absorbed(int d, int il, double theta, int G, const double *qbar, const double *mnorm,
                         int64_t n, const double *keys, const int64_t *pos, int post_rope,
                         int64_t p_now, int n_off, const int64_t *offsets, double *out)
 {
@@ -284,7 +305,9 @@ void ora_score_absorbed(int d, double theta, int G, const double *qbar, const do
     for (int64_t j = 0; j < n; j++) {
         ldbl s = 0.0L;
         for (int f = 0; f < F; f++) {
-            ldbl kr = keys[j * d + f], ki = keys[j * d + f + F];
+            int ire, iim;
+            pair_dims(d, il, f, &ire, &iim);
+            ldbl kr = keys[j * d + ire], ki = keys[j * d + iim];
             ldbl br = ar[f], bi = ai[f];
             if (!post_rope) {
                 ldbl a = w[f] * (ldbl)(p_now - pos[j]), ec = cosl(a), es = sinl(a);

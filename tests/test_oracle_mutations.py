@@ -29,8 +29,10 @@ MUTATIONS = [
     ("de-rotation by +angle",
      [("*re = xr * c + xi * s;", "*re = xr * c - xi * s;"),
       ("*im = xi * c - xr * s;", "*im = xi * c + xr * s;")]),
-    ("interleaved pairing",
-     [("ldbl xr = key[f], xi = key[f + F];", "ldbl xr = key[2 * f], xi = key[2 * f + 1];")]),
+    ("interleaved pairing where rotate-half is asked",
+     [("        *ire = f;\n        *iim = f + d / 2;", "        *ire = 2 * f;\n        *iim = 2 * f + 1;")]),
+    ("interleaved pair with real and imaginary swapped",
+     [("        *ire = 2 * f;\n        *iim = 2 * f + 1;", "        *ire = 2 * f + 1;\n        *iim = 2 * f;")]),
     ("phase sign flipped",
      [("ldbl phi = qa[g * F + f] - atan2l(ki, kr);", "ldbl phi = atan2l(ki, kr) - qa[g * F + f];")]),
     ("distance uses slot sign reversed",
@@ -41,7 +43,7 @@ MUTATIONS = [
     ("calibration norm of the mean",
      [("mnorm[f] = (double)(sn / (ldbl)nq);", "mnorm[f] = (double)hypotl(sr / (ldbl)nq, si / (ldbl)nq);")]),
     ("calibration drops the imaginary half",
-     [("ldbl xr = q[t * d + f], xi = q[t * d + f + F];", "ldbl xr = q[t * d + f], xi = 0.0L * q[t * d + f + F];")]),
+     [("ldbl xr = q[t * d + ire], xi = q[t * d + iim];", "ldbl xr = q[t * d + ire], xi = 0.0L * q[t * d + iim];")]),
     ("tie-break keeps the older slot",
      [("if (a->i != b->i) return a->i > b->i ? -1 : 1;", "if (a->i != b->i) return a->i < b->i ? -1 : 1;")]),
     ("window not protected",
@@ -56,6 +58,7 @@ MUTATIONS = [
 PIN_FUNCS = [
     lambda: pins.test_omega_is_theta_power(),
     lambda: pins.test_trig_series_equals_rope_dot_at_every_distance(0),
+    lambda: pins.test_trig_series_equals_rope_dot_other_layouts(64, True),
     lambda: pins.test_golden_closed_forms(),
     lambda: pins.test_identical_queries_give_attention_logit_sum(True),
     lambda: pins.test_identical_queries_give_attention_logit_sum(False),

@@ -49,6 +49,29 @@ def rope_ld(x, p, theta):
     return out
 
 
+def rope_il_ld(x, p, theta):
+    """Interleaved RoPE (GPT-J / Meta-Llama complex layout) of x [..., d] at position p:
+    x'[2f] = x[2f] cos(w_f p) - x[2f+1] sin(w_f p);  x'[2f+1] = x[2f+1] cos + x[2f] sin."""
+    x = np.asarray(x, dtype=LD)
+    d = x.shape[-1]
+    a = omega_ld(theta, d) * LD(p)
+    c, s = np.cos(a), np.sin(a)
+    out = np.empty_like(x)
+    out[..., 0::2] = x[..., 0::2] * c - x[..., 1::2] * s
+    out[..., 1::2] = x[..., 1::2] * c + x[..., 0::2] * s
+    return out
+
+
+def pair_abs_il(x):
+    x = np.asarray(x, dtype=np.float64)
+    return np.hypot(x[..., 0::2], x[..., 1::2])
+
+
+def as_centre_il(v):
+    v = np.asarray(v, dtype=np.float64)
+    return np.stack([v[..., 0::2], v[..., 1::2]], axis=-1)
+
+
 def dot_ld(a, b):
     return np.sum(np.asarray(a, dtype=LD) * np.asarray(b, dtype=LD), axis=-1)
 
@@ -104,6 +127,29 @@ def test_trig_series_equals_rope_dot_at_every_distance(seed):
     assert worst < 1e-12, worst
 
 
+@pytest.mark.parametrize("d,interleaved", [(64, False), (256, False), (64, True), (128, True),
+                                           (256, True)])
+def test_trig_series_equals_rope_dot_other_layouts(d, interleaved):
+    """The same identity for head dims 64 and 256 and for interleaved pairs (2f, 2f+1),
+    against an explicit rotation of the matching layout."""
+    rng = np.random.default_rng(d + 7 * interleaved)
+    theta = 1e4 if d == 256 else 1e6
+    rope = rope_il_ld if interleaved else rope_ld
+    pabs = pair_abs_il if interleaved else pair_abs
+    q = rng.standard_normal(d) * np.exp(rng.standard_normal(d))
+    k = rng.standard_normal(d) * np.exp(rng.standard_normal(d))
+    scale = float(np.sum(pabs(q) * pabs(k)))
+    qb = as_centre_il(q) if interleaved else as_centre(q)
+    worst = 0.0
+    for dist in list(range(0, 600, 13)) + list(rng.integers(0, 2**17, size=20)):
+        dist = int(dist)
+        for j in (0, 4099):
+            ref = dot_ld(rope(q, j + dist, theta), rope(k, j, theta))
+            got = oracle.trig_series(theta, qb, k, dist, interleaved=interleaved)
+            worst = max(worst, abs(float(ref) - got) / scale)
+    assert worst < 1e-12, worst
+
+
 def test_trig_series_negative_distance():
     rng = np.random.default_rng(7)
     d, theta = 128, 1e6
@@ -133,13 +179,13 @@ def test_golden_closed_forms():
 
 # ------------------------------------- whole score: textbook special cases
 
-def _explicit_logit_sum(qs, k_cached, pos, post_rope, p_now, offsets, theta):
+def _explicit_logit_sum(qs, k_cached, pos, post_rope, p_now, offsets, theta, rope=rope_ld):
     """(1/G) sum_g sum_delta RoPE(q_g, p_now+delta) . k_post, k_post = the key as RoPE'd at pos."""
-    k_post = np.asarray(k_cached, dtype=LD) if post_rope else rope_ld(k_cached, pos, theta)
+    k_post = np.asarray(k_cached, dtype=LD) if post_rope else rope(k_cached, pos, theta)
     tot = LD(0)
     for q in qs:
         for dlt in offsets:
-            tot += dot_ld(rope_ld(q, p_now + dlt, theta), k_post)
+            tot += dot_ld(rope(q, p_now + dlt, theta), k_post)
     return tot / LD(len(qs))
 
 
@@ -171,6 +217,35 @@ def test_identical_queries_give_attention_logit_sum(post_rope):
     for tier in ("literal", "collapsed", "absorbed"):
         fn = getattr(oracle, "score_" + tier)
         got = fn(theta, centres, mnorms, keys, pos, post_rope, p_now, offsets)
+        assert np.max(np.abs(got - ref) / scale) < 1e-12, tier
+
+
+@pytest.mark.parametrize("post_rope", [True, False])
+@pytest.mark.parametrize("d,interleaved", [(64, False), (256, False), (128, True), (64, True)])
+def test_identical_queries_logit_sum_other_layouts(post_rope, d, interleaved):
+    """The textbook attention-logit special case for head dims 64/256 and interleaved pairs."""
+    rng = np.random.default_rng(17 + d + interleaved)
+    theta, G, nq = 1e4, 2, 3
+    offsets = [1, 2, 4, 8, 16, 32, 64, 128]
+    rope = rope_il_ld if interleaved else rope_ld
+    pabs = pair_abs_il if interleaved else pair_abs
+    qs = rng.standard_normal((G, d))
+    cm = [oracle.calib(np.repeat(qs[g][None], nq, axis=0), interleaved=interleaved) for g in range(G)]
+    centres = np.array([c for c, _ in cm])
+    mnorms = np.array([m for _, m in cm])
+    n = 12
+    pos = rng.integers(0, 20000, size=n)
+    p_now = 20000
+    keys_pre = rng.standard_normal((n, d))
+    keys = np.array([rope(keys_pre[j], pos[j], theta) for j in range(n)], dtype=np.float64) \
+        if post_rope else keys_pre
+    ref = np.array([float(_explicit_logit_sum(qs, keys[j], pos[j], post_rope, p_now, offsets, theta,
+                                              rope)) for j in range(n)])
+    scale = np.array([len(offsets) * np.mean([np.sum(pabs(q) * pabs(keys[j])) for q in qs])
+                      for j in range(n)])
+    for tier in ("literal", "collapsed", "absorbed"):
+        fn = getattr(oracle, "score_" + tier)
+        got = fn(theta, centres, mnorms, keys, pos, post_rope, p_now, offsets, interleaved=interleaved)
         assert np.max(np.abs(got - ref) / scale) < 1e-12, tier
 
 
@@ -274,6 +349,16 @@ def test_calib_single_query():
     np.testing.assert_array_equal(c[:, 0], q[0, :64])
     np.testing.assert_array_equal(c[:, 1], q[0, 64:])
     np.testing.assert_allclose(m, np.hypot(q[0, :64], q[0, 64:]), rtol=1e-15)
+
+
+def test_calib_interleaved_pairs():
+    """Interleaved layout: pair f is dims (2f, 2f+1)."""
+    rng = np.random.default_rng(33)
+    q = rng.standard_normal((500, 64)) + rng.standard_normal(64)
+    c, m = oracle.calib(q, interleaved=True)
+    np.testing.assert_allclose(c[:, 0], q[:, 0::2].mean(axis=0), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(c[:, 1], q[:, 1::2].mean(axis=0), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(m, np.hypot(q[:, 0::2], q[:, 1::2]).mean(axis=0), rtol=1e-13)
 
 
 def test_calib_matches_numpy_and_triangle_inequality():
