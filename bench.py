@@ -8,7 +8,7 @@ offline and timed separately.  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload qwen3_8b_32k] [--budget B] [--key-mode post|pre]
-                  [--elem bf16|fp8]
+                  [--elem bf16|fp8] [--head-dim 64|128|256] [--rope half|interleaved]
 
 N > 1 (under torchrun): every rank compacts its own cache of the same shape
 (independent sequences; no collective on the data path), timing is the max
@@ -43,12 +43,12 @@ FALLBACK_HBM_GBS = 6650.0
 ELEM_BYTES = {"bf16": 2, "fp8": 1}
 
 
-def score_bytes_per_key(eb: int) -> int:
-    return 128 * eb + 4  # read the key, write its fp32 score
+def score_bytes_per_key(eb: int, d: int = 128) -> int:
+    return d * eb + 4  # read the key, write its fp32 score
 
 
-def kept_bytes(eb: int) -> int:
-    return 4 * 128 * eb + 8  # read + write K and V of a kept key, read + write its position
+def kept_bytes(eb: int, d: int = 128) -> int:
+    return 4 * d * eb + 8  # read + write K and V of a kept key, read + write its position
 
 
 def parse():
@@ -64,6 +64,10 @@ def parse():
     ap.add_argument("--key-mode", choices=["post", "pre"], default="post")
     ap.add_argument("--elem", choices=sorted(ELEM_BYTES), default="bf16",
                     help="K/V cache element type (fp8 = OCP e4m3, converted from the bf16 cache)")
+    ap.add_argument("--head-dim", type=int, choices=[64, 128, 256], default=None,
+                    help="override the workload's head dim (same heads and lengths)")
+    ap.add_argument("--rope", choices=["half", "interleaved"], default=None,
+                    help="override the workload's RoPE pairing")
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="timed steps replay CUDA graphs of the calls (default) or call eagerly")
     ap.add_argument("--no-e2e", action="store_true")
@@ -82,9 +86,9 @@ def workload_config(wl, B, key_mode, launch="eager", elem="bf16"):
             "batch": wl.batch, "keys_per_head": lo if lo == hi else [lo, hi], "budget": B,
             "window": wl.window, "offsets": wl.n_offsets, "key_mode": key_mode + "_rope",
             "launch": launch,
-            "layout": wl.layout, "kv_elem": elem,
+            "layout": wl.layout, "kv_elem": elem, "rope": wl.rope_style,
             "l2": "inputs larger than L2: K+V %.1f GB read per step, no flush" % (
-                2 * 128 * eb * wl.n_layers * wl.batch * wl.n_kv_heads * np.mean(wl.seq_len) / 1e9)}
+                2 * wl.head_dim * eb * wl.n_layers * wl.batch * wl.n_kv_heads * np.mean(wl.seq_len) / 1e9)}
 
 
 def measured_peak():
@@ -181,6 +185,15 @@ class ClockSampler:
 
 # ------------------------------------------------------- multi-rank logic
 
+def with_layout(wl, a):
+    """The workload with --head-dim / --rope applied (same heads, lengths and budget)."""
+    if a.head_dim:
+        wl = wl.with_(head_dim=a.head_dim)
+    if a.rope:
+        wl = wl.with_(rope_style=a.rope)
+    return wl
+
+
 def rank_workload(wl, rank: int, B: int):
     """Rank r compacts its own independent cache of the same shape (other sequences):
     same workload, seed offset by the rank.  No rank reads another's rows."""
@@ -212,6 +225,7 @@ def run_ours(a, rank, world, local_rank):
     B = a.budget or wl0.budget
     if a.layers:
         wl0 = wl0.with_(n_layers=min(a.layers, wl0.n_layers))
+    wl0 = with_layout(wl0, a)
     wl = rank_workload(wl0, rank, B)
     key_mode = tri.TRI_KEYS_PRE_ROPE if a.key_mode == "pre" else tri.TRI_KEYS_POST_ROPE
     if wl.layout != "contig":
@@ -224,13 +238,15 @@ def run_ours(a, rank, world, local_rank):
         torch.cuda.empty_cache()
     L, S, Hh = wl.n_layers, len(cache.lens), wl.n_kv_heads
     R, total = cache.n_rows, cache.total
-    m = tri.model(L, wl.n_q_heads, Hh, wl.theta)
+    m = tri.model(L, wl.n_q_heads, Hh, wl.theta, head_dim=wl.head_dim,
+                  rope_style=tri.TRI_ROPE_INTERLEAVED if wl.interleaved else tri.TRI_ROPE_HALF)
+    D = wl.head_dim
     kv = tri.kv_contig(S, cache.row_off, total, tri.elem_type_of(cache.K))
     stream = torch.cuda.current_stream(dev)
 
     # offline calibration (timed separately, not part of a step)
-    centres = torch.empty(L, wl.n_q_heads, 64, 2, dtype=torch.float32, device=dev)
-    mnorm = torch.empty(L, wl.n_q_heads, 64, dtype=torch.float32, device=dev)
+    centres = torch.empty(L, wl.n_q_heads, D // 2, 2, dtype=torch.float32, device=dev)
+    mnorm = torch.empty(L, wl.n_q_heads, D // 2, dtype=torch.float32, device=dev)
     tri.tri_calib(m, cache.qcal, wl.n_calib, centres, mnorm)
     torch.cuda.synchronize()
     c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -242,7 +258,7 @@ def run_ours(a, rank, world, local_rank):
 
     ws = tri.alloc_workspace(m, S, B, device=dev)
     scores = torch.empty(total, dtype=torch.float32, device=dev)
-    Ko = torch.empty(R, B, 128, dtype=cache.K.dtype, device=dev)
+    Ko = torch.empty(R, B, D, dtype=cache.K.dtype, device=dev)
     Vo = torch.empty_like(Ko)
     po = torch.empty(R, B, dtype=torch.int32, device=dev)
     kept = torch.empty(R, B, dtype=torch.int32, device=dev)
@@ -308,7 +324,7 @@ def run_ours(a, rank, world, local_rank):
 
     lens_rows = np.diff(cache.row_off_np)
     keys_step = int(total)
-    alg_bytes = float(np.sum(128.0 * eb * lens_rows + np.minimum(lens_rows, B) * kept_bytes(eb)))
+    alg_bytes = float(np.sum(float(D) * eb * lens_rows + np.minimum(lens_rows, B) * kept_bytes(eb, D)))
     if key_mode == tri.TRI_KEYS_PRE_ROPE:
         alg_bytes += 4.0 * total
     ms_step = ms / a.steps
@@ -321,7 +337,7 @@ def run_ours(a, rank, world, local_rank):
                       world, dev)
 
     peak, peak_kind = measured_peak()
-    score_bytes = score_bytes_per_key(eb) * total
+    score_bytes = score_bytes_per_key(eb, D) * total
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     path_gbs = alg_bytes / (ms_step / 1e3) / 1e9
     line = {
@@ -330,7 +346,7 @@ def run_ours(a, rank, world, local_rank):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(wl, B, a.key_mode, "cuda_graph" if a.launch == "graph" else "eager", a.elem),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(total, a.elem),
+                     "frac": achieved / peak, "traffic": recorded_traffic(total, a.elem) if (D, wl.rope_style) == (128, "half") else None,
                      "kernel": "tri_score (prep + score kernels)", "peak_kind": peak_kind,
                      "bytes_per_launch": score_bytes, "ms_per_launch": score_ms},
         "path_roofline": {"bytes_per_step": alg_bytes, "achieved_gbs": path_gbs,
@@ -410,7 +426,7 @@ def oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs, ms, rows_meta, seconds, m
         Kb = K_rows[j]
         Kf = oracle.e4m3_bits_to_f64(Kb) if Kb.dtype == np.uint8 else oracle.bf16_bits_to_f64(Kb)
         s = oracle.row_scores(wl.theta, cs, ms, h, wl.group, Kf, pos_rows[j], True, p_now, wl.offsets,
-                              "collapsed")
+                              "collapsed", wl.interleaved)
         kept = oracle.select(s, B, wl.window)
         oracle.gather(K_rows[j], kept)
         oracle.gather(V_rows[j], kept)
@@ -437,7 +453,7 @@ def cpu_baseline(wl, B, cache, seconds):
         pos_rows.append(cache.pos[a:b].cpu().numpy().astype(np.int64))
         _, s, h = cache.row_lhs(r)
         meta.append((h, int(cache.lens[s])))
-    cs, ms = H.oracle_calibration(cache.qcal[:1])
+    cs, ms = H.oracle_calibration(cache.qcal[:1], wl.interleaved)
     keys, n_rows, dt = oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs[0], ms[0], meta, seconds, 64)
     return {"value": keys / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{n_rows} rows x {len(K_rows[0])} keys of layer 0 (score collapsed fp64 + select + gather), "
@@ -450,7 +466,7 @@ def run_reference(a, rank, world):
 
     wl0 = synth.WORKLOADS[a.workload]
     B = a.budget or wl0.budget
-    wl = wl0.with_(budget=B)
+    wl = with_layout(wl0.with_(budget=B), a)
     cache = synth.make_contig(wl, "cpu", layers=[0], lens=wl.seq_lengths()[:1])
     if a.elem == "fp8":
         cache.K = synth.to_fp8(cache.K)
@@ -463,7 +479,7 @@ def run_reference(a, rank, world):
         V_rows.append(H.raw_bits(cache.V[a_:b_]))
         pos_rows.append(cache.pos[a_:b_].numpy().astype(np.int64))
         meta.append((r % Hh, int(cache.lens[0])))
-    cs, ms = H.oracle_calibration(cache.qcal)
+    cs, ms = H.oracle_calibration(cache.qcal, wl.interleaved)
     for i in range(a.warmup):
         oracle_sample(wl, B, K_rows[i % Hh:i % Hh + 1], V_rows[i % Hh:i % Hh + 1], pos_rows[i % Hh:i % Hh + 1],
                       cs[0], ms[0], meta[i % Hh:i % Hh + 1], 0.0, 1)

@@ -15,8 +15,10 @@
  *                                    + sum_f (E|q_f^g| - |qbar_f^g|) |k_f| ],
  *   w_f = rope_theta^(-2f/d),  phi_f^g = arg qbar_f^g - arg k_f,
  *
- * k the pre-RoPE key, pairs f = dims (f, f + d/2) (rotate-half RoPE, as in
- * Qwen3/Llama), group(h) = query heads h*G .. h*G+G-1, G = n_q_heads/n_kv_heads.
+ * k the pre-RoPE key, f = 0 .. d/2-1 over frequency pairs: dims (f, f + d/2) with
+ * rotate-half RoPE (Qwen3 / Llama-HF / GPT-NeoX), dims (2f, 2f + 1) with
+ * interleaved RoPE (GPT-J / Meta-Llama); group(h) = query heads h*G .. h*G+G-1,
+ * G = n_q_heads/n_kv_heads.
  *
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers on the current device, allocated
@@ -48,7 +50,7 @@ typedef struct CUstream_st *tri_stream_t; /* same type as cudaStream_t */
 typedef enum {
     TRI_OK = 0,
     TRI_ERR_INVALID_ARG = 1,         /* null pointer, negative size, inconsistent shapes */
-    TRI_ERR_UNSUPPORTED = 2,         /* head_dim != 128, block size not a power of two, ... */
+    TRI_ERR_UNSUPPORTED = 2,         /* head_dim not 64/128/256, block size not a power of two, ... */
     TRI_ERR_ALIGNMENT = 3,           /* a pointer is not aligned as documented */
     TRI_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < tri_workspace_size(...) */
     TRI_ERR_CUDA = 5,                /* a CUDA launch or copy failed */
@@ -61,18 +63,20 @@ typedef enum {
 #define TRI_FLAG_BLOCK_TABLE 0x4u /* paged: block id out of [0, n_blocks) or row too long for the table; the key is skipped */
 
 #define TRI_MAX_OFFSETS 64
-#define TRI_HEAD_DIM 128
 
 enum { TRI_KV_CONTIG = 0, TRI_KV_PAGED = 1 };
+enum { TRI_ROPE_HALF = 0, TRI_ROPE_INTERLEAVED = 1 }; /* pair f = dims (f, f+d/2) or (2f, 2f+1) */
 enum { TRI_ELEM_BF16 = 0, TRI_ELEM_FP8_E4M3 = 1 }; /* K/V element type */
 enum { TRI_KEYS_POST_ROPE = 0, TRI_KEYS_PRE_ROPE = 1 };
 
 typedef struct {
-    int32_t head_dim;   /* d; only 128 is supported */
+    int32_t head_dim;   /* d: 64, 128 or 256 */
     int32_t n_layers;   /* L >= 1 */
     int32_t n_q_heads;  /* Hq >= 1 */
     int32_t n_kv_heads; /* H >= 1, Hq % H == 0 */
     double rope_theta;  /* theta > 1 */
+    int32_t rope_style; /* TRI_ROPE_HALF (0, the default of a zeroed struct) or TRI_ROPE_INTERLEAVED */
+    int32_t pad_;       /* zero */
 } tri_model;
 
 /*
@@ -150,13 +154,14 @@ tri_status tri_workspace_init(void *ws, size_t ws_bytes, tri_stream_t stream);
  * Offline calibration (digest, 流程详解 step 1): for every (layer l, query head g)
  * and pair f, the complex mean of the pre-RoPE queries and the mean of their
  * magnitudes,
- *   centres[l][g][f] = (1/nq) sum_t (q[t][f] + i q[t][f+64])          (re, im)
- *   mean_norm[l][g][f] = (1/nq) sum_t |q[t][f] + i q[t][f+64]|,
- * accumulated in fp64, stored fp32.
- *   qpre:      bf16 [n_layers][n_q_heads][nq][128], 16-byte aligned
+ *   centres[l][g][f] = (1/nq) sum_t (q[t][a_f] + i q[t][b_f])          (re, im)
+ *   mean_norm[l][g][f] = (1/nq) sum_t |q[t][a_f] + i q[t][b_f]|,
+ * with (a_f, b_f) the dims of pair f under m->rope_style, accumulated in fp64,
+ * stored fp32.
+ *   qpre:      bf16 [n_layers][n_q_heads][nq][d], 16-byte aligned
  *   nq:        queries per head, >= 1
- *   centres:   float [n_layers][n_q_heads][64][2]
- *   mean_norm: float [n_layers][n_q_heads][64]
+ *   centres:   float [n_layers][n_q_heads][d/2][2]
+ *   mean_norm: float [n_layers][n_q_heads][d/2]
  */
 tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *centres,
                      float *mean_norm, tri_stream_t stream);
@@ -168,7 +173,7 @@ tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *ce
  *   K:         keys (kv->elem_type) in kv's layout, 16-byte aligned
  *   pos:       int32 position of every cached slot (kv's layout).  Read only
  *              for TRI_KEYS_PRE_ROPE; may be NULL for TRI_KEYS_POST_ROPE.
- *   centres, mean_norm: calibration of tri_calib, [n_layers][n_q_heads][64](x2);
+ *   centres, mean_norm: calibration of tri_calib, [n_layers][n_q_heads][d/2](x2);
  *              centres 8-byte aligned, mean_norm 4-byte aligned
  *   p_now:     device int64 [n_seqs], the position of each sequence's next token
  *   offsets:   HOST int32 [n_offsets], the future offsets delta, 1 <= n_offsets
@@ -229,7 +234,7 @@ tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream);
  * an interface convenience.
  *
  * Same arguments and results as tri_score, minus ws/ws_bytes.  The scratch is
- * a fixed array inside the library (about 3 MiB on every GPU that loads it,
+ * a fixed array inside the library (about 6 MiB on every GPU that loads it,
  * held until the process exits), enough for at most TRI_NOALLOC_MAX_ROWS rows
  * (n_layers * n_seqs * n_kv_heads); more rows return
  * TRI_ERR_WORKSPACE_TOO_SMALL before anything is launched.  The call

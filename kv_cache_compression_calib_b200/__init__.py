@@ -20,7 +20,7 @@ import torch
 from . import _abi
 from ._abi import (TRI_ELEM_BF16, TRI_ELEM_FP8_E4M3, TRI_FLAG_BLOCK_TABLE,  # noqa: F401
                    TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS, TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
-                   TRI_MAX_OFFSETS, TriKvDesc, TriModel, TriOutDesc)
+                   TRI_MAX_OFFSETS, TRI_ROPE_HALF, TRI_ROPE_INTERLEAVED, TriKvDesc, TriModel, TriOutDesc)
 
 _L = _abi.load()
 
@@ -60,8 +60,9 @@ def library_path() -> str:
 # ------------------------------------------------------------- descriptors
 
 def model(n_layers: int, n_q_heads: int, n_kv_heads: int, rope_theta: float,
-          head_dim: int = 128) -> TriModel:
-    return TriModel(head_dim, n_layers, n_q_heads, n_kv_heads, float(rope_theta))
+          head_dim: int = 128, rope_style: int = TRI_ROPE_HALF) -> TriModel:
+    """Model shape; ``rope_style`` TRI_ROPE_HALF pairs dims (f, f+d/2), TRI_ROPE_INTERLEAVED (2f, 2f+1)."""
+    return TriModel(head_dim, n_layers, n_q_heads, n_kv_heads, float(rope_theta), int(rope_style), 0)
 
 
 # A descriptor holds raw device pointers; it also keeps a reference to the tensors

@@ -20,7 +20,8 @@ TRI_FLAG_NONFINITE = 0x2
 TRI_FLAG_BLOCK_TABLE = 0x4
 
 TRI_MAX_OFFSETS = 64
-TRI_HEAD_DIM = 128
+TRI_ROPE_HALF = 0
+TRI_ROPE_INTERLEAVED = 1
 TRI_KV_CONTIG = 0
 TRI_KV_PAGED = 1
 TRI_ELEM_BF16 = 0
@@ -37,7 +38,8 @@ TRI_NOALLOC_MAX_ROWS = 4096
 class TriModel(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
-                ("rope_theta", ctypes.c_double)]
+                ("rope_theta", ctypes.c_double), ("rope_style", ctypes.c_int32),
+                ("pad_", ctypes.c_int32)]
 
 
 class TriKvDesc(ctypes.Structure):

@@ -38,7 +38,8 @@ int pow2_shift(int32_t x) {
 
 tri_status check_model(const tri_model *m) {
     if (!m) return TRI_ERR_INVALID_ARG;
-    if (m->head_dim != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+    if (m->head_dim != 64 && m->head_dim != 128 && m->head_dim != 256) return TRI_ERR_UNSUPPORTED;
+    if (m->rope_style != TRI_ROPE_HALF && m->rope_style != TRI_ROPE_INTERLEAVED) return TRI_ERR_INVALID_ARG;
     if (m->n_layers < 1 || m->n_q_heads < 1 || m->n_kv_heads < 1) return TRI_ERR_INVALID_ARG;
     if (m->n_q_heads % m->n_kv_heads) return TRI_ERR_INVALID_ARG;
     if (!std::isfinite(m->rope_theta) || !(m->rope_theta > 1.0)) return TRI_ERR_INVALID_ARG;
@@ -59,6 +60,8 @@ tri_status check_kv(const tri_model *m, const tri_kv_desc *kv, Geometry *geo) {
     geo->Hq = m->n_q_heads;
     geo->G = m->n_q_heads / m->n_kv_heads;
     geo->layout = kv->layout;
+    geo->D = m->head_dim;
+    geo->il = m->rope_style == TRI_ROPE_INTERLEAVED;
     geo->total = kv->total_keys;
     geo->row_off = kv->row_off;
     if (kv->elem_type == TRI_ELEM_BF16) geo->elem_bytes = 2;
@@ -118,7 +121,7 @@ const char *tri_last_error(void) { return g_last_error; }
 
 size_t tri_workspace_size(const tri_model *m, int32_t n_seqs, int32_t B) {
     if (check_model(m) != TRI_OK || n_seqs < 1 || B < 1) return 0;
-    return ws_total(rows_of(m, n_seqs), B);
+    return ws_total(rows_of(m, n_seqs), B, m->head_dim);
 }
 
 tri_status tri_workspace_init(void *ws, size_t ws_bytes, tri_stream_t stream) {
@@ -136,6 +139,8 @@ tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *ce
     const int64_t heads = (int64_t)m->n_layers * m->n_q_heads;
     if (heads > 0x7fffffffLL) return TRI_ERR_UNSUPPORTED;
     CalibParams p;
+    p.D = m->head_dim;
+    p.il = m->rope_style == TRI_ROPE_INTERLEAVED;
     p.q = (const uint16_t *)qpre;
     p.nq = nq;
     p.n_heads = (int32_t)heads;
@@ -160,7 +165,7 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
         !aligned(p_now, 8) || (pos && !aligned(pos, 4)))
         return TRI_ERR_ALIGNMENT;
     const int64_t R = rows_of(m, kv->n_seqs);
-    if ((st = check_ws(ws, ws_bytes, ws_idx_offset(R))) != TRI_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, ws_idx_offset(R, m->head_dim))) != TRI_OK) return st;
     char *w = (char *)ws;
     cudaStream_t s = (cudaStream_t)stream;
 
@@ -217,10 +222,10 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
         return TRI_ERR_INVALID_ARG;
     }
     const int64_t R = rows_of(m, kv->n_seqs);
-    if ((st = check_ws(ws, ws_bytes, kept_idx ? 256 : ws_total(R, B))) != TRI_OK) return st;
+    if ((st = check_ws(ws, ws_bytes, kept_idx ? 256 : ws_total(R, B, m->head_dim))) != TRI_OK) return st;
     char *w = (char *)ws;
     cudaStream_t s = (cudaStream_t)stream;
-    int32_t *kept = kept_idx ? kept_idx : (int32_t *)(w + ws_idx_offset(R));
+    int32_t *kept = kept_idx ? kept_idx : (int32_t *)(w + ws_idx_offset(R, m->head_dim));
 
     SelectParams sp;
     sp.geo = geo;

@@ -2,10 +2,10 @@
 // order, into the output cache ("TriAttention：基于三角函数 KV 压缩的高效长推理",
 // 流程详解 step 4: later attention reads only the compressed cache).
 //
-// Flat grid over (row, chunk of kept slots).  A record (one key or value: 256
-// bytes in bf16, 128 in fp8) is moved as 16-byte vectors by 16 (8) lanes, so
-// each warp instruction copies two (four) whole records; every thread keeps 4
-// K and 4 V vectors in flight.  Source reads
+// Flat grid over (row, chunk of kept slots).  A record (one key or value: d
+// elements, 64 to 512 bytes) is moved as 16-byte vectors by record/16 lanes,
+// so each warp instruction copies 512 bytes of whole records; every thread
+// keeps 4 K and 4 V vectors in flight.  Source reads
 // bypass L1; destination writes are streaming stores (not re-read here).
 // Paged input and/or output addresses go through the block tables.
 #include "tri_internal.cuh"
@@ -15,7 +15,7 @@ namespace tri {
 constexpr int kGatherThreads = 256;
 constexpr int kGatherIters = 4;
 
-// RB: record bytes (128 dims x element size).  A record is moved as RB/16
+// RB: record bytes (d x element size).  A record is moved as RB/16
 // 16-byte vectors by RB/16 lanes, so a warp instruction moves 512 bytes.
 template <int RB>
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherParams p) {
@@ -99,7 +99,13 @@ static cudaError_t launch_gather_t(const GatherParams &p, cudaStream_t s) {
 }
 
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t s) {
-    return p.geo.elem_bytes == 1 ? launch_gather_t<kD>(p, s) : launch_gather_t<2 * kD>(p, s);
+    switch (p.geo.D * p.geo.elem_bytes) {
+        case 64: return launch_gather_t<64>(p, s);
+        case 128: return launch_gather_t<128>(p, s);
+        case 256: return launch_gather_t<256>(p, s);
+        case 512: return launch_gather_t<512>(p, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace tri

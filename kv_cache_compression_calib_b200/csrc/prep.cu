@@ -3,16 +3,15 @@
 //   A_f = (1/G) sum_g qbar_f^g * e^{i w_f p_now} * sum_delta e^{i w_f delta}
 //         (without the e^{i w_f p_now} factor for a pre-RoPE cache),
 //   c_f = (1/G) sum_g (E|q_f^g| - |qbar_f^g|),
-// formed in fp64 and stored fp32 in the workspace ([R][8][24]: for lane group
-// g, pairs 8g..8g+7 as Re A, Im A, c), plus the table T_f = w_f / 2pi in 0.64
-// fixed point that the score kernel uses for per-key phases.  Every phase
+// formed in fp64 and stored fp32 in the workspace ([R][d/16][24]: for lane
+// group g, pairs 8g..8g+7 as Re A, Im A, c), plus the table T_f = w_f / 2pi in
+// 0.64 fixed point that the score kernel uses for per-key phases.  Every phase
 // w_f * n is reduced exactly as (n * T_f) mod 2^64 and evaluated in fp64.
 #include "tri_internal.cuh"
 
 namespace tri {
 
 constexpr int kPrepParts = 4;
-constexpr int kPrepThreads = kPrepParts * kF;
 constexpr double kTurnScale = 2.9358905032820014e+18;    // 2^64 / (2 pi)
 constexpr double kTurnToRad64 = 3.4061215800865545e-19;  // 2 pi / 2^64
 
@@ -22,23 +21,24 @@ __device__ __forceinline__ void sincos_turns(unsigned long long t, double *sn, d
     sincos((double)(long long)t * kTurnToRad64, sn, cs);
 }
 
-// One CTA per row; thread (part, f) sums the offsets e = part, part+4, ... of
-// pair f, then the 64 threads of part 0 finish the row's coefficients.  All
-// phases w_f * n are reduced exactly as (n * T_f) mod 2^64, T_f = w_f / 2pi in
-// 0.64 fixed point, and evaluated in fp64.
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) {
-    __shared__ double part_re[kPrepParts][kF], part_im[kPrepParts][kF];
+// One CTA of 4F threads per row (F = d/2 pairs); thread (part, f) sums the
+// offsets e = part, part+4, ... of pair f, then the F threads of part 0 finish
+// the row's coefficients.  All phases w_f * n are reduced exactly as
+// (n * T_f) mod 2^64, T_f = w_f / 2pi in 0.64 fixed point, and evaluated in fp64.
+template <int F>
+__global__ void __launch_bounds__(kPrepParts * F) prep_kernel(const PrepParams p) {
+    __shared__ double part_re[kPrepParts][F], part_im[kPrepParts][F];
     const Geometry &geo = p.geo;
     const int r = blockIdx.x;
-    const int f = threadIdx.x & (kF - 1);
-    const int part = threadIdx.x >> 6;
+    const int f = threadIdx.x % F;
+    const int part = threadIdx.x / F;
     const int h = r % geo.H;
     const int s = (r / geo.H) % geo.S;
     const int l = r / (geo.H * geo.S);
     const int64_t qh0 = (int64_t)l * geo.Hq + (int64_t)h * geo.G;
     // The offsets' phasor sums depend on kernel parameters only: form them before
     // waiting for the preceding kernel on the stream.
-    const double w = pow(p.theta, -2.0 * (double)f / (double)kD);
+    const double w = pow(p.theta, -2.0 * (double)f / (double)(2 * F));
     const unsigned long long T = __double2ull_rn(w * kTurnScale);
     double sr = 0.0, si = 0.0;
     for (int e = part; e < p.n_off; e += kPrepParts) {
@@ -56,8 +56,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             if (j < geo.G) {
-                qv[j] = reinterpret_cast<const float2 *>(p.centres)[(qh0 + j) * kF + f];
-                mv[j] = p.mean_norm[(qh0 + j) * kF + f];
+                qv[j] = reinterpret_cast<const float2 *>(p.centres)[(qh0 + j) * F + f];
+                mv[j] = p.mean_norm[(qh0 + j) * F + f];
             }
         }
         pnow = p.p_now[s];
@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 if (g0 + j < geo.G) {
-                    qv[j] = reinterpret_cast<const float2 *>(p.centres)[(qh0 + g0 + j) * kF + f];
-                    mv[j] = p.mean_norm[(qh0 + g0 + j) * kF + f];
+                    qv[j] = reinterpret_cast<const float2 *>(p.centres)[(qh0 + g0 + j) * F + f];
+                    mv[j] = p.mean_norm[(qh0 + g0 + j) * F + f];
                 }
             }
         }
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
         ar = tr * cs - ti * sn;
         ai = tr * sn + ti * cs;
     }
-    float *c = p.coef + (int64_t)r * kCoefPerRow + (f >> 3) * kCoefPerGroup;
+    float *c = p.coef + (int64_t)r * (3 * F) + (f >> 3) * kCoefPerGroup;
     c[f & 7] = (float)ar;
     c[8 + (f & 7)] = (float)ai;
     c[16 + (f & 7)] = (float)cf;
@@ -121,7 +121,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const PrepParams p) 
 cudaError_t launch_prep(const PrepParams &p, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
-    return launch_pdl(prep_kernel, dim3((unsigned)R), dim3(kPrepThreads), 0, s, p);
+    switch (p.geo.D) {
+        case 64: return launch_pdl(prep_kernel<32>, dim3((unsigned)R), dim3(kPrepParts * 32), 0, s, p);
+        case 128: return launch_pdl(prep_kernel<64>, dim3((unsigned)R), dim3(kPrepParts * 64), 0, s, p);
+        case 256: return launch_pdl(prep_kernel<128>, dim3((unsigned)R), dim3(kPrepParts * 128), 0, s, p);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace tri

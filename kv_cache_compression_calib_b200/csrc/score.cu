@@ -12,9 +12,10 @@
 //   c_f = (1/G) sum_g (E|q_f^g| - |qbar_f^g|).
 // The delta sum collapses by angle addition into one complex constant per f,
 // and the GQA mean into A_f (the score is linear in the per-head terms).  The
-// per-key work is then a 64-pair dot product plus 64 magnitudes: 256 B of
-// bf16 read per key, ~6 FP32 ops per pair - bound by HBM, not arithmetic, so
-// no tensor cores (no dense contraction here).
+// per-key work is then a d/2-pair dot product plus d/2 magnitudes against
+// per-row constants: d x 2 bytes of bf16 (d bytes of fp8) read per key, ~6 FP32
+// ops per pair - bound by HBM, not arithmetic, so no tensor cores (there is no
+// dense contraction here).
 //
 // For a cache of pre-RoPE keys, the literal one-(sin, cos)-per-(key, pair)
 // form is used instead: A'_f = (1/G) sum_g qbar_f^g sum_delta e^{i w_f delta}
@@ -23,14 +24,16 @@
 // turn (integer multiply mod 2^64), so fp32 never holds a large angle.
 //
 // prep_kernel (prep.cu) forms A_f, c_f per row in fp64 and stores fp32.
-// score_kernel
-// streams the keys: each warp owns a contiguous span of the concatenated key
-// space (all rows end to end, so ragged rows balance across the whole grid);
-// per batch of 32 keys, lane (q, g) loads the 16-byte real and imaginary
-// halves of pairs 8g..8g+7 for keys 4u+q, u = 0..7 (two full 128-byte lines
-// per key per instruction), accumulates 8 pairs in fp32, and a butterfly
-// reduce-scatter over the 8 lanes of a key leaves lane i holding key i's
-// score for one coalesced 128-byte store.
+// score_kernel streams the keys: each warp owns a contiguous span of the
+// concatenated key space (all rows end to end, so ragged rows balance across
+// the whole grid).  A key of head dim d is shared by d/16 lanes, each owning 8
+// frequency pairs (with rotate-half RoPE: 8 consecutive real parts and the 8
+// matching imaginary parts d/2 elements later; with interleaved RoPE: 16
+// consecutive elements), so a warp instruction covers 32 / (d/16) keys'
+// records.  Every lane keeps U keys' loads in flight (U = 4 for d = 64, else
+// 8), accumulates its 8 pairs in fp32, and a butterfly reduce-scatter over the
+// lanes of a key leaves one full score per lane; a shuffle orders them for one
+// coalesced store per batch (32 keys, 16 for d = 256).
 #include "tri_internal.cuh"
 
 namespace tri {
@@ -49,7 +52,7 @@ struct RowCtx {
     float ar[8], ai[8], cc[8];
 };
 
-__device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, int g) {
+__device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, int gl, int coef_per_row) {
     const Geometry &geo = p.geo;
     c.r = r;
     c.lo = geo.row_off[r];
@@ -61,7 +64,7 @@ __device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, 
     c.table = geo.block_table + (int64_t)s * geo.max_blocks;
     c.layer_blk = (int64_t)l * geo.n_blocks;
     c.p_now = p.p_now[s];
-    const float4 *cp = reinterpret_cast<const float4 *>(p.coef + (int64_t)r * kCoefPerRow + g * kCoefPerGroup);
+    const float4 *cp = reinterpret_cast<const float4 *>(p.coef + (int64_t)r * coef_per_row + gl * kCoefPerGroup);
     const float4 v0 = cp[0], v1 = cp[1], v2 = cp[2], v3 = cp[3], v4 = cp[4], v5 = cp[5];
     c.ar[0] = v0.x; c.ar[1] = v0.y; c.ar[2] = v0.z; c.ar[3] = v0.w;
     c.ar[4] = v1.x; c.ar[5] = v1.y; c.ar[6] = v1.z; c.ar[7] = v1.w;
@@ -103,19 +106,30 @@ __device__ __forceinline__ void unpack_e4m3x8(const uint2 v, float (&x)[8]) {
     x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
 }
 
-// Lane g's share of one key record: the real parts (dims 8g..8g+7) and the
-// imaginary parts (dims 64+8g..64+8g+7) of pairs 8g..8g+7, as stored - 2 x 16
-// bytes for bf16, 2 x 8 bytes for fp8 e4m3.  A warp instruction covers four
-// keys' halves, each a contiguous 128 (bf16) or 64 (fp8) bytes.
-template <int ELEM>
+__device__ __forceinline__ void unpack_bf16_pairs(const uint4 a, const uint4 b, float (&x)[8], float (&y)[8]) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        x[i] = bf16lo(w[i]);
+        y[i] = bf16hi(w[i]);
+    }
+}
+
+// Lane gl's share of one key record, as stored: the 8 pairs 8gl .. 8gl+7 of a
+// key with F = d/2 pairs.  Rotate-half (IL = false): real parts at dims
+// 8gl..8gl+7, imaginary parts F dims later - 2 x 16 bytes for bf16, 2 x 8 bytes
+// for fp8.  Interleaved (IL = true): dims 16gl..16gl+15, (re, im) adjacent -
+// 32 bytes for bf16, 16 for fp8.  Every load is naturally aligned: records are
+// 64..512 bytes long and start at multiples of their length from K.
+template <int ELEM, bool IL, int F>
 struct KeyChunk;
 
-template <>
-struct KeyChunk<2> {
+template <int F>
+struct KeyChunk<2, false, F> {
     uint4 re, im;
-    __device__ __forceinline__ void load(const char *key, int g, unsigned long long pol) {
-        re = ld_stream16(key + 16 * g, pol);
-        im = ld_stream16(key + 2 * kF + 16 * g, pol);
+    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
+        re = ld_stream16(key + 16 * gl, pol);
+        im = ld_stream16(key + 2 * F + 16 * gl, pol);
     }
     __device__ __forceinline__ void zero() { re = im = make_uint4(0u, 0u, 0u, 0u); }
     __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
@@ -124,17 +138,48 @@ struct KeyChunk<2> {
     }
 };
 
-template <>
-struct KeyChunk<1> {
+template <int F>
+struct KeyChunk<1, false, F> {
     uint2 re, im;
-    __device__ __forceinline__ void load(const char *key, int g, unsigned long long pol) {
-        re = ld_stream8(key + 8 * g, pol);
-        im = ld_stream8(key + kF + 8 * g, pol);
+    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
+        re = ld_stream8(key + 8 * gl, pol);
+        im = ld_stream8(key + F + 8 * gl, pol);
     }
     __device__ __forceinline__ void zero() { re = im = make_uint2(0u, 0u); }
     __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
         unpack_e4m3x8(re, x);
         unpack_e4m3x8(im, y);
+    }
+};
+
+template <int F>
+struct KeyChunk<2, true, F> {
+    uint4 a, b;
+    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
+        a = ld_stream16(key + 32 * gl, pol);
+        b = ld_stream16(key + 32 * gl + 16, pol);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const { unpack_bf16_pairs(a, b, x, y); }
+};
+
+template <int F>
+struct KeyChunk<1, true, F> {
+    uint4 v;
+    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
+        v = ld_stream16(key + 16 * gl, pol);
+    }
+    __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float2 p0 = e4m3x2_to_float2(w[i]), p1 = e4m3x2_to_float2(w[i] >> 16);
+            x[2 * i] = p0.x;
+            y[2 * i] = p0.y;
+            x[2 * i + 1] = p1.x;
+            y[2 * i + 1] = p1.y;
+        }
     }
 };
 
@@ -171,49 +216,64 @@ __device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&
     return (a0 + a1) + a2;
 }
 
-template <bool PRE, int ELEM>
-__device__ __forceinline__ float chunk_partial(const KeyChunk<ELEM> &kc, const RowCtx &c,
-                                               const unsigned long long (&T)[8], int64_t delta) {
+template <bool PRE, typename Chunk>
+__device__ __forceinline__ float chunk_partial(const Chunk &kc, const RowCtx &c, const unsigned long long (&T)[8],
+                                               int64_t delta) {
     float x[8], y[8];
     kc.unpack(x, y);
     return PRE ? partial_pre(x, y, c, T, delta) : partial_post(x, y, c);
 }
 
-template <bool PAGED, bool PRE, int ELEM>
-__device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx &c, int64_t k, int g,
+// Compile-time shape of one instantiation: LPK lanes per key (d / 16), NG keys
+// per warp instruction, U keys per lane per batch, KB keys per batch.
+template <int LPK>
+struct Shape {
+    static constexpr int NG = 32 / LPK;
+    static constexpr int U = LPK == 4 ? 4 : 8;
+    static constexpr int KB = NG * U;
+    static constexpr int F = 8 * LPK;
+};
+
+template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
+__device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx &c, int64_t k, int gl,
                                              unsigned long long pol, const unsigned long long (&T)[8]) {
+    constexpr int F = Shape<LPK>::F;
     const int64_t slot = key_slot<PAGED>(p, c, k);
     if (slot < 0) {
         atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
         return 0.f;
     }
-    KeyChunk<ELEM> kc;
-    kc.load(p.K + slot * (kD * ELEM), g, pol);
+    KeyChunk<ELEM, IL, F> kc;
+    kc.load(p.K + slot * (2 * F * ELEM), gl, pol);
     const int64_t delta = PRE ? c.p_now - (int64_t)__ldg(p.pos + slot) : 0;
-    return chunk_partial<PRE, ELEM>(kc, c, T, delta);
+    return chunk_partial<PRE>(kc, c, T, delta);
 }
 
-template <bool PAGED, bool PRE, int ELEM>
+template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
 __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const ScoreParams p) {
+    using Sh = Shape<LPK>;
+    constexpr int NG = Sh::NG, U = Sh::U, KB = Sh::KB, F = Sh::F;
+    constexpr int RB = 2 * F * ELEM;  // record bytes
     grid_dependency_wait();
     grid_dependents_launch();
     const Geometry &geo = p.geo;
     const int lane = threadIdx.x & 31;
-    const int q = lane >> 3;  // key of the 4-key group
-    const int g = lane & 7;   // pairs 8g .. 8g+7
+    const int q = lane / LPK;   // key of the NG-key group
+    const int gl = lane % LPK;  // pairs 8gl .. 8gl+7
     const int64_t nwarps = (int64_t)gridDim.x * (kScoreThreads / 32);
     const int64_t wid = (int64_t)blockIdx.x * (kScoreThreads / 32) + (threadIdx.x >> 5);
     const int64_t total = geo.total;
     int64_t per = (total + nwarps - 1) / nwarps;
-    per = (per + 31) & ~int64_t(31);
+    per = (per + KB - 1) / KB * KB;
     const int64_t beg = wid * per;
     const int64_t end = min(total, beg + per);
     if (beg >= end) return;
     const int R = geo.L * geo.S * geo.H;
+    const int cpr = LPK * kCoefPerGroup;
 
     unsigned long long T[8];
 #pragma unroll
-    for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * g + i] : 0ull;
+    for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * gl + i] : 0ull;
     const unsigned long long pol = policy_evict_first();
 
     // Row holding key `beg`: the last r with row_off[r] <= beg.
@@ -226,21 +286,21 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
     int r0 = rl;
     while (r0 < R - 1 && geo.row_off[r0 + 1] <= beg) r0++;
     RowCtx c;
-    set_row(c, p, r0, g);
+    set_row(c, p, r0, gl, cpr);
 
-    for (int64_t b0 = beg; b0 < end; b0 += 32) {
-        const int64_t bend = min(b0 + 32, end);
-        float part[8];
-        if (bend == b0 + 32 && b0 >= c.lo && bend <= c.hi) {
-            // Whole batch inside the current row: issue all 16 loads, then compute.
-            KeyChunk<ELEM> kc[8];
-            int64_t slot[8];
-            int32_t kpos[8];
+    for (int64_t b0 = beg; b0 < end; b0 += KB) {
+        const int64_t bend = min(b0 + KB, end);
+        float part[U];
+        if (bend == b0 + KB && b0 >= c.lo && bend <= c.hi) {
+            // Whole batch inside the current row: issue all loads, then compute.
+            KeyChunk<ELEM, IL, F> kc[U];
+            int64_t slot[U];
+            int32_t kpos[U];
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
-                slot[u] = key_slot<PAGED>(p, c, b0 + 4 * u + q);
+            for (int u = 0; u < U; u++) {
+                slot[u] = key_slot<PAGED>(p, c, b0 + NG * u + q);
                 if (slot[u] >= 0) {
-                    kc[u].load(p.K + slot[u] * (kD * ELEM), g, pol);
+                    kc[u].load(p.K + slot[u] * RB, gl, pol);
                     kpos[u] = PRE ? __ldg(p.pos + slot[u]) : 0;
                 } else {
                     kc[u].zero();
@@ -248,25 +308,25 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 8; u++) {
+            for (int u = 0; u < U; u++) {
                 if (PAGED && slot[u] < 0) {
                     atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
                     part[u] = 0.f;
                 } else {
-                    part[u] = chunk_partial<PRE, ELEM>(kc[u], c, T, c.p_now - (int64_t)kpos[u]);
+                    part[u] = chunk_partial<PRE>(kc[u], c, T, c.p_now - (int64_t)kpos[u]);
                 }
             }
         } else {
             // Batch crosses a row boundary or the span end: one segment per row.
 #pragma unroll
-            for (int u = 0; u < 8; u++) part[u] = 0.f;
+            for (int u = 0; u < U; u++) part[u] = 0.f;
             int64_t k0 = b0;
             for (;;) {
                 const int64_t seg_end = min(bend, c.hi);
 #pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    const int64_t k = b0 + 4 * u + q;
-                    if (k >= k0 && k < seg_end) part[u] += key_partial<PAGED, PRE, ELEM>(p, c, k, g, pol, T);
+                for (int u = 0; u < U; u++) {
+                    const int64_t k = b0 + NG * u + q;
+                    if (k >= k0 && k < seg_end) part[u] += key_partial<PAGED, PRE, ELEM, IL, LPK>(p, c, k, gl, pol, T);
                 }
                 if (bend <= c.hi) break;
                 k0 = max(k0, c.hi);
@@ -276,61 +336,74 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
                     atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
                     break;
                 }
-                set_row(c, p, r, g);
+                set_row(c, p, r, gl, cpr);
                 if (c.lo != k0) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
             }
         }
-        // Butterfly reduce-scatter over the 8 lanes (bits of g) sharing a key:
-        // afterwards lane (q, g) holds the full score of key 4g + q.
-        {
-            const bool h2 = (g >> 2) & 1;
+        // Butterfly reduce-scatter over the lanes sharing a key: at the stage of
+        // lane bit `half`, a lane keeps the upper or lower half of its partials
+        // and adds its partner's copy of that half.  Afterwards lane (q, gl) holds
+        // key NG * (gl % U) + q summed over the lanes that differ from it in the
+        // low log2(U) bits of gl; with LPK = 2U one more exchange adds the other
+        // half of the pairs.
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float send = h2 ? part[i] : part[i + 4];
-                const float keep = h2 ? part[i + 4] : part[i];
-                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-            }
-            const bool h1 = (g >> 1) & 1;
+        for (int half = U / 2; half >= 1; half >>= 1) {
+            const bool up = (gl & half) != 0;
 #pragma unroll
-            for (int i = 0; i < 2; i++) {
-                const float send = h1 ? part[i] : part[i + 2];
-                const float keep = h1 ? part[i + 2] : part[i];
-                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+            for (int i = 0; i < half; i++) {
+                const float send = up ? part[i] : part[i + half];
+                const float keep = up ? part[i + half] : part[i];
+                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
             }
-            const bool h0 = g & 1;
-            const float send = h0 ? part[0] : part[1];
-            const float keep = h0 ? part[1] : part[0];
-            part[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
         }
-        const float v = __shfl_sync(0xffffffffu, part[0], 8 * (lane & 3) + (lane >> 2));
-        if (b0 + lane < bend) p.scores[b0 + lane] = v;
+        if (LPK > U) part[0] += __shfl_xor_sync(0xffffffffu, part[0], U);
+        // Lane i < KB stores key b0 + i, held by lane (i % NG) * LPK + i / NG.
+        const int src = lane < KB ? (lane % NG) * LPK + lane / NG : lane;
+        const float v = __shfl_sync(0xffffffffu, part[0], src);
+        if (lane < KB && b0 + lane < bend) p.scores[b0 + lane] = v;
     }
 }
 
-template <bool PAGED, bool PRE, int ELEM>
+template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
 static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
+    auto kern = score_kernel<PAGED, PRE, ELEM, IL, LPK>;
     static int occ[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     int &o = occ[dev & 63];
     if (o == 0) {
-        cudaError_t e =
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, score_kernel<PAGED, PRE, ELEM>, kScoreThreads, 0);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kScoreThreads, 0);
         if (e != cudaSuccess) return e;
         if (o < 1) o = 1;
     }
-    const int64_t want = (p.geo.total + 32 * (kScoreThreads / 32) - 1) / (32 * (kScoreThreads / 32));
+    constexpr int KB = Shape<LPK>::KB;
+    const int64_t want = (p.geo.total + KB * (kScoreThreads / 32) - 1) / (KB * (kScoreThreads / 32));
     int64_t grid = (int64_t)sm_count() * o;
     if (want < grid) grid = want;
     if (grid < 1) grid = 1;
-    return launch_pdl(score_kernel<PAGED, PRE, ELEM>, dim3((unsigned)grid), dim3(kScoreThreads), 0, s, p);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kScoreThreads), 0, s, p);
+}
+
+template <int ELEM, bool IL, int LPK>
+static cudaError_t launch_score_d(const ScoreParams &p, int pre_rope, cudaStream_t s) {
+    if (p.geo.layout == TRI_KV_PAGED)
+        return pre_rope ? launch_score_t<true, true, ELEM, IL, LPK>(p, s) : launch_score_t<true, false, ELEM, IL, LPK>(p, s);
+    return pre_rope ? launch_score_t<false, true, ELEM, IL, LPK>(p, s) : launch_score_t<false, false, ELEM, IL, LPK>(p, s);
+}
+
+template <int ELEM, bool IL>
+static cudaError_t launch_score_l(const ScoreParams &p, int pre_rope, cudaStream_t s) {
+    switch (p.geo.D) {
+        case 64: return launch_score_d<ELEM, IL, 4>(p, pre_rope, s);
+        case 128: return launch_score_d<ELEM, IL, 8>(p, pre_rope, s);
+        case 256: return launch_score_d<ELEM, IL, 16>(p, pre_rope, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 template <int ELEM>
 static cudaError_t launch_score_e(const ScoreParams &p, int pre_rope, cudaStream_t s) {
-    const bool paged = p.geo.layout == TRI_KV_PAGED;
-    if (paged) return pre_rope ? launch_score_t<true, true, ELEM>(p, s) : launch_score_t<true, false, ELEM>(p, s);
-    return pre_rope ? launch_score_t<false, true, ELEM>(p, s) : launch_score_t<false, false, ELEM>(p, s);
+    return p.geo.il ? launch_score_l<ELEM, true>(p, pre_rope, s) : launch_score_l<ELEM, false>(p, pre_rope, s);
 }
 
 cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s) {

@@ -9,9 +9,10 @@
 // the same computation as tri_score with the workspace replaced by a fixed
 // scratch array compiled into the library.
 //
-// The scratch is one file-scope __device__ array of kNoAllocBytes (1 KiB of
-// flag word and turn table plus 768 B of coefficients per row, for at most
-// TRI_NOALLOC_MAX_ROWS = 4096 rows: about 3 MiB).  Every GPU that loads the
+// The scratch is one file-scope __device__ array of kNoAllocBytes (1.25 KiB of
+// flag word and turn table plus up to 1536 B of coefficients per row - 6 B per
+// head dim - for at most TRI_NOALLOC_MAX_ROWS = 4096 rows at the largest head
+// dim, 256: about 6 MiB).  Every GPU that loads the
 // library holds its own copy until the process exits.  In host code the
 // array's name only stands in for it; the device address is fetched once per
 // device with cudaGetSymbolAddress, on the first call made with that device
@@ -23,7 +24,8 @@
 namespace {
 
 constexpr int64_t kNoAllocMaxRows = TRI_NOALLOC_MAX_ROWS;
-constexpr size_t kNoAllocBytes = tri::kWsCoef + (size_t)kNoAllocMaxRows * tri::kCoefPerRow * sizeof(float);
+constexpr size_t kNoAllocBytes =
+    tri::kWsCoef + (size_t)kNoAllocMaxRows * (3 * tri::kMaxF) * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_score_scratch[kNoAllocBytes];
 

@@ -13,24 +13,26 @@
 
 namespace tri {
 
-constexpr int kD = TRI_HEAD_DIM;  // head dim
-constexpr int kF = kD / 2;        // frequency pairs
-constexpr int kCoefPerGroup = 24; // 8 pairs x (Re A, Im A, c)
-constexpr int kCoefPerRow = 8 * kCoefPerGroup;
+constexpr int kMaxD = 256;            // largest supported head dim
+constexpr int kMaxF = kMaxD / 2;      // its frequency pairs
+constexpr int kCoefPerGroup = 24;     // 8 pairs x (Re A, Im A, c)
+inline int coef_per_row(int D) { return (D / 16) * kCoefPerGroup; }  // 3 floats per pair
 
 // Workspace layout (byte offsets from the 256-byte aligned base).
 constexpr size_t kWsFlags = 0;       // uint32 flag word
-constexpr size_t kWsTurns = 256;     // uint64 [64]: w_f / 2pi in 0.64 fixed point
-constexpr size_t kWsCoef = 1024;     // float [R][8][24]
-inline size_t ws_coef_bytes(int64_t R) { return ((size_t)R * kCoefPerRow * 4 + 255) & ~size_t(255); }
-inline size_t ws_idx_offset(int64_t R) { return kWsCoef + ws_coef_bytes(R); }
-inline size_t ws_total(int64_t R, int64_t B) {
-    return ws_idx_offset(R) + (((size_t)R * (size_t)B * 4 + 255) & ~size_t(255));
+constexpr size_t kWsTurns = 256;     // uint64 [d/2 <= 128]: w_f / 2pi in 0.64 fixed point
+constexpr size_t kWsCoef = 1280;     // float [R][d/16][24]
+inline size_t ws_coef_bytes(int64_t R, int D) { return ((size_t)R * coef_per_row(D) * 4 + 255) & ~size_t(255); }
+inline size_t ws_idx_offset(int64_t R, int D) { return kWsCoef + ws_coef_bytes(R, D); }
+inline size_t ws_total(int64_t R, int64_t B, int D) {
+    return ws_idx_offset(R, D) + (((size_t)R * (size_t)B * 4 + 255) & ~size_t(255));
 }
 
 struct Geometry {  // row numbering and cache addressing
     int32_t L, S, H, Hq, G;
     int32_t layout;
+    int32_t D;           // head dim: 64, 128 or 256
+    int32_t il;          // 1: interleaved RoPE pairs (2f, 2f+1); 0: rotate-half (f, f+D/2)
     int32_t elem_bytes;  // 2: bf16, 1: fp8 e4m3
     int32_t max_blocks, block_shift;  // paged: block_size = 1 << block_shift
     int64_t n_blocks;
@@ -89,6 +91,7 @@ struct GatherParams {
 };
 
 struct CalibParams {
+    int32_t D, il;
     const uint16_t *q;
     int64_t nq;
     int32_t n_heads;  // L * Hq

@@ -11,8 +11,9 @@ position-stable centres):
     exp(N(0,1)) and phase U[0, 2pi);
   * pre-RoPE key pairs k_f = mu_f + eps, eps real and imaginary parts i.i.d.
     N(0, (r |mu_f|)^2), r the head's noise ratio;
-  * keys are RoPE-rotated at their position (rotate-half pairs (f, f+d/2),
-    w_f = theta^(-2f/d), angles reduced in fp64) and rounded to bf16;
+  * keys are RoPE-rotated at their position (pairs (f, f+d/2) for
+    rotate-half RoPE, (2f, 2f+1) for interleaved RoPE; w_f = theta^(-2f/d),
+    angles reduced in fp64) and rounded to bf16;
   * calibration queries: every query head draws its own centres and ratio and
     its pre-RoPE queries the same way (not rotated);
   * values are i.i.d. N(0, 1) in bf16;
@@ -102,8 +103,21 @@ def layer_heads(wl: Workload, layer: int, device) -> LayerHeads:
     return LayerHeads(kre, kim, ksc, qre, qim, qsc, zero)
 
 
+def place_pairs(out: torch.Tensor, re: torch.Tensor, im: torch.Tensor, interleaved: bool) -> torch.Tensor:
+    """Write pair values into the last dim of ``out``: (f, f+d/2) or (2f, 2f+1)."""
+    F = out.shape[-1] // 2
+    if interleaved:
+        out[..., 0::2] = re
+        out[..., 1::2] = im
+    else:
+        out[..., :F] = re
+        out[..., F:] = im
+    return out
+
+
 def head_keys(heads: LayerHeads, h: int, positions: torch.Tensor, g: torch.Generator,
-              theta: float, d: int, rotate: bool = True, arange_n: int = 0) -> torch.Tensor:
+              theta: float, d: int, rotate: bool = True, arange_n: int = 0,
+              interleaved: bool = False) -> torch.Tensor:
     """Keys of KV head h at ``positions``: bf16 [n][d] (RoPE'd unless rotate=False)."""
     n = positions.shape[0]
     F = d // 2
@@ -116,10 +130,7 @@ def head_keys(heads: LayerHeads, h: int, positions: torch.Tensor, g: torch.Gener
         c, s = _rotation_arange(arange_n, theta, d, dev) if arange_n else rotation(positions, theta, d)
         c, s = c[:n], s[:n]
         kr, ki = kr * c - ki * s, kr * s + ki * c
-    out = torch.empty(n, d, dtype=torch.bfloat16, device=dev)
-    out[:, :F] = kr
-    out[:, F:] = ki
-    return out
+    return place_pairs(torch.empty(n, d, dtype=torch.bfloat16, device=dev), kr, ki, interleaved)
 
 
 def calib_queries(wl: Workload, layer: int, device, heads: LayerHeads = None) -> torch.Tensor:
@@ -130,9 +141,8 @@ def calib_queries(wl: Workload, layer: int, device, heads: LayerHeads = None) ->
     er = torch.randn(Hq, n, F, generator=g, device=device)
     ei = torch.randn(Hq, n, F, generator=g, device=device)
     out = torch.empty(Hq, n, wl.head_dim, dtype=torch.bfloat16, device=device)
-    out[..., :F] = heads.q_re[:, None, :] + heads.q_scale[:, None, :] * er
-    out[..., F:] = heads.q_im[:, None, :] + heads.q_scale[:, None, :] * ei
-    return out
+    return place_pairs(out, heads.q_re[:, None, :] + heads.q_scale[:, None, :] * er,
+                       heads.q_im[:, None, :] + heads.q_scale[:, None, :] * ei, wl.interleaved)
 
 
 @dataclass
@@ -194,7 +204,8 @@ def make_contig(wl: Workload, device, layers=None, lens=None, with_values: bool 
             for h in range(H):
                 a, b = int(row_off[r]), int(row_off[r + 1])
                 if n:
-                    K[a:b] = head_keys(heads, h, p, gk, wl.theta, d, rotate, arange_n=nmax)
+                    K[a:b] = head_keys(heads, h, p, gk, wl.theta, d, rotate, arange_n=nmax,
+                                       interleaved=wl.interleaved)
                     if V is not None:
                         V[a:b] = torch.randn(n, d, generator=gv, device=device).to(torch.bfloat16)
                     pos[a:b] = p.to(torch.int32)
@@ -250,7 +261,8 @@ def make_paged(wl: Workload, device, layer: int = 0, lens=None, max_blocks: int 
         blk = tt[s, p // bs]
         slot = p % bs
         for h in range(H):
-            K[blk, slot, h] = head_keys(heads, h, p, gk, wl.theta, d, True, arange_n=nmax)
+            K[blk, slot, h] = head_keys(heads, h, p, gk, wl.theta, d, True, arange_n=nmax,
+                                        interleaved=wl.interleaved)
             V[blk, slot, h] = torch.randn(n, d, generator=gv, device=device).to(torch.bfloat16)
             pos[blk, slot, h] = p.to(torch.int32)
     return PagedCache(wl, lens, K, V, pos, torch.as_tensor(table, device=device), table,
@@ -269,7 +281,7 @@ def decode_keys(wl: Workload, layer: int, round_idx: int, start: np.ndarray, cou
     for s in range(S):
         p = torch.arange(int(start[s]), int(start[s]) + count, device=device)
         for h in range(H):
-            Kn[s, :, h] = head_keys(heads, h, p, g, wl.theta, d, True)
+            Kn[s, :, h] = head_keys(heads, h, p, g, wl.theta, d, True, interleaved=wl.interleaved)
             Vn[s, :, h] = torch.randn(count, d, generator=g, device=device).to(torch.bfloat16)
     return Kn, Vn
 

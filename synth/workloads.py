@@ -30,6 +30,7 @@ class Workload:
     rescore_every: int = 0  # paged decode rounds: new tokens per round
     rounds: int = 0
     head_dim: int = 128
+    rope_style: str = "half"  # "half": pair f = dims (f, f+d/2); "interleaved": (2f, 2f+1)
     theta: float = 1e6
     n_calib: int = 1024  # calibration queries per query head
     seed: int = 20261202
@@ -37,6 +38,10 @@ class Workload:
     @property
     def offsets(self) -> list:
         return [2 ** e for e in range(self.n_offsets)]
+
+    @property
+    def interleaved(self) -> bool:
+        return self.rope_style == "interleaved"
 
     @property
     def group(self) -> int:

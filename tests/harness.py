@@ -30,7 +30,7 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return oracle.bf16_bits_to_f64(bits16(t))
 
 
-def oracle_calibration(qcal: torch.Tensor):
+def oracle_calibration(qcal: torch.Tensor, interleaved: bool = False):
     """Oracle calibration of queries bf16 [L][Hq][nq][d] -> (centres fp64 [L][Hq][F][2],
     mnorm fp64 [L][Hq][F])."""
     L, Hq, nq, d = qcal.shape
@@ -39,7 +39,7 @@ def oracle_calibration(qcal: torch.Tensor):
     ms = np.empty((L, Hq, d // 2))
     for l in range(L):
         for g in range(Hq):
-            cs[l, g], ms[l, g] = oracle.calib(q[l, g])
+            cs[l, g], ms[l, g] = oracle.calib(q[l, g], interleaved=interleaved)
     return cs, ms
 
 
@@ -48,7 +48,15 @@ def as_f32_exact(a: np.ndarray) -> np.ndarray:
     return np.asarray(a, dtype=np.float32).astype(np.float64)
 
 
-def series_bound(theta, centres_l, mnorms_l, h, G, keys, offsets) -> np.ndarray:
+def pair_norms(keys: np.ndarray, interleaved: bool = False) -> np.ndarray:
+    """|k_f| per key and pair: dims (f, f+d/2), or (2f, 2f+1) when interleaved."""
+    F = keys.shape[1] // 2
+    if interleaved:
+        return np.hypot(keys[:, 0::2], keys[:, 1::2])
+    return np.hypot(keys[:, :F], keys[:, F:])
+
+
+def series_bound(theta, centres_l, mnorms_l, h, G, keys, offsets, interleaved=False) -> np.ndarray:
     """Absolute-value bound M_j = sum_f (|A_f| + |c_f|) |k_f| of a row's score series
     (the scale the score tolerance is relative to; scores can cancel near 0)."""
     d = keys.shape[1]
@@ -59,7 +67,7 @@ def series_bound(theta, centres_l, mnorms_l, h, G, keys, offsets) -> np.ndarray:
     qc = qb[..., 0] + 1j * qb[..., 1]
     Q = qc.mean(axis=0)
     c = (mnorms_l[h * G:(h + 1) * G] - np.abs(qc)).mean(axis=0)
-    kn = np.hypot(keys[:, :F], keys[:, F:])
+    kn = pair_norms(keys, interleaved)
     return kn @ (np.abs(Q) * np.abs(S) + np.abs(c))
 
 

@@ -48,7 +48,12 @@ def test_workspace_size():
     assert n >= R * 768 + R * 2048 * 4 and n % 256 == 0
     assert tri.tri_workspace_size(m, 0, 2048) == 0
     assert tri.tri_workspace_size(m, 1, 0) == 0
-    assert tri.tri_workspace_size(tri.model(1, 32, 8, 1e6, head_dim=64), 1, 16) == 0
+    assert tri.tri_workspace_size(tri.model(1, 32, 8, 1e6, head_dim=96), 1, 16) == 0
+    assert tri.tri_workspace_size(tri.model(1, 32, 8, 1e6, rope_style=2), 1, 16) == 0
+    # per-row coefficients: 3 floats per pair, d/2 pairs
+    for d in (64, 128, 256):
+        md = tri.model(36, 32, 8, 1e6, head_dim=d, rope_style=tri.TRI_ROPE_INTERLEAVED)
+        assert tri.tri_workspace_size(md, 1, 2048) >= R * 6 * d + R * 2048 * 4
 
 
 # Fake (never dereferenced) device addresses: the host checks run first.
@@ -97,7 +102,9 @@ def test_score_rejects_bad_arguments(kwargs, status):
 
 
 def test_score_rejects_bad_model_and_layout():
-    assert _score(tri.model(1, 32, 8, 1e6, head_dim=64), _kv()) == _abi.TRI_ERR_UNSUPPORTED
+    assert _score(tri.model(1, 32, 8, 1e6, head_dim=96), _kv()) == _abi.TRI_ERR_UNSUPPORTED
+    assert _score(tri.model(1, 32, 8, 1e6, head_dim=512), _kv()) == _abi.TRI_ERR_UNSUPPORTED
+    assert _score(tri.model(1, 32, 8, 1e6, rope_style=-1), _kv()) == _abi.TRI_ERR_INVALID_ARG
     assert _score(tri.model(1, 30, 8, 1e6), _kv()) == _abi.TRI_ERR_INVALID_ARG
     assert _score(tri.model(1, 32, 8, 0.5), _kv()) == _abi.TRI_ERR_INVALID_ARG
     assert _score(tri.model(0, 32, 8, 1e6), _kv()) == _abi.TRI_ERR_INVALID_ARG

@@ -22,7 +22,8 @@ POST, PRE = tri.TRI_KEYS_POST_ROPE, tri.TRI_KEYS_PRE_ROPE
 
 
 def model_of(wl, n_layers):
-    return tri.model(n_layers, wl.n_q_heads, wl.n_kv_heads, wl.theta)
+    style = tri.TRI_ROPE_INTERLEAVED if wl.interleaved else tri.TRI_ROPE_HALF
+    return tri.model(n_layers, wl.n_q_heads, wl.n_kv_heads, wl.theta, head_dim=wl.head_dim, rope_style=style)
 
 
 def to_dev(cache: synth.ContigCache) -> synth.ContigCache:
@@ -35,7 +36,7 @@ def to_dev(cache: synth.ContigCache) -> synth.ContigCache:
 
 
 def oracle_centres(cache):
-    cs, ms = H.oracle_calibration(cache.qcal)
+    cs, ms = H.oracle_calibration(cache.qcal, cache.wl.interleaved)
     return H.as_f32_exact(cs), H.as_f32_exact(ms)
 
 
@@ -52,8 +53,9 @@ def oracle_scores(cache, cs, ms, post_rope=True, tier="literal", rows=None):
         if b == a:
             continue
         out[a:b] = oracle.row_scores(wl.theta, cs[li], ms[li], h, wl.group, K[a:b], pos[a:b],
-                                     post_rope, int(cache.lens[s]), wl.offsets, tier)
-        bounds[a:b] = H.series_bound(wl.theta, cs[li], ms[li], h, wl.group, K[a:b], wl.offsets)
+                                     post_rope, int(cache.lens[s]), wl.offsets, tier, wl.interleaved)
+        bounds[a:b] = H.series_bound(wl.theta, cs[li], ms[li], h, wl.group, K[a:b], wl.offsets,
+                                     wl.interleaved)
     return out, bounds
 
 
@@ -61,7 +63,7 @@ def gpu_score(cache, cs, ms, key_mode=POST, B=1):
     wl = cache.wl
     m = model_of(wl, len(cache.layers))
     S = len(cache.lens)
-    kv = tri.kv_contig(S, cache.row_off, cache.total)
+    kv = tri.kv_contig(S, cache.row_off, cache.total, tri.elem_type_of(cache.K))
     c32 = torch.tensor(cs, dtype=torch.float32, device=DEV)
     m32 = torch.tensor(ms, dtype=torch.float32, device=DEV)
     ws = tri.alloc_workspace(m, S, B)
@@ -77,10 +79,10 @@ def gpu_compact(cache, scores, B, W):
     m = model_of(wl, len(cache.layers))
     S = len(cache.lens)
     R = cache.n_rows
-    kv = tri.kv_contig(S, cache.row_off, cache.total)
+    kv = tri.kv_contig(S, cache.row_off, cache.total, tri.elem_type_of(cache.K))
     ws = tri.alloc_workspace(m, S, B)
-    Ko = torch.zeros(R, B, 128, dtype=torch.bfloat16, device=DEV)
-    Vo = torch.zeros(R, B, 128, dtype=torch.bfloat16, device=DEV)
+    Ko = torch.zeros(R, B, wl.head_dim, dtype=cache.K.dtype, device=DEV)
+    Vo = torch.zeros(R, B, wl.head_dim, dtype=cache.K.dtype, device=DEV)
     po = torch.full((R, B), -7, dtype=torch.int32, device=DEV)
     kept = torch.full((R, B), -1, dtype=torch.int32, device=DEV)
     cnt = torch.full((R,), -1, dtype=torch.int32, device=DEV)
@@ -93,9 +95,9 @@ def gpu_compact(cache, scores, B, W):
 
 def check_compaction_exact(cache, res, ref_scores32, B, W):
     """Kept sets == oracle.select of the same fp32 scores; K/V/pos == oracle.gather."""
-    Kb, Vb = H.bits16(cache.K), H.bits16(cache.V)
+    Kb, Vb = H.raw_bits(cache.K), H.raw_bits(cache.V)
     pos = cache.pos.cpu().numpy()
-    Kob, Vob = res["K"].view(torch.int16).numpy(), res["V"].view(torch.int16).numpy()
+    Kob, Vob = H.raw_bits(res["K"]), H.raw_bits(res["V"])
     for r in range(cache.n_rows):
         a, b = cache.row_off_np[r], cache.row_off_np[r + 1]
         ref = oracle.select(ref_scores32[a:b], B, W)
