@@ -70,6 +70,14 @@ def _declare(L) -> None:
         fn = getattr(L, name)
         fn.restype = None
         fn.argtypes = score_args
+    L.ora_calib_online.restype = None
+    L.ora_calib_online.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, _f64p, _i64p, ctypes.c_int64,
+                                   ctypes.c_double, _f64p, _f64p]
+    L.ora_key_centres.restype = None
+    L.ora_key_centres.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int64, _f64p, _i64p,
+                                  ctypes.c_int, _f64p, _f64p]
+    L.ora_calib_stats.restype = None
+    L.ora_calib_stats.argtypes = [ctypes.c_int, _f64p, _f64p, ctypes.c_void_p, ctypes.c_void_p, _f64p, _f64p]
     L.ora_select.restype = ctypes.c_int64
     L.ora_select.argtypes = [ctypes.c_int64, _f64p, ctypes.c_int64, ctypes.c_int64, _i64p]
     L.ora_gather_bytes.restype = None
@@ -135,6 +143,49 @@ def calib(q: np.ndarray, interleaved: bool = False):
     mnorm = np.empty(d // 2)
     lib().ora_calib(d, int(bool(interleaved)), nq, q, centre, mnorm)
     return centre, mnorm
+
+
+def calib_online(batches, decay: float = 1.0, interleaved: bool = False):
+    """Centres after a stream of query batches (each [n_b][d]) where every new batch
+    multiplies the weight of all earlier queries by ``decay``.  Returns (centre, mnorm)."""
+    q = _f64(np.concatenate([np.asarray(b, dtype=np.float64) for b in batches], axis=0))
+    upd = _i64(np.concatenate([np.full(len(b), i) for i, b in enumerate(batches)]))
+    d = q.shape[1]
+    centre = np.empty((d // 2, 2))
+    mnorm = np.empty(d // 2)
+    lib().ora_calib_online(d, int(bool(interleaved)), q.shape[0], q, upd, len(batches), float(decay), centre,
+                           mnorm)
+    return centre, mnorm
+
+
+def key_centres(theta: float, keys: np.ndarray, pos: np.ndarray, post_rope: bool,
+                interleaved: bool = False):
+    """Pre-RoPE key centre [F][2] and mean magnitude [F] of one row's keys [n][d]
+    (de-rotated by their positions when ``post_rope``)."""
+    keys = _f64(keys)
+    n, d = keys.shape
+    pos = _i64(pos)
+    centre = np.empty((d // 2, 2))
+    mnorm = np.empty(d // 2)
+    lib().ora_key_centres(d, int(bool(interleaved)), float(theta), n, keys, pos, 1 if post_rope else 0, centre,
+                          mnorm)
+    return centre, mnorm
+
+
+def calib_stats(centre: np.ndarray, mnorm: np.ndarray, ref_centre=None, ref_mnorm=None):
+    """(concentration [F], (head concentration, drift vs the reference)) of one head."""
+    centre = _f64(centre)
+    mnorm = _f64(mnorm)
+    F = mnorm.shape[0]
+    conc = np.empty(F)
+    head = np.empty(2)
+    if ref_centre is None:
+        lib().ora_calib_stats(F, centre, mnorm, None, None, conc, head)
+    else:
+        rc, rm = _f64(ref_centre), _f64(ref_mnorm)
+        lib().ora_calib_stats(F, centre, mnorm, rc.ctypes.data_as(ctypes.c_void_p),
+                              rm.ctypes.data_as(ctypes.c_void_p), conc, head)
+    return conc, (float(head[0]), float(head[1]))
 
 
 def _score(fn, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets, interleaved=False):

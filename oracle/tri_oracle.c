@@ -386,3 +386,98 @@ void ora_gather_bytes(int64_t n, const int64_t *idx, int64_t width, const unsign
     for (int64_t t = 0; t < n; t++)
         memcpy(dst + t * width, src + idx[t] * width, (size_t)width);
 }
+
+/* ------------------------------------------------- calibration, continued */
+
+/*
+ * Online (decode-time) centre update, written as the weighted statistics it
+ * maintains.  Queries arrive in n_updates batches; query t came with batch
+ * update_of[t] (0 .. n_updates-1), and each later batch multiplies the weight
+ * of everything seen before it by `decay` (0 < decay <= 1; 1 keeps the plain
+ * mean of every query seen).  So query t carries the weight
+ *   w_t = decay^(n_updates - 1 - update_of[t]),
+ * and per pair f
+ *   centre_f = sum_t w_t q_f(t) / sum_t w_t,   mnorm_f = sum_t w_t |q_f(t)| / sum_t w_t,
+ * the centres of digest step 1 over a (decayed) stream of queries.
+ *   q: [nq][d] pre-RoPE queries of one head; centre: [F][2]; mnorm: [F].
+ */
+void ora_calib_online(int d, int il, int64_t nq, const double *q, const int64_t *update_of,
+                      int64_t n_updates, double decay, double *centre, double *mnorm)
+{
+    const int F = d / 2;
+    for (int f = 0; f < F; f++) {
+        int ire, iim;
+        pair_dims(d, il, f, &ire, &iim);
+        ldbl sr = 0.0L, si = 0.0L, sn = 0.0L, sw = 0.0L;
+        for (int64_t t = 0; t < nq; t++) {
+            ldbl w = powl((ldbl)decay, (ldbl)(n_updates - 1 - update_of[t]));
+            ldbl xr = q[t * d + ire], xi = q[t * d + iim];
+            sr += w * xr;
+            si += w * xi;
+            sn += w * hypotl(xr, xi);
+            sw += w;
+        }
+        centre[2 * f] = (double)(sr / sw);
+        centre[2 * f + 1] = (double)(si / sw);
+        mnorm[f] = (double)(sn / sw);
+    }
+}
+
+/*
+ * Key centres (digest, 流程详解 step 1: the pre-RoPE centres of Q *and* K): per
+ * pair f of one cache row, the complex mean of the pre-RoPE keys and the mean
+ * of their magnitudes.  post_rope != 0: the cached keys are de-rotated by their
+ * own positions first (key_pair).  An empty row has centre 0 and mnorm 0.
+ *   keys: [n][d], pos: [n]; centre: [F][2]; mnorm: [F].
+ */
+void ora_key_centres(int d, int il, double theta, int64_t n, const double *keys, const int64_t *pos,
+                     int post_rope, double *centre, double *mnorm)
+{
+    const int F = d / 2;
+    for (int f = 0; f < F; f++) {
+        ldbl w = omega_l(theta, d, f);
+        ldbl sr = 0.0L, si = 0.0L, sn = 0.0L;
+        for (int64_t j = 0; j < n; j++) {
+            ldbl kr, ki;
+            key_pair(d, il, keys + j * d, f, post_rope, w, pos[j], &kr, &ki);
+            sr += kr;
+            si += ki;
+            sn += hypotl(kr, ki);
+        }
+        centre[2 * f] = n ? (double)(sr / (ldbl)n) : 0.0;
+        centre[2 * f + 1] = n ? (double)(si / (ldbl)n) : 0.0;
+        mnorm[f] = n ? (double)(sn / (ldbl)n) : 0.0;
+    }
+}
+
+/*
+ * Concentration and drift of one head's statistics (the pages name Q/K
+ * concentration as the premise, digest section 核心洞见, and the sensitivity
+ * of the calibration to a shift between calibration and deployment data as an
+ * open risk, digest sections 不足 and 复现注意事项):
+ *   conc[f]  = |centre_f| / mnorm_f      (1: every query on the centre's
+ *              direction; near 0: directions spread out; 0 when mnorm_f = 0)
+ *   head[0]  = sum_f |centre_f| / sum_f mnorm_f      (0 when the sum is 0)
+ *   head[1]  = sum_f (|centre_f - ref_f| + |mnorm_f - ref_mnorm_f|) / sum_f ref_mnorm_f
+ *              (0 without a reference or when its norm sum is 0): the
+ *              relative L1 change of the two statistics the score uses.
+ *   centre, ref: [F][2]; mnorm, ref_mnorm: [F]; conc: [F]; head: [2].
+ */
+void ora_calib_stats(int F, const double *centre, const double *mnorm, const double *ref,
+                     const double *ref_mnorm, double *conc, double *head)
+{
+    ldbl sc = 0.0L, sm = 0.0L, dd = 0.0L, rm = 0.0L;
+    for (int f = 0; f < F; f++) {
+        ldbl a = hypotl(centre[2 * f], centre[2 * f + 1]);
+        conc[f] = mnorm[f] > 0.0 ? (double)(a / (ldbl)mnorm[f]) : 0.0;
+        sc += a;
+        sm += mnorm[f];
+        if (ref) {
+            dd += hypotl((ldbl)centre[2 * f] - ref[2 * f], (ldbl)centre[2 * f + 1] - ref[2 * f + 1]);
+            dd += fabsl((ldbl)mnorm[f] - ref_mnorm[f]);
+            rm += ref_mnorm[f];
+        }
+    }
+    head[0] = sm > 0.0L ? (double)(sc / sm) : 0.0;
+    head[1] = (ref && rm > 0.0L) ? (double)(dd / rm) : 0.0;
+}

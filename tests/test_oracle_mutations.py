@@ -44,6 +44,15 @@ MUTATIONS = [
      [("mnorm[f] = (double)(sn / (ldbl)nq);", "mnorm[f] = (double)hypotl(sr / (ldbl)nq, si / (ldbl)nq);")]),
     ("calibration drops the imaginary half",
      [("ldbl xr = q[t * d + ire], xi = q[t * d + iim];", "ldbl xr = q[t * d + ire], xi = 0.0L * q[t * d + iim];")]),
+    ("online decay favours older batches",
+     [("powl((ldbl)decay, (ldbl)(n_updates - 1 - update_of[t]))", "powl((ldbl)decay, (ldbl)update_of[t])")]),
+    ("online weights not normalised",
+     [("centre[2 * f] = (double)(sr / sw);", "centre[2 * f] = (double)(sr / (ldbl)nq);")]),
+    ("drift without the norm term",
+     [("dd += fabsl((ldbl)mnorm[f] - ref_mnorm[f]);", "dd += 0.0L;")]),
+    ("concentration inverted",
+     [("conc[f] = mnorm[f] > 0.0 ? (double)(a / (ldbl)mnorm[f]) : 0.0;",
+       "conc[f] = a > 0.0L ? (double)((ldbl)mnorm[f] / a) : 0.0;")]),
     ("tie-break keeps the older slot",
      [("if (a->i != b->i) return a->i > b->i ? -1 : 1;", "if (a->i != b->i) return a->i < b->i ? -1 : 1;")]),
     ("window not protected",
@@ -70,6 +79,9 @@ PIN_FUNCS = [
     lambda: pins.test_select_matches_lexsort_and_invariants(),
     lambda: pins.test_select_all_equal_keeps_most_recent(),
     lambda: pins.test_gather_matches_fancy_indexing(),
+    lambda: pins.test_calib_online_equals_weighted_mean(),
+    lambda: pins.test_key_centres_undo_rope(False),
+    lambda: pins.test_calib_stats_closed_forms(),
 ]
 
 

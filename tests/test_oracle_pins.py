@@ -465,3 +465,70 @@ def test_e4m3_decoding_matches_definition_and_torch():
     np.testing.assert_array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
     # hand-checked codes: 1.0, the largest finite 448, the smallest subnormal 2^-9, -2
     assert got[0x38] == 1.0 and got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0xC0] == -2.0
+
+
+# ------------------------------------------------ online centres, diagnostics
+
+def test_calib_online_equals_weighted_mean():
+    """decay = 1: the plain mean of every query seen (numpy, one concatenation);
+    decay < 1: numpy.average with weight decay^(batches after the query's own)."""
+    rng = np.random.default_rng(51)
+    d = 16
+    batches = [rng.standard_normal((n, d)) + 1.5 for n in (5, 1, 7, 3)]
+    q = np.concatenate(batches)
+    F = d // 2
+    c, m = oracle.calib_online(batches, 1.0)
+    np.testing.assert_allclose(c[:, 0], q[:, :F].mean(axis=0), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(c[:, 1], q[:, F:].mean(axis=0), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(m, np.hypot(q[:, :F], q[:, F:]).mean(axis=0), rtol=1e-14)
+    decay = 0.7
+    w = np.concatenate([np.full(len(b), decay ** (len(batches) - 1 - i)) for i, b in enumerate(batches)])
+    c, m = oracle.calib_online(batches, decay)
+    np.testing.assert_allclose(c[:, 0], np.average(q[:, :F], axis=0, weights=w), rtol=1e-13)
+    np.testing.assert_allclose(c[:, 1], np.average(q[:, F:], axis=0, weights=w), rtol=1e-13)
+    np.testing.assert_allclose(m, np.average(np.hypot(q[:, :F], q[:, F:]), axis=0, weights=w), rtol=1e-13)
+    ci, mi = oracle.calib_online(batches, decay, interleaved=True)
+    np.testing.assert_allclose(ci[:, 1], np.average(q[:, 1::2], axis=0, weights=w), rtol=1e-13)
+    np.testing.assert_allclose(mi, np.average(np.hypot(q[:, 0::2], q[:, 1::2]), axis=0, weights=w), rtol=1e-13)
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_key_centres_undo_rope(interleaved):
+    """Keys rotated by an explicit RoPE at random positions: their key centre is the
+    numpy mean of the pre-RoPE pairs; a pre-RoPE cache needs no positions."""
+    rng = np.random.default_rng(52 + interleaved)
+    d, theta, n = 64, 1e4, 40
+    pre = rng.standard_normal((n, d)) + 2.0
+    pos = rng.integers(0, 200000, size=n)
+    rope = rope_il_ld if interleaved else rope_ld
+    post = np.array([rope(pre[j], pos[j], theta) for j in range(n)], dtype=np.float64)
+    re, im = (pre[:, 0::2], pre[:, 1::2]) if interleaved else (pre[:, :d // 2], pre[:, d // 2:])
+    for keys, post_rope in ((post, True), (pre, False)):
+        c, m = oracle.key_centres(theta, keys, pos, post_rope, interleaved)
+        np.testing.assert_allclose(c[:, 0], re.mean(axis=0), rtol=0, atol=1e-12 * np.abs(re).max())
+        np.testing.assert_allclose(c[:, 1], im.mean(axis=0), rtol=0, atol=1e-12 * np.abs(im).max())
+        np.testing.assert_allclose(m, np.hypot(re, im).mean(axis=0), rtol=1e-12)
+    c, m = oracle.key_centres(theta, np.zeros((0, d)), np.zeros(0), True, interleaved)
+    assert np.all(c == 0) and np.all(m == 0)
+
+
+def test_calib_stats_closed_forms():
+    # one pair: centre 3+4i (|c| = 5), mean norm 10 -> concentration 1/2
+    conc, (hc, drift) = oracle.calib_stats(np.array([[3.0, 4.0]]), np.array([10.0]))
+    assert conc[0] == 0.5 and hc == 0.5 and drift == 0.0
+    # drift against centre 0, norm 5: (|3+4i - 0| + |10 - 5|) / 5 = 2
+    _, (_, drift) = oracle.calib_stats(np.array([[3.0, 4.0]]), np.array([10.0]), np.zeros((1, 2)), np.array([5.0]))
+    assert drift == 2.0
+    # all queries identical: every pair fully concentrated; q and -q: none
+    rng = np.random.default_rng(53)
+    q = rng.standard_normal(32)
+    c, m = oracle.calib(np.stack([q, q, q]))
+    conc, (hc, drift) = oracle.calib_stats(c, m, c, m)
+    np.testing.assert_allclose(conc, 1.0, rtol=1e-15)
+    assert abs(hc - 1.0) < 1e-15 and drift == 0.0
+    c, m = oracle.calib(np.stack([q, -q]))
+    conc, (hc, _) = oracle.calib_stats(c, m)
+    assert np.all(conc == 0.0) and hc == 0.0
+    # a zero-norm pair reports 0, not NaN
+    conc, (hc, _) = oracle.calib_stats(np.zeros((2, 2)), np.zeros(2))
+    assert np.all(conc == 0.0) and hc == 0.0
