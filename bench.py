@@ -102,7 +102,7 @@ def measured_peak():
 
 def score_kernel_sha():
     h = hashlib.sha256()
-    for f in ("score.cu", "tri_internal.cuh"):
+    for f in ("score.cu", "keys.cuh", "tri_internal.cuh"):
         with open(os.path.join(ROOT, "kv_cache_compression_calib_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -330,6 +330,8 @@ def run_ours(a, rank, world, local_rank):
     ms_step = ms / a.steps
     value = throughput(keys_step, world, ms_step)
 
+    diagnostics = time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream)
+
     # ---- end to end through the public API: pinned host inputs, copies in the region
     e2e = None
     if not a.no_e2e:
@@ -352,6 +354,7 @@ def run_ours(a, rank, world, local_rank):
         "path_roofline": {"bytes_per_step": alg_bytes, "achieved_gbs": path_gbs,
                           "frac_of_measured": path_gbs / peak, "frac_of_8tbs": path_gbs / NOMINAL_HBM_GBS},
         "calib_ms": calib_ms,
+        "diagnostics": diagnostics,
         "gpu_launches": 4 * a.steps,
         "clocks": clocks,
         "e2e": e2e,
@@ -359,6 +362,45 @@ def run_ours(a, rank, world, local_rank):
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, B, cache, a.cpu_seconds)
     return line
+
+
+def time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream, reps=5):
+    """Off-step calls, timed with CUDA events (mean of `reps` after one warm-up):
+    the key-centre pass over the whole cache (reads every key once: d x elem bytes
+    per key) and one online centre update with 64 new queries per head."""
+    D, L, Hq = wl.head_dim, wl.n_layers, wl.n_q_heads
+    R, S = cache.n_rows, len(cache.lens)
+    kc = torch.empty(R, D // 2, 2, device=dev)
+    kn = torch.empty(R, D // 2, device=dev)
+    kws = tri.alloc_key_centres_workspace(m, S, device=dev)
+    q = cache.qcal[:, :, :64].contiguous()
+    sums = torch.zeros(L, Hq, D // 2, 3, dtype=torch.float64, device=dev)
+    weight = torch.zeros(L, Hq, dtype=torch.float64, device=dev)
+    uc = torch.empty(L, Hq, D // 2, 2, device=dev)
+    un = torch.empty(L, Hq, D // 2, device=dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    kc_ms = timed(lambda: tri.tri_key_centres(m, kv, cache.K, cache.pos, key_mode, kc, kn, kws, stream))
+    st, flags = tri.tri_status_check(kws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} in the key-centre pass")
+    up_ms = timed(lambda: tri.tri_calib_update(m, q, 64, 0.99, sums, weight, uc, un, stream))
+    peak, kind = measured_peak()
+    kc_bytes = float(cache.total) * D * eb
+    return {"key_centres_ms": kc_ms, "key_centres_bytes": kc_bytes,
+            "key_centres_gbs": kc_bytes / (kc_ms / 1e3) / 1e9,
+            "key_centres_frac": kc_bytes / (kc_ms / 1e3) / 1e9 / peak, "peak_kind": kind,
+            "calib_update_ms": up_ms, "calib_update_queries_per_head": 64}
 
 
 def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream, world,

@@ -226,6 +226,68 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
 tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream);
 
 /*
+ * Online (decode-time) calibration update (digest, 流程详解 step 1, with the
+ * calibration/deployment shift the digest flags as a risk in sections 不足 and
+ * 复现注意事项): the centres of tri_calib maintained over a stream of query
+ * batches.  Each call, per (layer l, query head g):
+ *   sums   <- decay * sums + sum over this call's queries of (re q_f, im q_f, |q_f|)
+ *   weight <- decay * weight + nq
+ *   centres = sums[0..1] / weight,  mean_norm = sums[2] / weight
+ * so a query that arrived k calls ago carries weight decay^k (decay = 1: the
+ * plain mean of every query seen).  fp64 state and accumulation, fp32 outputs;
+ * deterministic.
+ *   qpre:      bf16 [n_layers][n_q_heads][nq][d] new pre-RoPE queries, 16-byte aligned
+ *   nq:        queries per head in this call, >= 1
+ *   decay:     0 < decay <= 1
+ *   sums:      device double [n_layers][n_q_heads][d/2][3], caller-owned state,
+ *              zeroed by the caller before the first call; updated in place
+ *   weight:    device double [n_layers][n_q_heads], same ownership
+ *   centres, mean_norm: outputs as for tri_calib
+ */
+tri_status tri_calib_update(const tri_model *m, const void *qpre, int64_t nq, double decay, double *sums,
+                            double *weight, float *centres, float *mean_norm, tri_stream_t stream);
+
+/*
+ * Concentration and drift diagnostics of n_heads sets of centre statistics
+ * (query heads from tri_calib / tri_calib_update, or cache rows from
+ * tri_key_centres).  The premise of the method is that pre-RoPE Q/K
+ * concentrate around their centres (digest, section 核心洞见); the digest flags
+ * the sensitivity to calibration/deployment shift as open (sections 不足,
+ * 复现注意事项).  Per head, in fp64:
+ *   concentration[f] = |centre_f| / mean_norm_f   (0 where mean_norm_f = 0)
+ *   head_stats[0]    = sum_f |centre_f| / sum_f mean_norm_f
+ *   head_stats[1]    = sum_f (|centre_f - ref_f| + |mean_norm_f - ref_norm_f|) / sum_f ref_norm_f
+ *                      (relative L1 drift; 0 when ref_centres is NULL)
+ *   centres, mean_norm:         float [n_heads][d/2][2] (8-byte aligned), [n_heads][d/2]
+ *   ref_centres, ref_mean_norm: the same shapes, or both NULL
+ *   concentration:              float [n_heads][d/2] or NULL
+ *   head_stats:                 float [n_heads][2] or NULL (not both NULL)
+ */
+tri_status tri_calib_stats(const tri_model *m, int64_t n_heads, const float *centres, const float *mean_norm,
+                           const float *ref_centres, const float *ref_mean_norm, float *concentration,
+                           float *head_stats, tri_stream_t stream);
+
+/*
+ * Pre-RoPE key centres of every cache row (digest, 流程详解 step 1 extracts the
+ * centres of Q and K): per row r and pair f,
+ *   centres[r][f]   = (1/N_r) sum_j k_f^pre(j)      (re, im)
+ *   mean_norm[r][f] = (1/N_r) sum_j |k_f(j)|
+ * (0 for an empty row).  key_mode TRI_KEYS_POST_ROPE: the cache holds RoPE'd
+ * keys and each is de-rotated by e^{-i w_f pos} (pos required; phase reduced
+ * exactly in 64-bit fixed-point turns); TRI_KEYS_PRE_ROPE: keys are used as
+ * stored (pos may be NULL).  fp64 accumulation in a fixed order.
+ *   kv, K, pos: the cache as for tri_score (bf16 or fp8, contiguous or paged)
+ *   centres:    float [R][d/2][2];  mean_norm: float [R][d/2]
+ *   ws:         tri_key_centres_ws_size bytes, 256-byte aligned; its first
+ *               word is a flag word (TRI_FLAG_ROW_OFFSETS, TRI_FLAG_BLOCK_TABLE)
+ *               read by tri_status_check
+ */
+size_t tri_key_centres_ws_size(const tri_model *m, int32_t n_seqs);
+tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void *K, const int32_t *pos,
+                           int32_t key_mode, float *centres, float *mean_norm, void *ws, size_t ws_bytes,
+                           tri_stream_t stream);
+
+/*
  * tri_score without a workspace argument, for callers that cannot allocate
  * device memory where they score: code running inside another framework's
  * memory pool that forbids foreign allocations, plugins whose host process

@@ -153,6 +153,44 @@ def tri_compact(m: TriModel, kv: TriKvDesc, scores: torch.Tensor, B: int, W: int
                           _s(stream)), "tri_compact")
 
 
+def tri_calib_update(m: TriModel, qpre: torch.Tensor, nq: int, decay: float, sums: torch.Tensor,
+                     weight: torch.Tensor, centres: torch.Tensor, mean_norm: torch.Tensor, stream=None) -> None:
+    """Fold a batch of pre-RoPE queries into the decayed running statistics (fp64
+    ``sums`` [L][Hq][d/2][3], ``weight`` [L][Hq]) and write the updated centres."""
+    _check(_L.tri_calib_update(ctypes.byref(m), _p(qpre), int(nq), float(decay), _p(sums), _p(weight), _p(centres),
+                               _p(mean_norm), _s(stream)), "tri_calib_update")
+
+
+def tri_calib_stats(m: TriModel, n_heads: int, centres: torch.Tensor, mean_norm: torch.Tensor,
+                    ref_centres=None, ref_mean_norm=None, concentration=None, head_stats=None,
+                    stream=None) -> None:
+    """Per-pair concentration and per-head (concentration, drift vs the reference)."""
+    _check(_L.tri_calib_stats(ctypes.byref(m), int(n_heads), _p(centres), _p(mean_norm), _p(ref_centres),
+                              _p(ref_mean_norm), _p(concentration), _p(head_stats), _s(stream)),
+           "tri_calib_stats")
+
+
+def tri_key_centres_ws_size(m: TriModel, n_seqs: int) -> int:
+    return int(_L.tri_key_centres_ws_size(ctypes.byref(m), int(n_seqs)))
+
+
+def tri_key_centres(m: TriModel, kv: TriKvDesc, K: torch.Tensor, pos, key_mode: int, centres: torch.Tensor,
+                    mean_norm: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    """Pre-RoPE key centre [R][d/2][2] and mean magnitude [R][d/2] of every cache row."""
+    _check(_L.tri_key_centres(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(pos), int(key_mode), _p(centres),
+                              _p(mean_norm), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "tri_key_centres")
+
+
+def alloc_key_centres_workspace(m: TriModel, n_seqs: int, device=None, stream=None) -> torch.Tensor:
+    n = tri_key_centres_ws_size(m, n_seqs)
+    if n == 0:
+        raise TriError(_abi.TRI_ERR_INVALID_ARG, "tri_key_centres_ws_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    tri_workspace_init(ws, stream)
+    return ws
+
+
 def tri_status_check(ws: torch.Tensor, stream=None):
     """Synchronise, read and clear the device flag word.  Returns (status, flags)."""
     flags = ctypes.c_uint32(0)

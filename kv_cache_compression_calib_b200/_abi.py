@@ -31,7 +31,8 @@ TRI_KEYS_PRE_ROPE = 1
 
 # Every symbol include/tri.h declares.
 EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_size", "tri_workspace_init", "tri_calib",
-           "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc")
+           "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc", "tri_calib_update",
+           "tri_calib_stats", "tri_key_centres_ws_size", "tri_key_centres")
 TRI_NOALLOC_MAX_ROWS = 4096
 
 
@@ -80,6 +81,16 @@ def load(path: str = LIB_PATH):
     L.tri_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
     L.tri_calib.restype = ctypes.c_int
     L.tri_calib.argtypes = [ctypes.POINTER(TriModel), _P, ctypes.c_int64, _P, _P, _P]
+    L.tri_calib_update.restype = ctypes.c_int
+    L.tri_calib_update.argtypes = [ctypes.POINTER(TriModel), _P, ctypes.c_int64, ctypes.c_double, _P, _P, _P, _P,
+                                   _P]
+    L.tri_calib_stats.restype = ctypes.c_int
+    L.tri_calib_stats.argtypes = [ctypes.POINTER(TriModel), ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P]
+    L.tri_key_centres_ws_size.restype = ctypes.c_size_t
+    L.tri_key_centres_ws_size.argtypes = [ctypes.POINTER(TriModel), ctypes.c_int32]
+    L.tri_key_centres.restype = ctypes.c_int
+    L.tri_key_centres.argtypes = [ctypes.POINTER(TriModel), ctypes.POINTER(TriKvDesc), _P, _P, ctypes.c_int32, _P,
+                                  _P, _P, ctypes.c_size_t, _P]
     L.tri_score.restype = ctypes.c_int
     L.tri_score.argtypes = [ctypes.POINTER(TriModel), ctypes.POINTER(TriKvDesc), _P, _P, _P, _P, _P,
                             ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, ctypes.c_int32, _P, _P,

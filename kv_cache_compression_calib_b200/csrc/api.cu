@@ -257,6 +257,86 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
     return cuda_status(launch_gather(gp, s), "gather_kernel launch");
 }
 
+tri_status tri_calib_update(const tri_model *m, const void *qpre, int64_t nq, double decay, double *sums,
+                            double *weight, float *centres, float *mean_norm, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    if (!qpre || !sums || !weight || !centres || !mean_norm || nq < 1) return TRI_ERR_INVALID_ARG;
+    if (!std::isfinite(decay) || !(decay > 0.0) || decay > 1.0) return TRI_ERR_INVALID_ARG;
+    if (!aligned(qpre, 16) || !aligned(sums, 8) || !aligned(weight, 8) || !aligned(centres, 4) ||
+        !aligned(mean_norm, 4))
+        return TRI_ERR_ALIGNMENT;
+    const int64_t heads = (int64_t)m->n_layers * m->n_q_heads;
+    if (heads > 0x7fffffffLL) return TRI_ERR_UNSUPPORTED;
+    CalibUpdateParams p;
+    p.c.D = m->head_dim;
+    p.c.il = m->rope_style == TRI_ROPE_INTERLEAVED;
+    p.c.q = (const uint16_t *)qpre;
+    p.c.nq = nq;
+    p.c.n_heads = (int32_t)heads;
+    p.c.centres = centres;
+    p.c.mean_norm = mean_norm;
+    p.decay = decay;
+    p.sums = sums;
+    p.weight = weight;
+    return cuda_status(launch_calib_update(p, (cudaStream_t)stream), "calib_update_kernel launch");
+}
+
+tri_status tri_calib_stats(const tri_model *m, int64_t n_heads, const float *centres, const float *mean_norm,
+                           const float *ref_centres, const float *ref_mean_norm, float *concentration,
+                           float *head_stats, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    if (n_heads < 1 || !centres || !mean_norm || (!concentration && !head_stats)) return TRI_ERR_INVALID_ARG;
+    if ((ref_centres == nullptr) != (ref_mean_norm == nullptr)) return TRI_ERR_INVALID_ARG;
+    if (!aligned(centres, 8) || !aligned(mean_norm, 4) || (ref_centres && !aligned(ref_centres, 8)) ||
+        (ref_mean_norm && !aligned(ref_mean_norm, 4)) || (concentration && !aligned(concentration, 4)) ||
+        (head_stats && !aligned(head_stats, 4)))
+        return TRI_ERR_ALIGNMENT;
+    StatsParams p;
+    p.F = m->head_dim / 2;
+    p.n_heads = n_heads;
+    p.centres = centres;
+    p.mean_norm = mean_norm;
+    p.ref_centres = ref_centres;
+    p.ref_mean_norm = ref_mean_norm;
+    p.concentration = concentration;
+    p.head_stats = head_stats;
+    return cuda_status(launch_stats(p, (cudaStream_t)stream), "stats_kernel launch");
+}
+
+size_t tri_key_centres_ws_size(const tri_model *m, int32_t n_seqs) {
+    if (check_model(m) != TRI_OK || n_seqs < 1) return 0;
+    const size_t R = (size_t)rows_of(m, n_seqs);
+    return 256 + ((R * kKeyCentreChunks * (size_t)(m->head_dim / 2) * 3 * sizeof(double) + 255) & ~size_t(255));
+}
+
+tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void *K, const int32_t *pos,
+                           int32_t key_mode, float *centres, float *mean_norm, void *ws, size_t ws_bytes,
+                           tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    Geometry geo;
+    if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
+    if (!K || !centres || !mean_norm) return TRI_ERR_INVALID_ARG;
+    if (key_mode != TRI_KEYS_POST_ROPE && key_mode != TRI_KEYS_PRE_ROPE) return TRI_ERR_INVALID_ARG;
+    if (key_mode == TRI_KEYS_POST_ROPE && !pos) return TRI_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(centres, 4) || !aligned(mean_norm, 4) || (pos && !aligned(pos, 4)))
+        return TRI_ERR_ALIGNMENT;
+    if ((st = check_ws(ws, ws_bytes, tri_key_centres_ws_size(m, kv->n_seqs))) != TRI_OK) return st;
+    KeyCentreParams p;
+    p.geo = geo;
+    p.K = (const char *)K;
+    p.pos = pos;
+    p.post_rope = key_mode == TRI_KEYS_POST_ROPE;
+    p.theta = m->rope_theta;
+    p.partial = (double *)((char *)ws + 256);
+    p.centres = centres;
+    p.mean_norm = mean_norm;
+    p.flags = (unsigned *)((char *)ws + kWsFlags);
+    return cuda_status(launch_key_centres(p, (cudaStream_t)stream), "key_centre_kernel launch");
+}
+
 tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream) {
     tri_status st = check_ws(ws, 256, 256);
     if (st != TRI_OK) return st;

@@ -34,12 +34,11 @@
 // 8), accumulates its 8 pairs in fp32, and a butterfly reduce-scatter over the
 // lanes of a key leaves one full score per lane; a shuffle orders them for one
 // coalesced store per batch (32 keys, 16 for d = 256).
-#include "tri_internal.cuh"
+#include "keys.cuh"
 
 namespace tri {
 
 constexpr int kScoreThreads = 256;
-constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
 
 struct RowCtx {
     int r;
@@ -88,101 +87,6 @@ __device__ __forceinline__ int64_t key_slot(const ScoreParams &p, const RowCtx &
     return ((((c.layer_blk + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) * geo.H) + c.h;
 }
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4 v, float (&x)[8]) {
-    x[0] = bf16lo(v.x); x[1] = bf16hi(v.x); x[2] = bf16lo(v.y); x[3] = bf16hi(v.y);
-    x[4] = bf16lo(v.z); x[5] = bf16hi(v.z); x[6] = bf16lo(v.w); x[7] = bf16hi(v.w);
-}
-
-// Two packed e4m3 values (low byte first) to floats: exact via f16.
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-    return __half22float2(__half2(h));
-}
-
-__device__ __forceinline__ void unpack_e4m3x8(const uint2 v, float (&x)[8]) {
-    const float2 a = e4m3x2_to_float2(v.x), b = e4m3x2_to_float2(v.x >> 16);
-    const float2 c = e4m3x2_to_float2(v.y), d = e4m3x2_to_float2(v.y >> 16);
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-    x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
-}
-
-__device__ __forceinline__ void unpack_bf16_pairs(const uint4 a, const uint4 b, float (&x)[8], float (&y)[8]) {
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        x[i] = bf16lo(w[i]);
-        y[i] = bf16hi(w[i]);
-    }
-}
-
-// Lane gl's share of one key record, as stored: the 8 pairs 8gl .. 8gl+7 of a
-// key with F = d/2 pairs.  Rotate-half (IL = false): real parts at dims
-// 8gl..8gl+7, imaginary parts F dims later - 2 x 16 bytes for bf16, 2 x 8 bytes
-// for fp8.  Interleaved (IL = true): dims 16gl..16gl+15, (re, im) adjacent -
-// 32 bytes for bf16, 16 for fp8.  Every load is naturally aligned: records are
-// 64..512 bytes long and start at multiples of their length from K.
-template <int ELEM, bool IL, int F>
-struct KeyChunk;
-
-template <int F>
-struct KeyChunk<2, false, F> {
-    uint4 re, im;
-    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
-        re = ld_stream16(key + 16 * gl, pol);
-        im = ld_stream16(key + 2 * F + 16 * gl, pol);
-    }
-    __device__ __forceinline__ void zero() { re = im = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
-        unpack_bf16x8(re, x);
-        unpack_bf16x8(im, y);
-    }
-};
-
-template <int F>
-struct KeyChunk<1, false, F> {
-    uint2 re, im;
-    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
-        re = ld_stream8(key + 8 * gl, pol);
-        im = ld_stream8(key + F + 8 * gl, pol);
-    }
-    __device__ __forceinline__ void zero() { re = im = make_uint2(0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
-        unpack_e4m3x8(re, x);
-        unpack_e4m3x8(im, y);
-    }
-};
-
-template <int F>
-struct KeyChunk<2, true, F> {
-    uint4 a, b;
-    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
-        a = ld_stream16(key + 32 * gl, pol);
-        b = ld_stream16(key + 32 * gl + 16, pol);
-    }
-    __device__ __forceinline__ void zero() { a = b = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const { unpack_bf16_pairs(a, b, x, y); }
-};
-
-template <int F>
-struct KeyChunk<1, true, F> {
-    uint4 v;
-    __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
-        v = ld_stream16(key + 16 * gl, pol);
-    }
-    __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const float2 p0 = e4m3x2_to_float2(w[i]), p1 = e4m3x2_to_float2(w[i] >> 16);
-            x[2 * i] = p0.x;
-            y[2 * i] = p0.y;
-            x[2 * i + 1] = p1.x;
-            y[2 * i + 1] = p1.y;
-        }
-    }
-};
-
 // Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|.
 __device__ __forceinline__ float partial_post(const float (&x)[8], const float (&y)[8], const RowCtx &c) {
     float a0 = 0.f, a1 = 0.f, a2 = 0.f;
@@ -197,14 +101,13 @@ __device__ __forceinline__ float partial_post(const float (&x)[8], const float (
 
 // Pre-RoPE cache: rotate A'_i by w_i (p_now - pos) first.  The phase in turns
 // is (delta * T_i) mod 2^64 with T_i = w_i / 2pi in 0.64 fixed point; its top
-// 32 bits as a signed integer are the angle in [-pi, pi).
+// 23 bits, read as signed, give the angle in [-pi, pi).
 __device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&y)[8], const RowCtx &c,
                                              const unsigned long long (&T)[8], int64_t delta) {
     float a0 = 0.f, a1 = 0.f, a2 = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-        const unsigned long long t = (unsigned long long)delta * T[i];
-        const float ang = (float)(int)(t >> 32) * kTurnToRad;
+        const float ang = turn_units23((unsigned long long)delta * T[i]) * kTurn23ToRad;
         float sn, cs;
         __sincosf(ang, &sn, &cs);
         const float br = c.ar[i] * cs - c.ai[i] * sn;
@@ -225,11 +128,13 @@ __device__ __forceinline__ float chunk_partial(const Chunk &kc, const RowCtx &c,
 }
 
 // Compile-time shape of one instantiation: LPK lanes per key (d / 16), NG keys
-// per warp instruction, U keys per lane per batch, KB keys per batch.
-template <int LPK>
+// per warp instruction, U keys per lane per batch, KB keys per batch.  The
+// pre-RoPE mode keeps 4 keys per lane in flight (its per-pair sin/cos needs the
+// registers; two CTAs per SM still keep enough bytes in flight).
+template <int LPK, bool PRE>
 struct Shape {
     static constexpr int NG = 32 / LPK;
-    static constexpr int U = LPK == 4 ? 4 : 8;
+    static constexpr int U = (LPK == 4 || PRE) ? 4 : 8;
     static constexpr int KB = NG * U;
     static constexpr int F = 8 * LPK;
 };
@@ -237,7 +142,7 @@ struct Shape {
 template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
 __device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx &c, int64_t k, int gl,
                                              unsigned long long pol, const unsigned long long (&T)[8]) {
-    constexpr int F = Shape<LPK>::F;
+    constexpr int F = Shape<LPK, PRE>::F;
     const int64_t slot = key_slot<PAGED>(p, c, k);
     if (slot < 0) {
         atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
@@ -250,8 +155,8 @@ __device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx 
 }
 
 template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
-__global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const ScoreParams p) {
-    using Sh = Shape<LPK>;
+__global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE) ? 3 : 2) score_kernel(const ScoreParams p) {
+    using Sh = Shape<LPK, PRE>;
     constexpr int NG = Sh::NG, U = Sh::U, KB = Sh::KB, F = Sh::F;
     constexpr int RB = 2 * F * ELEM;  // record bytes
     grid_dependency_wait();
@@ -344,8 +249,8 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
         // lane bit `half`, a lane keeps the upper or lower half of its partials
         // and adds its partner's copy of that half.  Afterwards lane (q, gl) holds
         // key NG * (gl % U) + q summed over the lanes that differ from it in the
-        // low log2(U) bits of gl; with LPK = 2U one more exchange adds the other
-        // half of the pairs.
+        // low log2(U) bits of gl; when LPK > U, plain exchanges over the remaining
+        // lane bits add the other lanes' pairs.
 #pragma unroll
         for (int half = U / 2; half >= 1; half >>= 1) {
             const bool up = (gl & half) != 0;
@@ -356,7 +261,8 @@ __global__ void __launch_bounds__(kScoreThreads, PRE ? 1 : 2) score_kernel(const
                 part[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
             }
         }
-        if (LPK > U) part[0] += __shfl_xor_sync(0xffffffffu, part[0], U);
+#pragma unroll
+        for (int o = U; o < LPK; o <<= 1) part[0] += __shfl_xor_sync(0xffffffffu, part[0], o);
         // Lane i < KB stores key b0 + i, held by lane (i % NG) * LPK + i / NG.
         const int src = lane < KB ? (lane % NG) * LPK + lane / NG : lane;
         const float v = __shfl_sync(0xffffffffu, part[0], src);
@@ -376,7 +282,7 @@ static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         if (o < 1) o = 1;
     }
-    constexpr int KB = Shape<LPK>::KB;
+    constexpr int KB = Shape<LPK, PRE>::KB;
     const int64_t want = (p.geo.total + KB * (kScoreThreads / 32) - 1) / (KB * (kScoreThreads / 32));
     int64_t grid = (int64_t)sm_count() * o;
     if (want < grid) grid = want;

@@ -98,7 +98,39 @@ struct CalibParams {
     float *centres, *mean_norm;
 };
 
+struct CalibUpdateParams {
+    CalibParams c;
+    double decay;
+    double *sums;    // [n_heads][F][3]: decayed sums of re, im, |q|
+    double *weight;  // [n_heads]: decayed query count
+};
+
+struct StatsParams {
+    int32_t F;
+    int64_t n_heads;
+    const float *centres, *mean_norm;          // [n][F][2], [n][F]
+    const float *ref_centres, *ref_mean_norm;  // same shapes, or null
+    float *concentration;                      // [n][F] or null
+    float *head_stats;                         // [n][2] or null
+};
+
+constexpr int kKeyCentreChunks = 16;  // CTAs per row of the key-centre pass
+
+struct KeyCentreParams {
+    Geometry geo;
+    const char *K;
+    const int32_t *pos;
+    int32_t post_rope;
+    double theta;
+    double *partial;  // [R][kKeyCentreChunks][F][3]
+    float *centres, *mean_norm;
+    unsigned *flags;
+};
+
 cudaError_t launch_calib(const CalibParams &p, cudaStream_t s);
+cudaError_t launch_calib_update(const CalibUpdateParams &p, cudaStream_t s);
+cudaError_t launch_stats(const StatsParams &p, cudaStream_t s);
+cudaError_t launch_key_centres(const KeyCentreParams &p, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams &p, cudaStream_t s);
 cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t s);
@@ -182,6 +214,17 @@ __device__ __forceinline__ void st_stream16(void *ptr, uint4 v) {
     asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
                  : "memory");
+}
+
+// A phase held as a 0.64 fixed-point fraction of a turn, as a float count of
+// 2^-23 turns in [-2^22, 2^22): the top 23 bits, re-centred by flipping their top
+// bit, placed in the mantissa of 2^23 (exact for any 23-bit integer) and the bias
+// 1.5 * 2^23 subtracted - integer and FP32-pipe operations only, no conversion
+// instruction.  Multiply by 2 pi / 2^23 for radians (step 7.5e-7 rad).
+constexpr float kTurn23ToRad = 7.490140565847157e-07f;  // 2 pi / 2^23
+__device__ __forceinline__ float turn_units23(unsigned long long t) {
+    const uint32_t u = (uint32_t)(t >> 41);
+    return __uint_as_float(0x4B000000u | (u ^ 0x400000u)) - 12582912.0f;
 }
 
 // Order-preserving map of fp32 scores to uint32: larger score -> larger key.

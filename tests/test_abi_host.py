@@ -143,6 +143,59 @@ def test_calib_rejects_bad_arguments():
     assert L.tri_calib(None, A, 8, A, A, None) == _abi.TRI_ERR_INVALID_ARG
 
 
+def test_calib_update_rejects_bad_arguments():
+    L = _abi.load()
+
+    def upd(q=A, nq=8, decay=0.9, sums=A, w=A, c=A, mn=A, m=M):
+        return L.tri_calib_update(ctypes.byref(m) if m is not None else None, q, nq, decay, sums, w, c, mn, None)
+
+    assert upd(q=None) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(nq=0) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(decay=0.0) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(decay=1.5) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(decay=float("nan")) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(sums=None) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(w=None) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(sums=A + 4) == _abi.TRI_ERR_ALIGNMENT
+    assert upd(q=A + 8) == _abi.TRI_ERR_ALIGNMENT
+    assert upd(m=None) == _abi.TRI_ERR_INVALID_ARG
+    assert upd(m=tri.model(1, 32, 8, 1e6, head_dim=80)) == _abi.TRI_ERR_UNSUPPORTED
+
+
+def test_calib_stats_rejects_bad_arguments():
+    L = _abi.load()
+
+    def st(n=32, c=A, mn=A, rc=None, rm=None, conc=A, hs=A):
+        return L.tri_calib_stats(ctypes.byref(M), n, c, mn, rc, rm, conc, hs, None)
+
+    assert st(n=0) == _abi.TRI_ERR_INVALID_ARG
+    assert st(c=None) == _abi.TRI_ERR_INVALID_ARG
+    assert st(conc=None, hs=None) == _abi.TRI_ERR_INVALID_ARG
+    assert st(rc=A) == _abi.TRI_ERR_INVALID_ARG  # reference centres without reference norms
+    assert st(c=A + 4) == _abi.TRI_ERR_ALIGNMENT
+    assert st(hs=A + 2) == _abi.TRI_ERR_ALIGNMENT
+
+
+def test_key_centres_rejects_bad_arguments():
+    L = _abi.load()
+    need = tri.tri_key_centres_ws_size(M, 1)
+    assert need >= 256 + 8 * 16 * 64 * 24 and need % 256 == 0
+    assert tri.tri_key_centres_ws_size(M, 0) == 0
+
+    def kc(kv=None, K=A, pos=A, mode=0, c=A, mn=A, ws=A, ws_bytes=1 << 30):
+        kv = kv or _kv()
+        return L.tri_key_centres(ctypes.byref(M), ctypes.byref(kv), K, pos, mode, c, mn, ws, ws_bytes, None)
+
+    assert kc(K=None) == _abi.TRI_ERR_INVALID_ARG
+    assert kc(pos=None) == _abi.TRI_ERR_INVALID_ARG  # a RoPE cache is de-rotated by position
+    assert kc(mode=7) == _abi.TRI_ERR_INVALID_ARG
+    assert kc(c=None) == _abi.TRI_ERR_INVALID_ARG
+    assert kc(K=A + 8) == _abi.TRI_ERR_ALIGNMENT
+    assert kc(ws_bytes=need - 1) == _abi.TRI_ERR_WORKSPACE_TOO_SMALL
+    assert kc(ws=A + 128) == _abi.TRI_ERR_ALIGNMENT
+    assert kc(kv=_kv(layout=1)) == _abi.TRI_ERR_INVALID_ARG
+
+
 def test_status_check_rejects_bad_workspace():
     L = _abi.load()
     assert L.tri_status_check(None, None, None) == _abi.TRI_ERR_INVALID_ARG
