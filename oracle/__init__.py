@@ -78,6 +78,9 @@ def _declare(L) -> None:
                                   ctypes.c_int, _f64p, _f64p]
     L.ora_calib_stats.restype = None
     L.ora_calib_stats.argtypes = [ctypes.c_int, _f64p, _f64p, ctypes.c_void_p, ctypes.c_void_p, _f64p, _f64p]
+    L.ora_attention.restype = None
+    L.ora_attention.argtypes = [ctypes.c_int, ctypes.c_int64, _f64p, _f64p, _f64p, ctypes.c_double, _f64p,
+                                ctypes.POINTER(ctypes.c_double)]
     L.ora_select.restype = ctypes.c_int64
     L.ora_select.argtypes = [ctypes.c_int64, _f64p, ctypes.c_int64, ctypes.c_int64, _i64p]
     L.ora_gather_bytes.restype = None
@@ -186,6 +189,17 @@ def calib_stats(centre: np.ndarray, mnorm: np.ndarray, ref_centre=None, ref_mnor
         lib().ora_calib_stats(F, centre, mnorm, rc.ctypes.data_as(ctypes.c_void_p),
                               rm.ctypes.data_as(ctypes.c_void_p), conc, head)
     return conc, (float(head[0]), float(head[1]))
+
+
+def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float):
+    """Softmax attention of one query [d] over keys/values [n][d]: (out [d], lse)."""
+    q = _f64(q)
+    keys = _f64(keys).reshape(-1, q.shape[0])
+    values = _f64(values).reshape(-1, q.shape[0])
+    out = np.empty(q.shape[0])
+    lse = ctypes.c_double(0.0)
+    lib().ora_attention(q.shape[0], keys.shape[0], q, keys, values, float(scale), out, ctypes.byref(lse))
+    return out, float(lse.value)
 
 
 def _score(fn, theta, qbar, mnorm, keys, pos, post_rope, p_now, offsets, interleaved=False):

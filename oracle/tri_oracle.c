@@ -481,3 +481,43 @@ void ora_calib_stats(int F, const double *centre, const double *mnorm, const dou
     head[0] = sm > 0.0L ? (double)(sc / sm) : 0.0;
     head[1] = (ref && rm > 0.0L) ? (double)(dd / rm) : 0.0;
 }
+
+/* ------------------------------------------------ attention over the cache */
+
+/*
+ * Decode attention of one query over one (compressed) cache row (digest,
+ * 流程详解 step 5: all later attention runs over the compressed cache):
+ *   s_j = scale * (q . k_j),   out = sum_j e^{s_j} v_j / sum_j e^{s_j},
+ *   lse = log sum_j e^{s_j}
+ * taken with the maximum subtracted first (softmax definition; long double).
+ * An empty row gives out = 0 and lse = -inf.
+ *   q: [d] (already RoPE'd at its position); keys, values: [n][d]; out: [d].
+ */
+void ora_attention(int d, int64_t n, const double *q, const double *keys, const double *values, double scale,
+                   double *out, double *lse)
+{
+    for (int t = 0; t < d; t++) out[t] = 0.0;
+    if (n == 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    ldbl *s = malloc(sizeof(ldbl) * (size_t)n);
+    ldbl m = -INFINITY;
+    for (int64_t j = 0; j < n; j++) {
+        ldbl a = 0.0L;
+        for (int t = 0; t < d; t++) a += (ldbl)q[t] * (ldbl)keys[j * d + t];
+        s[j] = (ldbl)scale * a;
+        if (s[j] > m) m = s[j];
+    }
+    ldbl den = 0.0L;
+    ldbl *acc = calloc((size_t)d, sizeof(ldbl));
+    for (int64_t j = 0; j < n; j++) {
+        ldbl p = expl(s[j] - m);
+        den += p;
+        for (int t = 0; t < d; t++) acc[t] += p * (ldbl)values[j * d + t];
+    }
+    for (int t = 0; t < d; t++) out[t] = (double)(acc[t] / den);
+    *lse = (double)(m + logl(den));
+    free(s);
+    free(acc);
+}

@@ -53,6 +53,10 @@ MUTATIONS = [
     ("concentration inverted",
      [("conc[f] = mnorm[f] > 0.0 ? (double)(a / (ldbl)mnorm[f]) : 0.0;",
        "conc[f] = a > 0.0L ? (double)((ldbl)mnorm[f] / a) : 0.0;")]),
+    ("attention scale dropped",
+     [("s[j] = (ldbl)scale * a;", "s[j] = a;")]),
+    ("attention normalised by the row length",
+     [("out[t] = (double)(acc[t] / den);", "out[t] = (double)(acc[t] / (ldbl)n);")]),
     ("tie-break keeps the older slot",
      [("if (a->i != b->i) return a->i > b->i ? -1 : 1;", "if (a->i != b->i) return a->i < b->i ? -1 : 1;")]),
     ("window not protected",
@@ -82,6 +86,7 @@ PIN_FUNCS = [
     lambda: pins.test_calib_online_equals_weighted_mean(),
     lambda: pins.test_key_centres_undo_rope(False),
     lambda: pins.test_calib_stats_closed_forms(),
+    lambda: pins.test_attention_matches_torch_sdpa_and_closed_forms(),
 ]
 
 

@@ -532,3 +532,44 @@ def test_calib_stats_closed_forms():
     # a zero-norm pair reports 0, not NaN
     conc, (hc, _) = oracle.calib_stats(np.zeros((2, 2)), np.zeros(2))
     assert np.all(conc == 0.0) and hc == 0.0
+
+
+# ------------------------------------------------------- decode attention
+
+def test_attention_matches_torch_sdpa_and_closed_forms():
+    import torch
+    rng = np.random.default_rng(61)
+    d = 64
+    for n in (1, 2, 7, 300):
+        q = rng.standard_normal(d)
+        k = rng.standard_normal((n, d)) * 0.7
+        v = rng.standard_normal((n, d))
+        scale = 1.0 / np.sqrt(d)
+        out, lse = oracle.attention(q, k, v, scale)
+        tq, tk, tv = (torch.from_numpy(x).to(torch.float64) for x in (q[None, None, None], k[None, None], v[None, None]))
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=scale)[0, 0, 0].numpy()
+        np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+        s = scale * (k @ q)
+        np.testing.assert_allclose(lse, np.log(np.sum(np.exp(s))), rtol=1e-13)
+    # q = 0: every weight equal -> mean of V, lse = log n
+    v = rng.standard_normal((5, d))
+    out, lse = oracle.attention(np.zeros(d), rng.standard_normal((5, d)), v, 1.0)
+    np.testing.assert_allclose(out, v.mean(axis=0), rtol=1e-14)
+    assert abs(lse - np.log(5.0)) < 1e-15
+    # two keys: out = sigmoid(s1 - s2) v1 + sigmoid(s2 - s1) v2
+    q = np.zeros(d)
+    q[0] = 1.0
+    k = np.zeros((2, d))
+    k[0, 0], k[1, 0] = 2.0, -1.0
+    v = rng.standard_normal((2, d))
+    out, lse = oracle.attention(q, k, v, 1.0)
+    w1 = 1.0 / (1.0 + np.exp(-3.0))
+    np.testing.assert_allclose(out, w1 * v[0] + (1 - w1) * v[1], rtol=1e-14)
+    assert abs(lse - np.log(np.exp(2.0) + np.exp(-1.0))) < 1e-14
+    # huge scores do not overflow (the maximum is subtracted first)
+    out, lse = oracle.attention(q, 1000.0 * k, v, 1.0)
+    np.testing.assert_allclose(out, v[0], rtol=1e-14)
+    assert abs(lse - 2000.0) < 1e-12
+    # empty row
+    out, lse = oracle.attention(q, np.zeros((0, d)), np.zeros((0, d)), 1.0)
+    assert np.all(out == 0) and lse == -np.inf
