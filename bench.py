@@ -331,6 +331,7 @@ def run_ours(a, rank, world, local_rank):
     value = throughput(keys_step, world, ms_step)
 
     diagnostics = time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream)
+    diagnostics.update(time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream))
 
     # ---- end to end through the public API: pinned host inputs, copies in the region
     e2e = None
@@ -401,6 +402,45 @@ def time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream, reps=5):
             "key_centres_gbs": kc_bytes / (kc_ms / 1e3) / 1e9,
             "key_centres_frac": kc_bytes / (kc_ms / 1e3) / 1e9 / peak, "peak_kind": kind,
             "calib_update_ms": up_ms, "calib_update_queries_per_head": 64}
+
+
+def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
+    """Decode attention (one query per query head) over the compacted [R][B] cache
+    the step wrote, timed with CUDA events; algorithmic bytes = K and V of every
+    kept key + queries + fp32 outputs.  Reported only when every row filled its
+    budget (the compacted rows are then end to end)."""
+    lens_rows = np.diff(cache.row_off_np)
+    if lens_rows.min() < B:
+        return {}
+    import math
+    D, L, Hq, S = wl.head_dim, wl.n_layers, wl.n_q_heads, len(cache.lens)
+    R = cache.n_rows
+    kvc = tri.kv_contig(S, torch.arange(R + 1, device=dev, dtype=torch.int64) * B, R * B, tri.elem_type_of(Ko))
+    q = synth.decode_queries(wl, 0, np.asarray(cache.lens), dev)[None].expand(L, -1, -1, -1).contiguous()
+    out = torch.empty(L, S, Hq, D, device=dev)
+    lse = torch.empty(L, S, Hq, device=dev)
+    ws = tri.alloc_attention_workspace(m, S, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    call = lambda: tri.tri_decode_attention(m, kvc, Ko, Vo, q, scale, out, lse, ws, stream)  # noqa: E731
+    call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st, flags = tri.tri_status_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} in decode attention")
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = float(R) * B * 2 * D * eb + q.numel() * 2 + out.numel() * 4 + lse.numel() * 4
+    peak, _ = measured_peak()
+    return {"decode_attention_ms": ms, "decode_attention_bytes": nbytes,
+            "decode_attention_gbs": nbytes / (ms / 1e3) / 1e9,
+            "decode_attention_frac": nbytes / (ms / 1e3) / 1e9 / peak,
+            "decode_attention_l2": "the compacted K+V (%.0f MB) fit in L2: timed warm" % (R * B * 2 * D * eb / 1e6)
+            if R * B * 2 * D * eb < 100e6 else "compacted K+V larger than L2"}
 
 
 def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream, world,

@@ -288,6 +288,33 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
                            tri_stream_t stream);
 
 /*
+ * Decode attention over a (compressed) cache (digest, 流程详解 step 5: every
+ * later attention step reads only the compressed cache; weights unchanged).
+ * For every layer l, sequence s and query head g (KV head h = g / G), over the
+ * keys k_j and values v_j of row (l, s, h):
+ *   s_j = softmax_scale * (q . k_j)
+ *   out = sum_j e^{s_j} v_j / sum_j e^{s_j},   lse = log sum_j e^{s_j}
+ * (out = 0 and lse = -inf for an empty row).  fp32 arithmetic: exact products
+ * of the stored elements, fp32 sums, online softmax in base 2.
+ *   kv, K, V:  the cache in either layout and element type; for the compacted
+ *              cache of tri_compact, row_off holds the kept counts' prefix sums
+ *              (contiguous [R][B] output with every row full: row_off[r] = r*B;
+ *              paged output: the fresh block table, row r holding min(N_r, B) keys)
+ *   q:         bf16 [n_layers][n_seqs][n_q_heads][d], RoPE'd at the position
+ *              being decoded (2-byte aligned)
+ *   softmax_scale: > 0 (usually 1/sqrt(d))
+ *   out:       float [n_layers][n_seqs][n_q_heads][d]
+ *   lse:       float [n_layers][n_seqs][n_q_heads] or NULL
+ *   ws:        tri_attention_ws_size bytes, 256-byte aligned; first word is a
+ *              flag word (TRI_FLAG_ROW_OFFSETS, TRI_FLAG_BLOCK_TABLE)
+ * G = n_q_heads / n_kv_heads must be <= 16 (else TRI_ERR_UNSUPPORTED).
+ */
+size_t tri_attention_ws_size(const tri_model *m, int32_t n_seqs);
+tri_status tri_decode_attention(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,
+                                const void *q, float softmax_scale, float *out, float *lse, void *ws,
+                                size_t ws_bytes, tri_stream_t stream);
+
+/*
  * tri_score without a workspace argument, for callers that cannot allocate
  * device memory where they score: code running inside another framework's
  * memory pool that forbids foreign allocations, plugins whose host process

@@ -191,6 +191,27 @@ def alloc_key_centres_workspace(m: TriModel, n_seqs: int, device=None, stream=No
     return ws
 
 
+def tri_attention_ws_size(m: TriModel, n_seqs: int) -> int:
+    return int(_L.tri_attention_ws_size(ctypes.byref(m), int(n_seqs)))
+
+
+def alloc_attention_workspace(m: TriModel, n_seqs: int, device=None, stream=None) -> torch.Tensor:
+    n = tri_attention_ws_size(m, n_seqs)
+    if n == 0:
+        raise TriError(_abi.TRI_ERR_INVALID_ARG, "tri_attention_ws_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    tri_workspace_init(ws, stream)
+    return ws
+
+
+def tri_decode_attention(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor,
+                         softmax_scale: float, out: torch.Tensor, lse, ws: torch.Tensor, stream=None) -> None:
+    """Softmax attention of one decode query per (layer, sequence, query head) over the cache rows."""
+    _check(_L.tri_decode_attention(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(V), _p(q), float(softmax_scale),
+                                   _p(out), _p(lse), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "tri_decode_attention")
+
+
 def tri_status_check(ws: torch.Tensor, stream=None):
     """Synchronise, read and clear the device flag word.  Returns (status, flags)."""
     flags = ctypes.c_uint32(0)

@@ -337,6 +337,39 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
     return cuda_status(launch_key_centres(p, (cudaStream_t)stream), "key_centre_kernel launch");
 }
 
+size_t tri_attention_ws_size(const tri_model *m, int32_t n_seqs) {
+    if (check_model(m) != TRI_OK || n_seqs < 1) return 0;
+    const size_t R = (size_t)rows_of(m, n_seqs);
+    const size_t G = (size_t)(m->n_q_heads / m->n_kv_heads);
+    return 256 + ((R * kAttnChunks * G * (size_t)(m->head_dim + 2) * sizeof(float) + 255) & ~size_t(255));
+}
+
+tri_status tri_decode_attention(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,
+                                const void *q, float softmax_scale, float *out, float *lse, void *ws,
+                                size_t ws_bytes, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    Geometry geo;
+    if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
+    if (geo.G > 16) return TRI_ERR_UNSUPPORTED;
+    if (!K || !V || !q || !out) return TRI_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f)) return TRI_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(q, 2) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+        return TRI_ERR_ALIGNMENT;
+    if ((st = check_ws(ws, ws_bytes, tri_attention_ws_size(m, kv->n_seqs))) != TRI_OK) return st;
+    AttnParams p;
+    p.geo = geo;
+    p.K = (const char *)K;
+    p.V = (const char *)V;
+    p.q = (const uint16_t *)q;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.part = (float *)((char *)ws + 256);
+    p.out = out;
+    p.lse = lse;
+    p.flags = (unsigned *)((char *)ws + kWsFlags);
+    return cuda_status(launch_attention(p, (cudaStream_t)stream), "attention kernel launch");
+}
+
 tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream) {
     tri_status st = check_ws(ws, 256, 256);
     if (st != TRI_OK) return st;

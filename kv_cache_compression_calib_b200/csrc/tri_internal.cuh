@@ -127,7 +127,21 @@ struct KeyCentreParams {
     unsigned *flags;
 };
 
+constexpr int kAttnChunks = 8;  // CTAs per cache row in decode attention
+
+struct AttnParams {
+    Geometry geo;        // the (compressed) cache: layout, head dim, element type
+    const char *K, *V;
+    const uint16_t *q;   // bf16 [L][S][Hq][D], RoPE'd at the decode position
+    float scale_log2;    // softmax scale * log2(e)
+    float *part;         // [R][kAttnChunks][G][D + 2]: unnormalised output, running max, running sum
+    float *out;          // [L][S][Hq][D]
+    float *lse;          // [L][S][Hq] or null
+    unsigned *flags;
+};
+
 cudaError_t launch_calib(const CalibParams &p, cudaStream_t s);
+cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_calib_update(const CalibUpdateParams &p, cudaStream_t s);
 cudaError_t launch_stats(const StatsParams &p, cudaStream_t s);
 cudaError_t launch_key_centres(const KeyCentreParams &p, cudaStream_t s);

@@ -292,3 +292,20 @@ FP8_MAX = 448.0  # largest finite OCP e4m3 value
 def to_fp8(t: torch.Tensor) -> torch.Tensor:
     """The cache as an fp8 e4m3 cache would store it: clamp to +-448, round to nearest."""
     return t.float().clamp_(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn)
+
+
+def decode_queries(wl: Workload, layer: int, p_now: np.ndarray, device, heads: LayerHeads = None) -> torch.Tensor:
+    """The next token's queries of every sequence: bf16 [S][Hq][d], drawn from the
+    layer's query centres like the calibration queries and RoPE-rotated at the
+    sequence's position p_now[s] (the position being decoded)."""
+    heads = heads if heads is not None else layer_heads(wl, layer, device)
+    g = _gen(device, wl.seed, wl.name, "decode_queries", layer)
+    S, Hq, F, d = len(p_now), wl.n_q_heads, wl.head_dim // 2, wl.head_dim
+    er = torch.randn(S, Hq, F, generator=g, device=device)
+    ei = torch.randn(S, Hq, F, generator=g, device=device)
+    qr = heads.q_re[None] + heads.q_scale[None] * er
+    qi = heads.q_im[None] + heads.q_scale[None] * ei
+    c, s = rotation(torch.as_tensor(np.asarray(p_now), device=device), wl.theta, d)  # [S][F]
+    c, s = c[:, None, :], s[:, None, :]
+    out = torch.empty(S, Hq, d, dtype=torch.bfloat16, device=device)
+    return place_pairs(out, qr * c - qi * s, qr * s + qi * c, wl.interleaved)

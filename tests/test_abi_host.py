@@ -196,6 +196,29 @@ def test_key_centres_rejects_bad_arguments():
     assert kc(kv=_kv(layout=1)) == _abi.TRI_ERR_INVALID_ARG
 
 
+def test_decode_attention_rejects_bad_arguments():
+    L = _abi.load()
+    need = tri.tri_attention_ws_size(M, 1)
+    assert need >= 256 + 8 * 8 * 4 * 130 * 4 and need % 256 == 0
+
+    def at(m=M, kv=None, K=A, V=2 * A, q=3 * A, scale=0.088, out=4 * A, lse=None, ws=5 * A, ws_bytes=1 << 30):
+        kv = kv or _kv()
+        return L.tri_decode_attention(ctypes.byref(m), ctypes.byref(kv), K, V, q, scale, out, lse, ws, ws_bytes,
+                                      None)
+
+    assert at(K=None) == _abi.TRI_ERR_INVALID_ARG
+    assert at(V=None) == _abi.TRI_ERR_INVALID_ARG
+    assert at(q=None) == _abi.TRI_ERR_INVALID_ARG
+    assert at(out=None) == _abi.TRI_ERR_INVALID_ARG
+    assert at(scale=0.0) == _abi.TRI_ERR_INVALID_ARG
+    assert at(scale=float("inf")) == _abi.TRI_ERR_INVALID_ARG
+    assert at(K=A + 8) == _abi.TRI_ERR_ALIGNMENT
+    assert at(q=3 * A + 1) == _abi.TRI_ERR_ALIGNMENT
+    assert at(lse=A + 2) == _abi.TRI_ERR_ALIGNMENT
+    assert at(ws_bytes=need - 1) == _abi.TRI_ERR_WORKSPACE_TOO_SMALL
+    assert at(m=tri.model(1, 64, 2, 1e6)) == _abi.TRI_ERR_UNSUPPORTED  # 32 query heads per KV head
+
+
 def test_status_check_rejects_bad_workspace():
     L = _abi.load()
     assert L.tri_status_check(None, None, None) == _abi.TRI_ERR_INVALID_ARG
