@@ -365,8 +365,28 @@ def run_ours(a, rank, world, local_rank):
     return line
 
 
+def graph_time(call, stream, reps):
+    """Mean device time of one `call(stream)` (its kernels captured once in a CUDA
+    graph and replayed `reps` times between CUDA events), so the host's launch
+    rate does not set the pace of short calls."""
+    call(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
 def time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream, reps=5):
-    """Off-step calls, timed with CUDA events (mean of `reps` after one warm-up):
+    """Off-step calls, timed by CUDA graph replay (mean of `reps` after one warm-up):
     the key-centre pass over the whole cache (reads every key once: d x elem bytes
     per key) and one online centre update with 64 new queries per head."""
     D, L, Hq = wl.head_dim, wl.n_layers, wl.n_q_heads
@@ -380,22 +400,12 @@ def time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream, reps=5):
     uc = torch.empty(L, Hq, D // 2, 2, device=dev)
     un = torch.empty(L, Hq, D // 2, device=dev)
 
-    def timed(fn):
-        fn()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / reps
-
-    kc_ms = timed(lambda: tri.tri_key_centres(m, kv, cache.K, cache.pos, key_mode, kc, kn, kws, stream))
+    kc_ms = graph_time(lambda s: tri.tri_key_centres(m, kv, cache.K, cache.pos, key_mode, kc, kn, kws, s), stream,
+                       reps)
     st, flags = tri.tri_status_check(kws, stream)
     if st != 0:
         raise RuntimeError(f"device flags {flags:#x} in the key-centre pass")
-    up_ms = timed(lambda: tri.tri_calib_update(m, q, 64, 0.99, sums, weight, uc, un, stream))
+    up_ms = graph_time(lambda s: tri.tri_calib_update(m, q, 64, 0.99, sums, weight, uc, un, s), stream, reps)
     peak, kind = measured_peak()
     kc_bytes = float(cache.total) * D * eb
     return {"key_centres_ms": kc_ms, "key_centres_bytes": kc_bytes,
@@ -406,7 +416,7 @@ def time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream, reps=5):
 
 def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
     """Decode attention (one query per query head) over the compacted [R][B] cache
-    the step wrote, timed with CUDA events; algorithmic bytes = K and V of every
+    the step wrote, timed by CUDA graph replay; algorithmic bytes = K and V of every
     kept key + queries + fp32 outputs.  Reported only when every row filled its
     budget (the compacted rows are then end to end)."""
     lens_rows = np.diff(cache.row_off_np)
@@ -421,19 +431,10 @@ def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
     lse = torch.empty(L, S, Hq, device=dev)
     ws = tri.alloc_attention_workspace(m, S, device=dev)
     scale = 1.0 / math.sqrt(D)
-    call = lambda: tri.tri_decode_attention(m, kvc, Ko, Vo, q, scale, out, lse, ws, stream)  # noqa: E731
-    call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    ms = graph_time(lambda s: tri.tri_decode_attention(m, kvc, Ko, Vo, q, scale, out, lse, ws, s), stream, reps)
     st, flags = tri.tri_status_check(ws, stream)
     if st != 0:
         raise RuntimeError(f"device flags {flags:#x} in decode attention")
-    ms = e0.elapsed_time(e1) / reps
     nbytes = float(R) * B * 2 * D * eb + q.numel() * 2 + out.numel() * 4 + lse.numel() * 4
     peak, _ = measured_peak()
     return {"decode_attention_ms": ms, "decode_attention_bytes": nbytes,

@@ -341,7 +341,7 @@ size_t tri_attention_ws_size(const tri_model *m, int32_t n_seqs) {
     if (check_model(m) != TRI_OK || n_seqs < 1) return 0;
     const size_t R = (size_t)rows_of(m, n_seqs);
     const size_t G = (size_t)(m->n_q_heads / m->n_kv_heads);
-    return 256 + ((R * kAttnChunks * G * (size_t)(m->head_dim + 2) * sizeof(float) + 255) & ~size_t(255));
+    return 256 + ((R * kAttnMaxChunks * G * (size_t)(m->head_dim + 2) * sizeof(float) + 255) & ~size_t(255));
 }
 
 tri_status tri_decode_attention(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,

@@ -127,14 +127,15 @@ struct KeyCentreParams {
     unsigned *flags;
 };
 
-constexpr int kAttnChunks = 8;  // CTAs per cache row in decode attention
+constexpr int kAttnMaxChunks = 32;  // most slices per cache row in decode attention
 
 struct AttnParams {
     Geometry geo;        // the (compressed) cache: layout, head dim, element type
     const char *K, *V;
     const uint16_t *q;   // bf16 [L][S][Hq][D], RoPE'd at the decode position
     float scale_log2;    // softmax scale * log2(e)
-    float *part;         // [R][kAttnChunks][G][D + 2]: unnormalised output, running max, running sum
+    int32_t chunks;      // CTAs per row (1 .. kAttnMaxChunks), set at launch
+    float *part;         // [R][chunks][G][D + 2]: unnormalised output, running max, running sum
     float *out;          // [L][S][Hq][D]
     float *lse;          // [L][S][Hq] or null
     unsigned *flags;
