@@ -70,6 +70,10 @@ def parse():
                     help="override the workload's RoPE pairing")
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="timed steps replay CUDA graphs of the calls (default) or call eagerly")
+    ap.add_argument("--path", choices=["split", "fused"], default="split",
+                    help="split: tri_score + tri_compact (the faster of the two on the 32K workload, by ~1%%); "
+                         "fused: one tri_score_compact call per step (rows up to TRI_FUSED_MAX_ROW keys, scores "
+                         "kept on chip, no score buffer)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -265,14 +269,25 @@ def run_ours(a, rank, world, local_rank):
     offsets = wl.offsets
 
     out_desc = tri.out_contig()
+    max_row = int(np.diff(cache.row_off_np).max())
+    fused = a.path == "fused"
 
-    def score_call():  # on the current stream (the capture stream while capturing)
-        tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode, scores, ws,
-                      torch.cuda.current_stream(dev))
+    if fused:
+        def score_call():  # the whole step: prep, fused score/select, gather
+            tri.tri_score_compact(m, kv, cache.K, cache.V, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode,
+                                  B, wl.window, max_row, out_desc, Ko, Vo, po, kept, None, None, ws,
+                                  torch.cuda.current_stream(dev))
 
-    def compact_call():
-        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, out_desc, Ko, Vo, po, kept, None,
-                        ws, torch.cuda.current_stream(dev))
+        def compact_call():
+            pass
+    else:
+        def score_call():  # on the current stream (the capture stream while capturing)
+            tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, offsets, key_mode, scores, ws,
+                          torch.cuda.current_stream(dev))
+
+        def compact_call():
+            tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, out_desc, Ko, Vo, po, kept,
+                            None, ws, torch.cuda.current_stream(dev))
 
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -337,10 +352,17 @@ def run_ours(a, rank, world, local_rank):
     e2e = None
     if not a.no_e2e:
         e2e = run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream,
-                      world, dev)
+                      world, dev, max_row if fused else None)
 
     peak, peak_kind = measured_peak()
-    score_bytes = score_bytes_per_key(eb, D) * total
+    if fused:  # one call per step: its roofline is the whole path's
+        score_bytes = alg_bytes
+        kernel = "tri_score_compact (prep + fused score/select + gather kernels)"
+        traffic = None
+    else:
+        score_bytes = score_bytes_per_key(eb, D) * total
+        kernel = "tri_score (prep + score kernels)"
+        traffic = recorded_traffic(total, a.elem) if (D, wl.rope_style) == (128, "half") else None
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     path_gbs = alg_bytes / (ms_step / 1e3) / 1e9
     line = {
@@ -349,14 +371,14 @@ def run_ours(a, rank, world, local_rank):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(wl, B, a.key_mode, "cuda_graph" if a.launch == "graph" else "eager", a.elem),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(total, a.elem) if (D, wl.rope_style) == (128, "half") else None,
-                     "kernel": "tri_score (prep + score kernels)", "peak_kind": peak_kind,
+                     "frac": achieved / peak, "traffic": traffic, "kernel": kernel, "peak_kind": peak_kind,
                      "bytes_per_launch": score_bytes, "ms_per_launch": score_ms},
         "path_roofline": {"bytes_per_step": alg_bytes, "achieved_gbs": path_gbs,
                           "frac_of_measured": path_gbs / peak, "frac_of_8tbs": path_gbs / NOMINAL_HBM_GBS},
         "calib_ms": calib_ms,
         "diagnostics": diagnostics,
-        "gpu_launches": 4 * a.steps,
+        "gpu_launches": (3 if fused else 4) * a.steps,
+        "path": "fused" if fused else "split",
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -445,7 +467,7 @@ def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
 
 
 def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream, world,
-            dev):
+            dev, fused_max_row=None):
     try:
         hK = cache.K.cpu().pin_memory()
         hV = cache.V.cpu().pin_memory()
@@ -470,10 +492,15 @@ def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, 
     def step():
         for d, h in ins:
             d.copy_(h, non_blocking=True)
-        tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, wl.offsets, key_mode, scores, ws,
-                      stream)
-        tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
-                        kept, None, ws, stream)
+        if fused_max_row is not None:
+            tri.tri_score_compact(m, kv, cache.K, cache.V, cache.pos, centres, mnorm, cache.p_now, wl.offsets,
+                                  key_mode, B, wl.window, fused_max_row, tri.out_contig(), Ko, Vo, po, kept, None,
+                                  None, ws, stream)
+        else:
+            tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, wl.offsets, key_mode, scores, ws,
+                          stream)
+            tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
+                            kept, None, ws, stream)
         for h, d in outs:
             h.copy_(d, non_blocking=True)
 

@@ -212,6 +212,19 @@ def tri_decode_attention(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.T
            "tri_decode_attention")
 
 
+def tri_score_compact(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.Tensor, pos, centres: torch.Tensor,
+                      mean_norm: torch.Tensor, p_now: torch.Tensor, offsets, key_mode: int, B: int, W: int,
+                      max_row_len: int, out: TriOutDesc, K_out: torch.Tensor, V_out: torch.Tensor, pos_out,
+                      kept_idx, kept_count, scores, ws: torch.Tensor, stream=None) -> None:
+    """tri_score + tri_compact in one call, fused on chip when max_row_len <= TRI_FUSED_MAX_ROW."""
+    offs = (ctypes.c_int32 * max(len(offsets), 1))(*[int(o) for o in offsets])
+    _check(_L.tri_score_compact(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(V), _p(pos), _p(centres),
+                                _p(mean_norm), _p(p_now), offs, len(offsets), int(key_mode), int(B), int(W),
+                                int(max_row_len), ctypes.byref(out), _p(K_out), _p(V_out), _p(pos_out),
+                                _p(kept_idx), _p(kept_count), _p(scores), _p(ws), ws.numel() * ws.element_size(),
+                                _s(stream)), "tri_score_compact")
+
+
 def tri_status_check(ws: torch.Tensor, stream=None):
     """Synchronise, read and clear the device flag word.  Returns (status, flags)."""
     flags = ctypes.c_uint32(0)

@@ -33,7 +33,8 @@ TRI_KEYS_PRE_ROPE = 1
 EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_size", "tri_workspace_init", "tri_calib",
            "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc", "tri_calib_update",
            "tri_calib_stats", "tri_key_centres_ws_size", "tri_key_centres", "tri_attention_ws_size",
-           "tri_decode_attention")
+           "tri_decode_attention", "tri_score_compact")
+TRI_FUSED_MAX_ROW = 32768
 TRI_NOALLOC_MAX_ROWS = 4096
 
 
@@ -87,6 +88,10 @@ def load(path: str = LIB_PATH):
                                    _P]
     L.tri_calib_stats.restype = ctypes.c_int
     L.tri_calib_stats.argtypes = [ctypes.POINTER(TriModel), ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P]
+    L.tri_score_compact.restype = ctypes.c_int
+    L.tri_score_compact.argtypes = [ctypes.POINTER(TriModel), ctypes.POINTER(TriKvDesc), _P, _P, _P, _P, _P, _P, _P,
+                                    ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                    ctypes.POINTER(TriOutDesc), _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     L.tri_attention_ws_size.restype = ctypes.c_size_t
     L.tri_attention_ws_size.argtypes = [ctypes.POINTER(TriModel), ctypes.c_int32]
     L.tri_decode_attention.restype = ctypes.c_int

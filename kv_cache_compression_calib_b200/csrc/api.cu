@@ -337,6 +337,110 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
     return cuda_status(launch_key_centres(p, (cudaStream_t)stream), "key_centre_kernel launch");
 }
 
+tri_status tri_score_compact(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,
+                             const int32_t *pos, const float *centres, const float *mean_norm, const int64_t *p_now,
+                             const int32_t *offsets, int32_t n_offsets, int32_t key_mode, int32_t B, int32_t W,
+                             int32_t max_row_len, const tri_out_desc *out, void *K_out, void *V_out,
+                             int32_t *pos_out, int32_t *kept_idx, int32_t *kept_count, float *scores, void *ws,
+                             size_t ws_bytes, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    Geometry geo;
+    if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
+    if (max_row_len < 0) return TRI_ERR_INVALID_ARG;
+    if (max_row_len > kFusedMaxRow) {
+        // Rows too long to hold on chip: the two-call path, through the caller's score buffer.
+        if (!scores) return TRI_ERR_INVALID_ARG;
+        if ((st = tri_score(m, kv, K, pos, centres, mean_norm, p_now, offsets, n_offsets, key_mode, scores, ws,
+                            ws_bytes, stream)) != TRI_OK)
+            return st;
+        return tri_compact(m, kv, scores, B, W, K, V, pos, out, K_out, V_out, pos_out, kept_idx, kept_count, ws,
+                           ws_bytes, stream);
+    }
+    // Checks of tri_score ...
+    if (!K || !centres || !mean_norm || !p_now || !offsets) return TRI_ERR_INVALID_ARG;
+    if (n_offsets < 1 || n_offsets > TRI_MAX_OFFSETS) return TRI_ERR_INVALID_ARG;
+    if (key_mode != TRI_KEYS_POST_ROPE && key_mode != TRI_KEYS_PRE_ROPE) return TRI_ERR_INVALID_ARG;
+    if (key_mode == TRI_KEYS_PRE_ROPE && !pos) return TRI_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || (scores && !aligned(scores, 4)) || !aligned(centres, 8) || !aligned(mean_norm, 4) ||
+        !aligned(p_now, 8) || (pos && !aligned(pos, 4)))
+        return TRI_ERR_ALIGNMENT;
+    // ... and of tri_compact.
+    if (B < 1 || W < 0 || W > B) return TRI_ERR_INVALID_ARG;
+    if (!V || !out || !K_out || !V_out) return TRI_ERR_INVALID_ARG;
+    if (pos_out && !pos) return TRI_ERR_INVALID_ARG;
+    if (K_out == K || V_out == V || K_out == V || V_out == K) return TRI_ERR_INVALID_ARG;
+    if (!aligned(V, 16) || !aligned(K_out, 16) || !aligned(V_out, 16) || (pos_out && !aligned(pos_out, 4)) ||
+        (kept_idx && !aligned(kept_idx, 4)) || (kept_count && !aligned(kept_count, 4)))
+        return TRI_ERR_ALIGNMENT;
+    int out_shift = 0;
+    if (out->layout == TRI_KV_PAGED) {
+        if (!out->block_table || out->max_blocks < 1 || out->n_blocks < 1) return TRI_ERR_INVALID_ARG;
+        if (!aligned(out->block_table, 4)) return TRI_ERR_ALIGNMENT;
+        out_shift = pow2_shift(out->block_size);
+        if (out_shift < 0) return TRI_ERR_UNSUPPORTED;
+    } else if (out->layout != TRI_KV_CONTIG) {
+        return TRI_ERR_INVALID_ARG;
+    }
+    const int64_t R = rows_of(m, kv->n_seqs);
+    if ((st = check_ws(ws, ws_bytes, kept_idx ? ws_idx_offset(R, m->head_dim) : ws_total(R, B, m->head_dim))) !=
+        TRI_OK)
+        return st;
+    char *w = (char *)ws;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t *kept = kept_idx ? kept_idx : (int32_t *)(w + ws_idx_offset(R, m->head_dim));
+
+    PrepParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.geo = geo;
+    pp.centres = centres;
+    pp.mean_norm = mean_norm;
+    pp.p_now = p_now;
+    pp.theta = m->rope_theta;
+    pp.n_off = n_offsets;
+    pp.pre_rope = key_mode == TRI_KEYS_PRE_ROPE;
+    for (int i = 0; i < n_offsets; i++) pp.offsets[i] = offsets[i];
+    pp.coef = (float *)(w + kWsCoef);
+    pp.turns = (unsigned long long *)(w + kWsTurns);
+    pp.flags = (unsigned *)(w + kWsFlags);
+    if ((st = cuda_status(launch_prep(pp, s), "prep_kernel launch")) != TRI_OK) return st;
+
+    FusedParams fp;
+    std::memset(&fp, 0, sizeof(fp));
+    fp.sp.geo = geo;
+    fp.sp.K = (const char *)K;
+    fp.sp.pos = pos;
+    fp.sp.p_now = p_now;
+    fp.sp.coef = pp.coef;
+    fp.sp.turns = pp.turns;
+    fp.sp.scores = scores;
+    fp.sp.flags = pp.flags;
+    fp.B = B;
+    fp.W = W;
+    fp.kept = kept;
+    fp.kept_count = kept_count;
+    if ((st = cuda_status(launch_fused(fp, pp.pre_rope, s), "fused_kernel launch")) != TRI_OK) return st;
+
+    GatherParams gp;
+    std::memset(&gp, 0, sizeof(gp));
+    gp.geo = geo;
+    gp.out_layout = out->layout;
+    gp.out_max_blocks = out->max_blocks;
+    gp.out_block_shift = out_shift;
+    gp.out_n_blocks = out->n_blocks;
+    gp.out_table = out->block_table;
+    gp.B = B;
+    gp.kept = kept;
+    gp.K = (const char *)K;
+    gp.V = (const char *)V;
+    gp.pos = pos_out ? pos : nullptr;
+    gp.K_out = (char *)K_out;
+    gp.V_out = (char *)V_out;
+    gp.pos_out = pos_out;
+    gp.flags = pp.flags;
+    return cuda_status(launch_gather(gp, s), "gather_kernel launch");
+}
+
 size_t tri_attention_ws_size(const tri_model *m, int32_t n_seqs) {
     if (check_model(m) != TRI_OK || n_seqs < 1) return 0;
     const size_t R = (size_t)rows_of(m, n_seqs);

@@ -1,0 +1,124 @@
+// Per-key scoring pieces shared by the streaming score kernel and the fused
+// score-and-select kernel: row context, record addressing, the per-lane partial
+// sums for post- and pre-RoPE caches, and the compile-time lane layout.
+#pragma once
+
+#include "keys.cuh"
+
+namespace tri {
+
+struct RowCtx {
+    int r;
+    int64_t lo, hi;
+    // paged addressing
+    const int32_t *table;
+    int64_t layer_blk;  // l * n_blocks
+    int h;
+    int64_t p_now;
+    float ar[8], ai[8], cc[8];
+};
+
+__device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, int gl, int coef_per_row) {
+    const Geometry &geo = p.geo;
+    c.r = r;
+    c.lo = geo.row_off[r];
+    c.hi = geo.row_off[r + 1];
+    const int h = r % geo.H;
+    const int s = (r / geo.H) % geo.S;
+    const int l = r / (geo.H * geo.S);
+    c.h = h;
+    c.table = geo.block_table + (int64_t)s * geo.max_blocks;
+    c.layer_blk = (int64_t)l * geo.n_blocks;
+    c.p_now = p.p_now[s];
+    const float4 *cp = reinterpret_cast<const float4 *>(p.coef + (int64_t)r * coef_per_row + gl * kCoefPerGroup);
+    const float4 v0 = cp[0], v1 = cp[1], v2 = cp[2], v3 = cp[3], v4 = cp[4], v5 = cp[5];
+    c.ar[0] = v0.x; c.ar[1] = v0.y; c.ar[2] = v0.z; c.ar[3] = v0.w;
+    c.ar[4] = v1.x; c.ar[5] = v1.y; c.ar[6] = v1.z; c.ar[7] = v1.w;
+    c.ai[0] = v2.x; c.ai[1] = v2.y; c.ai[2] = v2.z; c.ai[3] = v2.w;
+    c.ai[4] = v3.x; c.ai[5] = v3.y; c.ai[6] = v3.z; c.ai[7] = v3.w;
+    c.cc[0] = v4.x; c.cc[1] = v4.y; c.cc[2] = v4.z; c.cc[3] = v4.w;
+    c.cc[4] = v5.x; c.cc[5] = v5.y; c.cc[6] = v5.z; c.cc[7] = v5.w;
+}
+
+// Slot index (in units of one (slot, head) record) of global key k in row c,
+// or -1 if the paged table cannot place it.
+template <bool PAGED>
+__device__ __forceinline__ int64_t key_slot(const ScoreParams &p, const RowCtx &c, int64_t k) {
+    if (!PAGED) return k;
+    const Geometry &geo = p.geo;
+    const int64_t j = k - c.lo;
+    const int64_t bi = j >> geo.block_shift;
+    if (j < 0 || bi >= geo.max_blocks) return -1;
+    const int32_t blk = __ldg(c.table + bi);
+    if (blk < 0 || blk >= geo.n_blocks) return -1;
+    return ((((c.layer_blk + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) * geo.H) + c.h;
+}
+
+// Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|.
+__device__ __forceinline__ float partial_post(const float (&x)[8], const float (&y)[8], const RowCtx &c) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        a0 = fmaf(c.ar[i], x[i], a0);
+        a1 = fmaf(c.ai[i], y[i], a1);
+        a2 = fmaf(c.cc[i], sqrt_approx(fmaf(x[i], x[i], y[i] * y[i])), a2);
+    }
+    return (a0 + a1) + a2;
+}
+
+// Pre-RoPE cache: rotate A'_i by w_i (p_now - pos) first.  The phase in turns
+// is (delta * T_i) mod 2^64 with T_i = w_i / 2pi in 0.64 fixed point; its top
+// 23 bits, read as signed, give the angle in [-pi, pi).
+__device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&y)[8], const RowCtx &c,
+                                             const unsigned long long (&T)[8], int64_t delta) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const float ang = turn_units23((unsigned long long)delta * T[i]) * kTurn23ToRad;
+        float sn, cs;
+        __sincosf(ang, &sn, &cs);
+        const float br = c.ar[i] * cs - c.ai[i] * sn;
+        const float bi = c.ar[i] * sn + c.ai[i] * cs;
+        a0 = fmaf(br, x[i], a0);
+        a1 = fmaf(bi, y[i], a1);
+        a2 = fmaf(c.cc[i], sqrt_approx(fmaf(x[i], x[i], y[i] * y[i])), a2);
+    }
+    return (a0 + a1) + a2;
+}
+
+template <bool PRE, typename Chunk>
+__device__ __forceinline__ float chunk_partial(const Chunk &kc, const RowCtx &c, const unsigned long long (&T)[8],
+                                               int64_t delta) {
+    float x[8], y[8];
+    kc.unpack(x, y);
+    return PRE ? partial_pre(x, y, c, T, delta) : partial_post(x, y, c);
+}
+
+// Compile-time shape of one instantiation: LPK lanes per key (d / 16), NG keys
+// per warp instruction, U keys per lane per batch, KB keys per batch.  The
+// pre-RoPE mode keeps 4 keys per lane in flight (its per-pair sin/cos needs the
+// registers; two CTAs per SM still keep enough bytes in flight).
+template <int LPK, bool PRE>
+struct Shape {
+    static constexpr int NG = 32 / LPK;
+    static constexpr int U = (LPK == 4 || PRE) ? 4 : 8;
+    static constexpr int KB = NG * U;
+    static constexpr int F = 8 * LPK;
+};
+
+template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
+__device__ __forceinline__ float key_partial(const ScoreParams &p, const RowCtx &c, int64_t k, int gl,
+                                             unsigned long long pol, const unsigned long long (&T)[8]) {
+    constexpr int F = Shape<LPK, PRE>::F;
+    const int64_t slot = key_slot<PAGED>(p, c, k);
+    if (slot < 0) {
+        atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
+        return 0.f;
+    }
+    KeyChunk<ELEM, IL, F> kc;
+    kc.load(p.K + slot * (2 * F * ELEM), gl, pol);
+    const int64_t delta = PRE ? c.p_now - (int64_t)__ldg(p.pos + slot) : 0;
+    return chunk_partial<PRE>(kc, c, T, delta);
+}
+
+}  // namespace tri

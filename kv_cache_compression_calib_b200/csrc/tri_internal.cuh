@@ -141,7 +141,17 @@ struct AttnParams {
     unsigned *flags;
 };
 
+constexpr int kFusedMaxRow = TRI_FUSED_MAX_ROW;  // longest row the fused score-and-select kernel holds on chip
+
+struct FusedParams {
+    ScoreParams sp;       // cache, coefficients, scores (may be null: kept on chip only)
+    int32_t B, W;
+    int32_t *kept;        // [R][B]
+    int32_t *kept_count;  // [R] or null
+};
+
 cudaError_t launch_calib(const CalibParams &p, cudaStream_t s);
+cudaError_t launch_fused(const FusedParams &p, int pre_rope, cudaStream_t s);
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
 cudaError_t launch_calib_update(const CalibUpdateParams &p, cudaStream_t s);
 cudaError_t launch_stats(const StatsParams &p, cudaStream_t s);

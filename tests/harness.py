@@ -23,6 +23,11 @@ def raw_bits(t: torch.Tensor) -> np.ndarray:
     return bits16(t)
 
 
+def torch_bits(t: torch.Tensor) -> torch.Tensor:
+    """The stored bits of a bf16/fp8 tensor as an integer tensor (for exact comparison)."""
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t.view(torch.int16)
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a bf16 or fp8 e4m3 tensor's bits to float64 (host)."""
     if t.dtype == torch.float8_e4m3fn:

@@ -219,6 +219,25 @@ def test_decode_attention_rejects_bad_arguments():
     assert at(m=tri.model(1, 64, 2, 1e6)) == _abi.TRI_ERR_UNSUPPORTED  # 32 query heads per KV head
 
 
+def test_score_compact_rejects_bad_arguments():
+    L = _abi.load()
+
+    def sc(max_row=4096, scores=None, B=64, W=8, K=A, ws_bytes=1 << 30):
+        arr = (ctypes.c_int32 * 3)(1, 2, 4)
+        out = _abi.TriOutDesc(0, 0, None, 0, 0, 0)
+        return L.tri_score_compact(ctypes.byref(M), ctypes.byref(_kv()), K, 2 * A, None, A, A, A, arr, 3, 0, B, W,
+                                   max_row, ctypes.byref(out), 3 * A, 4 * A, None, None, None, scores, A, ws_bytes,
+                                   None)
+
+    assert sc(max_row=-1) == _abi.TRI_ERR_INVALID_ARG
+    assert sc(max_row=40000) == _abi.TRI_ERR_INVALID_ARG  # the unfused path needs a score buffer
+    assert sc(B=0) == _abi.TRI_ERR_INVALID_ARG
+    assert sc(W=65) == _abi.TRI_ERR_INVALID_ARG
+    assert sc(K=None) == _abi.TRI_ERR_INVALID_ARG
+    assert sc(K=A + 8) == _abi.TRI_ERR_ALIGNMENT
+    assert sc(ws_bytes=100) == _abi.TRI_ERR_WORKSPACE_TOO_SMALL
+
+
 def test_status_check_rejects_bad_workspace():
     L = _abi.load()
     assert L.tri_status_check(None, None, None) == _abi.TRI_ERR_INVALID_ARG
