@@ -106,7 +106,7 @@ def measured_peak():
 
 def score_kernel_sha():
     h = hashlib.sha256()
-    for f in ("score.cu", "keys.cuh", "tri_internal.cuh"):
+    for f in ("score.cu", "score_common.cuh", "keys.cuh", "tri_internal.cuh"):
         with open(os.path.join(ROOT, "kv_cache_compression_calib_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
