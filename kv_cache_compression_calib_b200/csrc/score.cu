@@ -41,7 +41,7 @@ namespace tri {
 constexpr int kScoreThreads = 256;
 
 template <bool PAGED, bool PRE, int ELEM, bool IL, int LPK>
-__global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE) ? 3 : 2) score_kernel(const ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE && !PAGED) ? 3 : 2) score_kernel(const ScoreParams p) {
     using Sh = Shape<LPK, PRE>;
     constexpr int NG = Sh::NG, U = Sh::U, KB = Sh::KB, F = Sh::F;
     constexpr int RB = 2 * F * ELEM;  // record bytes

@@ -55,35 +55,70 @@ __device__ __forceinline__ int64_t key_slot(const ScoreParams &p, const RowCtx &
 }
 
 // Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|.
+// Two fp32 lanes in one 64-bit register pair, for the packed fp32 instructions of
+// sm_100 (fma/mul .rn.f32x2: each lane rounds exactly as the scalar instruction).
+__device__ __forceinline__ unsigned long long f2(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 f2split(unsigned long long r) {
+    float2 v;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+    return v;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|, two pairs (i, i+1)
+// per packed instruction: the dot product and the squared norms in f32x2, one
+// square root per pair.
 __device__ __forceinline__ float partial_post(const float (&x)[8], const float (&y)[8], const RowCtx &c) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+    unsigned long long d = 0ull, e = 0ull;  // (even, odd) lanes of the dot product and the norm term
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        a0 = fmaf(c.ar[i], x[i], a0);
-        a1 = fmaf(c.ai[i], y[i], a1);
-        a2 = fmaf(c.cc[i], sqrt_approx(fmaf(x[i], x[i], y[i] * y[i])), a2);
+    for (int k = 0; k < 4; k++) {
+        const unsigned long long X = f2(x[2 * k], x[2 * k + 1]), Y = f2(y[2 * k], y[2 * k + 1]);
+        d = fma2(f2(c.ar[2 * k], c.ar[2 * k + 1]), X, d);
+        d = fma2(f2(c.ai[2 * k], c.ai[2 * k + 1]), Y, d);
+        const float2 q = f2split(fma2(X, X, mul2(Y, Y)));
+        e = fma2(f2(c.cc[2 * k], c.cc[2 * k + 1]), f2(sqrt_approx(q.x), sqrt_approx(q.y)), e);
     }
-    return (a0 + a1) + a2;
+    const float2 dd = f2split(d), ee = f2split(e);
+    return (dd.x + dd.y) + (ee.x + ee.y);
 }
 
 // Pre-RoPE cache: rotate A'_i by w_i (p_now - pos) first.  The phase in turns
 // is (delta * T_i) mod 2^64 with T_i = w_i / 2pi in 0.64 fixed point; its top
-// 23 bits, read as signed, give the angle in [-pi, pi).
+// 23 bits, read as signed, give the angle in [-pi, pi).  The rotation, the dot
+// product and the squared norms run two pairs per packed instruction.
 __device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&y)[8], const RowCtx &c,
                                              const unsigned long long (&T)[8], int64_t delta) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+    unsigned long long d = 0ull, e = 0ull;
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const float ang = turn_units23((unsigned long long)delta * T[i]) * kTurn23ToRad;
-        float sn, cs;
-        __sincosf(ang, &sn, &cs);
-        const float br = c.ar[i] * cs - c.ai[i] * sn;
-        const float bi = c.ar[i] * sn + c.ai[i] * cs;
-        a0 = fmaf(br, x[i], a0);
-        a1 = fmaf(bi, y[i], a1);
-        a2 = fmaf(c.cc[i], sqrt_approx(fmaf(x[i], x[i], y[i] * y[i])), a2);
+    for (int k = 0; k < 4; k++) {
+        float sn0, cs0, sn1, cs1;
+        __sincosf(turn_units23((unsigned long long)delta * T[2 * k]) * kTurn23ToRad, &sn0, &cs0);
+        __sincosf(turn_units23((unsigned long long)delta * T[2 * k + 1]) * kTurn23ToRad, &sn1, &cs1);
+        const unsigned long long AR = f2(c.ar[2 * k], c.ar[2 * k + 1]), AI = f2(c.ai[2 * k], c.ai[2 * k + 1]);
+        const unsigned long long CS = f2(cs0, cs1), SN = f2(sn0, sn1);
+        const unsigned long long BR = fma2(AR, CS, mul2(f2(-c.ai[2 * k], -c.ai[2 * k + 1]), SN));
+        const unsigned long long BI = fma2(AR, SN, mul2(AI, CS));
+        const unsigned long long X = f2(x[2 * k], x[2 * k + 1]), Y = f2(y[2 * k], y[2 * k + 1]);
+        d = fma2(BR, X, d);
+        d = fma2(BI, Y, d);
+        const float2 q = f2split(fma2(X, X, mul2(Y, Y)));
+        e = fma2(f2(c.cc[2 * k], c.cc[2 * k + 1]), f2(sqrt_approx(q.x), sqrt_approx(q.y)), e);
     }
-    return (a0 + a1) + a2;
+    const float2 dd = f2split(d), ee = f2split(e);
+    return (dd.x + dd.y) + (ee.x + ee.y);
 }
 
 template <bool PRE, typename Chunk>
