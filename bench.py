@@ -233,7 +233,7 @@ def run_ours(a, rank, world, local_rank):
     wl = rank_workload(wl0, rank, B)
     key_mode = tri.TRI_KEYS_PRE_ROPE if a.key_mode == "pre" else tri.TRI_KEYS_POST_ROPE
     if wl.layout != "contig":
-        raise SystemExit("bench.py times the contiguous workloads; the paged one is a parity case")
+        return run_paged(a, tri, wl, B, rank, world, dev)
     cache = synth.make_contig(wl, dev, rotate=(a.key_mode == "post"))
     eb = ELEM_BYTES[a.elem]
     if a.elem == "fp8":
@@ -384,6 +384,156 @@ def run_ours(a, rank, world, local_rank):
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, B, cache, a.cpu_seconds)
+    return line
+
+
+def run_paged(a, tri, wl, B, rank, world, dev):
+    """The paged serving workload: a step is round 0 (every sequence's prefill,
+    8K..32K keys per head in 16-token blocks, scored and compacted to B into a
+    fresh block table) plus `wl.rounds` re-score rounds (the retained B keys and
+    `wl.rescore_every` new decode tokens per head, scored and compacted into a
+    fresh table).  The rounds are replayed on one steady-state input of the
+    same shape as every later round (appending the decode tokens is the model's
+    own KV write and stays outside the timed region)."""
+    stream = torch.cuda.current_stream(dev)
+    fused = a.path == "fused"
+    S, Hh, bs, W, D = wl.batch, wl.n_kv_heads, wl.block_size, wl.window, wl.head_dim
+    lens = wl.seq_lengths()
+    pg = synth.make_paged(wl, dev, lens=lens)
+    eb = 2
+    if a.elem == "fp8":
+        pg.K, pg.V = synth.to_fp8(pg.K), synth.to_fp8(pg.V)
+        eb = 1
+    et = tri.elem_type_of(pg.K)
+    m = tri.model(1, wl.n_q_heads, Hh, wl.theta, head_dim=D,
+                  rope_style=tri.TRI_ROPE_INTERLEAVED if wl.interleaved else tri.TRI_ROPE_HALF)
+    qcal = synth.calib_queries(wl, 0, dev)[None].contiguous()
+    c = torch.empty(1, wl.n_q_heads, D // 2, 2, device=dev)
+    n = torch.empty(1, wl.n_q_heads, D // 2, device=dev)
+    tri.tri_calib(m, qcal, wl.n_calib, c, n)
+    new = wl.rescore_every
+    ob = (B + new + bs - 1) // bs
+    n_out = S * ob
+    rng = np.random.default_rng(5)
+    tables = [torch.as_tensor(rng.permutation(n_out).reshape(S, ob).astype(np.int32), device=dev) for _ in range(2)]
+    outs = [(torch.zeros(1, n_out, bs, Hh, D, dtype=pg.K.dtype, device=dev),
+             torch.zeros(1, n_out, bs, Hh, D, dtype=pg.K.dtype, device=dev),
+             torch.full((1, n_out, bs, Hh), -1, dtype=torch.int32, device=dev)) for _ in range(2)]
+    ws = tri.alloc_workspace(m, S, B, device=dev)
+    kept = torch.empty(S * Hh, B, dtype=torch.int32, device=dev)
+
+    def round_call(cur, p_now, K, V, P, table, nb, o):
+        row_off = torch.as_tensor(synth.paged_row_offsets(cur, Hh), device=dev)
+        total = int(synth.paged_row_offsets(cur, Hh)[-1])
+        kv = tri.kv_paged(S, row_off, total, table, bs, nb, et)
+        pn = torch.as_tensor(np.asarray(p_now), device=dev)
+        scores = torch.empty(total, device=dev)
+        Ko, Vo, Po = outs[o]
+        max_row = int(np.max(cur))
+        if fused:
+            def call(st):
+                tri.tri_score_compact(m, kv, K, V, P, c, n, pn, wl.offsets, tri.TRI_KEYS_POST_ROPE, B, W, max_row,
+                                      tri.out_paged(tables[o], bs, n_out), Ko, Vo, Po, kept, None, None, ws, st)
+        else:
+            def call(st):
+                tri.tri_score(m, kv, K, P, c, n, pn, wl.offsets, tri.TRI_KEYS_POST_ROPE, scores, ws, st)
+                tri.tri_compact(m, kv, scores, B, W, K, V, P, tri.out_paged(tables[o], bs, n_out), Ko, Vo, Po,
+                                kept, None, ws, st)
+        return call, total, (kv, pn, scores, row_off)
+
+    # round 0 on the prefill; then a steady-state input: its output plus `new` decode tokens
+    call0, keys0, keep0 = round_call(lens, lens, pg.K, pg.V, pg.pos, pg.block_table.to(dev), pg.K.shape[0], 0)
+    call0(stream)
+    torch.cuda.synchronize()
+    cur = np.minimum(lens, B)
+    Kn, Vn = synth.decode_keys(wl, 0, 0, lens, new, dev)
+    if a.elem == "fp8":
+        Kn, Vn = synth.to_fp8(Kn), synth.to_fp8(Vn)
+    tbl0 = tables[0].cpu().numpy()
+    K1, V1, P1 = outs[0]
+    for s_ in range(S):
+        j = np.arange(int(cur[s_]), int(cur[s_]) + new)
+        blk = torch.as_tensor(tbl0[s_, j // bs].astype(np.int64), device=dev)
+        slot = torch.as_tensor(j % bs, device=dev)
+        K1[0, blk, slot] = Kn[s_]
+        V1[0, blk, slot] = Vn[s_]
+        P1[0, blk, slot] = torch.arange(int(lens[s_]), int(lens[s_]) + new, device=dev, dtype=torch.int32)[:, None]
+    cur1 = cur + new
+    call1, keys1, keep1 = round_call(cur1, lens + new, K1, V1, P1, tables[0], n_out, 1)
+
+    graphs = []
+    for call in (call0, call1):
+        for _ in range(a.warmup):
+            call(stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(torch.cuda.current_stream())
+        graphs.append(g)
+    st, flags = tri.tri_status_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} after warm-up")
+    for _ in range(a.warmup):
+        graphs[0].replay()
+        for _ in range(wl.rounds):
+            graphs[1].replay()
+    sampler = ClockSampler(dev.index or 0)
+    sampler.start()
+    ev0 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t0.record(stream)
+    for i in range(a.steps):
+        ev0[i][0].record(stream)
+        graphs[0].replay()
+        ev0[i][1].record(stream)
+        for _ in range(wl.rounds):
+            graphs[1].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(wall0, wall1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    r0_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev0)
+    st, flags = tri.tri_status_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} in the timed region")
+    ms_step = ms / a.steps
+    keys_step = keys0 + wl.rounds * keys1
+    rows0 = np.repeat(lens, Hh)
+    rows1 = np.repeat(cur1, Hh)
+    kb = kept_bytes(eb, D)
+    bytes0 = float(np.sum(float(D) * eb * rows0 + np.minimum(rows0, B) * kb))
+    bytes1 = float(np.sum(float(D) * eb * rows1 + np.minimum(rows1, B) * kb))
+    alg_bytes = bytes0 + wl.rounds * bytes1
+    r1_ms = (ms_step - r0_ms) / wl.rounds
+    peak, peak_kind = measured_peak()
+    line = {
+        "metric": METRIC, "value": throughput(keys_step, world, ms_step), "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(wl, B, "post", "cuda_graph", a.elem), rounds=wl.rounds, new_tokens=new,
+                       keys_round0=int(keys0), keys_per_round=int(keys1)),
+        "roofline": {"bound": "hbm", "achieved": bytes0 / (r0_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": bytes0 / (r0_ms / 1e3) / 1e9 / peak, "traffic": None,
+                     "kernel": "round 0 (prep + fused score/select + gather kernels)" if fused else
+                     "round 0 (prep + score + select + gather kernels)", "peak_kind": peak_kind,
+                     "bytes_per_launch": bytes0, "ms_per_launch": r0_ms},
+        "path_roofline": {"bytes_per_step": alg_bytes, "achieved_gbs": alg_bytes / (ms_step / 1e3) / 1e9,
+                          "frac_of_measured": alg_bytes / (ms_step / 1e3) / 1e9 / peak,
+                          "frac_of_8tbs": alg_bytes / (ms_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
+                          "round0_ms": r0_ms, "round_ms": r1_ms,
+                          "round_frac_of_measured": bytes1 / (r1_ms / 1e3) / 1e9 / peak},
+        "gpu_launches": (3 if fused else 4) * (1 + wl.rounds) * a.steps,
+        "clocks": clocks,
+        "e2e": None,
+        "path": "fused" if fused else "split",
+    }
     return line
 
 
