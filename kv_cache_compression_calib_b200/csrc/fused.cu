@@ -96,14 +96,20 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
     unsigned long long T[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * gl + i] : 0ull;
+    float stc[8], sts[8];
+    if (PRE) phasors(T, -(int64_t)NG, stc, sts);
     const unsigned long long pol = policy_evict_first();
     RowCtx c;
     set_row(c, p, r, gl, LPK * kCoefPerGroup);
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     int nan = 0;
-    for (int64_t b0 = lo + (int64_t)warp * KB; b0 < hi; b0 += (int64_t)kFWarps * KB) {
+    // Batches on the same grid as the score kernel's (multiples of KB in the
+    // concatenated key space), so every key sees the same batch and the same
+    // per-lane arithmetic: bit-identical scores, pre-RoPE phasor chains included.
+    const int64_t grid0 = lo - lo % KB;
+    for (int64_t b0 = grid0 + (int64_t)warp * KB; b0 < hi; b0 += (int64_t)kFWarps * KB) {
         float part[U];
-        if (b0 + KB <= hi) {
+        if (b0 >= lo && b0 + KB <= hi) {
             KeyChunk<ELEM, IL, F> kc[U];
             int64_t slot[U];
             int32_t kpos[U];
@@ -118,20 +124,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
                     kpos[u] = 0;
                 }
             }
+            bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; u++) {
-                if (PAGED && slot[u] < 0) {
-                    atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
-                    part[u] = 0.f;
-                } else {
-                    part[u] = chunk_partial<PRE>(kc[u], c, T, c.p_now - (int64_t)kpos[u]);
-                }
+                ok[u] = !PAGED || slot[u] >= 0;
+                if (!ok[u]) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
             }
+            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, stc, sts, part);
         } else {
 #pragma unroll
             for (int u = 0; u < U; u++) {
                 const int64_t k = b0 + NG * u + q;
-                part[u] = k < hi ? key_partial<PAGED, PRE, ELEM, IL, LPK>(p, c, k, gl, pol, T) : 0.f;
+                part[u] = (k >= lo && k < hi) ? key_partial<PAGED, PRE, ELEM, IL, LPK>(p, c, k, gl, pol, T) : 0.f;
             }
         }
         // The score kernel's reduce-scatter, in the same order.
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
         for (int o = U; o < LPK; o <<= 1) part[0] += __shfl_xor_sync(0xffffffffu, part[0], o);
         const int src = lane < KB ? (lane % NG) * LPK + lane / NG : lane;
         const float v = __shfl_sync(0xffffffffu, part[0], src);
-        if (lane < KB && b0 + lane < hi) {
+        if (lane < KB && b0 + lane >= lo && b0 + lane < hi) {
             const int j = (int)(b0 + lane - lo);
             const uint32_t u = order_key(v);
             keys[j] = u;

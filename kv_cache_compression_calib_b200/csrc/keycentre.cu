@@ -15,7 +15,7 @@
 // chunks' partials in chunk order and divides.  Both passes sum in a fixed order,
 // so results are deterministic.  It reads every key once: an HBM-bound pass like
 // the scoring one (plus one sin/cos per (key, pair) for a RoPE cache).
-#include "keys.cuh"
+#include "score_common.cuh"
 
 namespace tri {
 
@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
     for (int i = 0; i < 8; i++)
         T[i] = POST ? __double2ull_rn(pow(p.theta, -2.0 * (double)(8 * gl + i) / (double)(2 * F)) * kKcTurnScale)
                     : 0ull;
+    float stc[8], sts[8];  // e^{+i w NG}: from one key's rotation to the next one's in a batch
+    if (POST) phasors(T, (int64_t)NG, stc, sts);
     const unsigned long long pol = policy_evict_first();
     const int32_t *table = geo.block_table + (int64_t)s * geo.max_blocks;
     const int64_t layer_blk = (int64_t)l * geo.n_blocks;
@@ -97,8 +99,16 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
                 kc[u].zero();
             }
         }
+        // Rotation phasors e^{i w pos} of the lane's keys: the first from its reduced
+        // phase, each next one by one complex step when positions advance by NG.
+        float cs[8], sn[8];
+        if (POST) phasors(T, (int64_t)kpos[0], cs, sn);
 #pragma unroll
         for (int u = 0; u < U; u++) {
+            if (POST && u > 0) {
+                if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
+                else phasors(T, (int64_t)kpos[u], cs, sn);
+            }
             if (slot[u] < 0) continue;
             float x[8], y[8];
             kc[u].unpack(x, y);
@@ -106,11 +116,8 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
             for (int i = 0; i < 8; i++) {
                 float xr = x[i], xi = y[i];
                 if (POST) {
-                    float sn_, cs_;
-                    __sincosf(turn_units23((unsigned long long)(long long)kpos[u] * T[i]) * kTurn23ToRad, &sn_,
-                              &cs_);
-                    xr = x[i] * cs_ + y[i] * sn_;
-                    xi = y[i] * cs_ - x[i] * sn_;
+                    xr = x[i] * cs[i] + y[i] * sn[i];
+                    xi = y[i] * cs[i] - x[i] * sn[i];
                 }
                 fr[i] += xr;
                 fi[i] += xi;

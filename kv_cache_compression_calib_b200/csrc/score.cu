@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE && !PAGED) ?
     unsigned long long T[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * gl + i] : 0ull;
+    float stc[8], sts[8];  // e^{-i w NG}: from one key's rotation to the next one's in a batch
+    if (PRE) phasors(T, -(int64_t)NG, stc, sts);
     const unsigned long long pol = policy_evict_first();
 
     // Row holding key `beg`: the last r with row_off[r] <= beg.
@@ -81,6 +83,11 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE && !PAGED) ?
 
     for (int64_t b0 = beg; b0 < end; b0 += KB) {
         const int64_t bend = min(b0 + KB, end);
+        if (b0 >= c.hi && c.r < R - 1) {  // the batch starts in a later row: move there first
+            int r = c.r + 1;
+            while (r < R - 1 && geo.row_off[r + 1] <= b0) r++;
+            set_row(c, p, r, gl, cpr);
+        }
         float part[U];
         if (bend == b0 + KB && b0 >= c.lo && bend <= c.hi) {
             // Whole batch inside the current row: issue all loads, then compute.
@@ -98,15 +105,13 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE && !PAGED) ?
                     kpos[u] = 0;
                 }
             }
+            bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; u++) {
-                if (PAGED && slot[u] < 0) {
-                    atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
-                    part[u] = 0.f;
-                } else {
-                    part[u] = chunk_partial<PRE>(kc[u], c, T, c.p_now - (int64_t)kpos[u]);
-                }
+                ok[u] = !PAGED || slot[u] >= 0;
+                if (!ok[u]) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
             }
+            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, stc, sts, part);
         } else {
             // Batch crosses a row boundary or the span end: one segment per row.
 #pragma unroll

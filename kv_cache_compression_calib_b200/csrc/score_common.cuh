@@ -97,18 +97,40 @@ __device__ __forceinline__ float partial_post(const float (&x)[8], const float (
 
 // Pre-RoPE cache: rotate A'_i by w_i (p_now - pos) first.  The phase in turns
 // is (delta * T_i) mod 2^64 with T_i = w_i / 2pi in 0.64 fixed point; its top
-// 23 bits, read as signed, give the angle in [-pi, pi).  The rotation, the dot
-// product and the squared norms run two pairs per packed instruction.
-__device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&y)[8], const RowCtx &c,
-                                             const unsigned long long (&T)[8], int64_t delta) {
+// 23 bits, read as signed, give the angle in [-pi, pi).
+__device__ __forceinline__ void phasors(const unsigned long long (&T)[8], int64_t delta, float (&cs)[8],
+                                        float (&sn)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        __sincosf(turn_units23((unsigned long long)delta * T[i]) * kTurn23ToRad, &sn[i], &cs[i]);
+}
+
+// (cs, sn) <- (cs, sn) * (stc, sts) for the 8 pairs: the phasors of a key NG
+// slots further on, from those of this one (consecutive positions).
+__device__ __forceinline__ void advance_phasors(float (&cs)[8], float (&sn)[8], const float (&stc)[8],
+                                                const float (&sts)[8]) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const unsigned long long C = f2(cs[2 * k], cs[2 * k + 1]), S = f2(sn[2 * k], sn[2 * k + 1]);
+        const unsigned long long TC = f2(stc[2 * k], stc[2 * k + 1]), TS = f2(sts[2 * k], sts[2 * k + 1]);
+        const float2 nc = f2split(fma2(C, TC, mul2(f2(-sn[2 * k], -sn[2 * k + 1]), TS)));
+        const float2 ns = f2split(fma2(C, TS, mul2(S, TC)));
+        cs[2 * k] = nc.x;
+        cs[2 * k + 1] = nc.y;
+        sn[2 * k] = ns.x;
+        sn[2 * k + 1] = ns.y;
+    }
+}
+
+// Partial score of a pre-RoPE key given its rotation phasors e^{i w_i delta}: the
+// rotation, the dot product and the squared norms two pairs per packed instruction.
+__device__ __forceinline__ float partial_pre_rot(const float (&x)[8], const float (&y)[8], const RowCtx &c,
+                                                 const float (&cs)[8], const float (&sn)[8]) {
     unsigned long long d = 0ull, e = 0ull;
 #pragma unroll
     for (int k = 0; k < 4; k++) {
-        float sn0, cs0, sn1, cs1;
-        __sincosf(turn_units23((unsigned long long)delta * T[2 * k]) * kTurn23ToRad, &sn0, &cs0);
-        __sincosf(turn_units23((unsigned long long)delta * T[2 * k + 1]) * kTurn23ToRad, &sn1, &cs1);
         const unsigned long long AR = f2(c.ar[2 * k], c.ar[2 * k + 1]), AI = f2(c.ai[2 * k], c.ai[2 * k + 1]);
-        const unsigned long long CS = f2(cs0, cs1), SN = f2(sn0, sn1);
+        const unsigned long long CS = f2(cs[2 * k], cs[2 * k + 1]), SN = f2(sn[2 * k], sn[2 * k + 1]);
         const unsigned long long BR = fma2(AR, CS, mul2(f2(-c.ai[2 * k], -c.ai[2 * k + 1]), SN));
         const unsigned long long BI = fma2(AR, SN, mul2(AI, CS));
         const unsigned long long X = f2(x[2 * k], x[2 * k + 1]), Y = f2(y[2 * k], y[2 * k + 1]);
@@ -119,6 +141,44 @@ __device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&
     }
     const float2 dd = f2split(d), ee = f2split(e);
     return (dd.x + dd.y) + (ee.x + ee.y);
+}
+
+__device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&y)[8], const RowCtx &c,
+                                             const unsigned long long (&T)[8], int64_t delta) {
+    float cs[8], sn[8];
+    phasors(T, delta, cs, sn);
+    return partial_pre_rot(x, y, c, cs, sn);
+}
+
+// Partials of one lane's U keys of a whole batch (keys NG slots apart).  Pre-RoPE:
+// the first key's phasors from the reduced phase, each next key's by one complex
+// step (stc, sts) = e^{-i w NG} when the positions advance by NG (any gap: the
+// key's own reduced phase).  Invalid (unplaceable) keys give 0.
+template <bool PRE, int U, int NG, typename Chunk>
+__device__ __forceinline__ void batch_partials(const Chunk (&kc)[U], const int32_t (&kpos)[U], const bool (&ok)[U],
+                                               const RowCtx &c, const unsigned long long (&T)[8],
+                                               const float (&stc)[8], const float (&sts)[8], float (&part)[U]) {
+    if (!PRE) {
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            float x[8], y[8];
+            kc[u].unpack(x, y);
+            part[u] = ok[u] ? partial_post(x, y, c) : 0.f;
+        }
+        return;
+    }
+    float cs[8], sn[8];
+    phasors(T, c.p_now - (int64_t)kpos[0], cs, sn);
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+        if (u > 0) {
+            if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
+            else phasors(T, c.p_now - (int64_t)kpos[u], cs, sn);
+        }
+        float x[8], y[8];
+        kc[u].unpack(x, y);
+        part[u] = ok[u] ? partial_pre_rot(x, y, c, cs, sn) : 0.f;
+    }
 }
 
 template <bool PRE, typename Chunk>
