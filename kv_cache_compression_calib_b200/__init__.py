@@ -40,7 +40,16 @@ def _check(st: int, what: str) -> None:
 
 
 def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor argument (None -> NULL).  Every tensor the library
+    reads or writes must be a contiguous CUDA tensor: a host pointer handed to a
+    kernel would fault, a strided view would be read as if it were dense."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor (call .contiguous())")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _s(stream):
@@ -80,7 +89,7 @@ def elem_type_of(t: torch.Tensor) -> int:
 def kv_contig(n_seqs: int, row_off: torch.Tensor, total_keys: int,
               elem_type: int = TRI_ELEM_BF16) -> TriKvDesc:
     """Rows laid end to end; ``row_off`` int64 [R+1] on the device."""
-    d = TriKvDesc(TRI_KV_CONTIG, n_seqs, int(total_keys), row_off.data_ptr(), None, 0, 0, 0,
+    d = TriKvDesc(TRI_KV_CONTIG, n_seqs, int(total_keys), _p(row_off).value, None, 0, 0, 0,
                   int(elem_type), 0)
     d._keep = (row_off,)
     return d
@@ -89,8 +98,8 @@ def kv_contig(n_seqs: int, row_off: torch.Tensor, total_keys: int,
 def kv_paged(n_seqs: int, row_off: torch.Tensor, total_keys: int, block_table: torch.Tensor,
              block_size: int, n_blocks: int, elem_type: int = TRI_ELEM_BF16) -> TriKvDesc:
     """vLLM block layout; ``block_table`` int32 [S][max_blocks] on the device."""
-    d = TriKvDesc(TRI_KV_PAGED, n_seqs, int(total_keys), row_off.data_ptr(),
-                  block_table.data_ptr(), block_table.shape[1], block_size, int(n_blocks),
+    d = TriKvDesc(TRI_KV_PAGED, n_seqs, int(total_keys), _p(row_off).value,
+                  _p(block_table).value, block_table.shape[1], block_size, int(n_blocks),
                   int(elem_type), 0)
     d._keep = (row_off, block_table)
     return d
@@ -101,7 +110,7 @@ def out_contig() -> TriOutDesc:
 
 
 def out_paged(block_table: torch.Tensor, block_size: int, n_blocks: int) -> TriOutDesc:
-    d = TriOutDesc(TRI_KV_PAGED, block_table.shape[1], block_table.data_ptr(), block_size, 0,
+    d = TriOutDesc(TRI_KV_PAGED, block_table.shape[1], _p(block_table).value, block_size, 0,
                    int(n_blocks))
     d._keep = (block_table,)
     return d

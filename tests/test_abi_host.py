@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import kv_cache_compression_calib_b200 as tri
 from kv_cache_compression_calib_b200 import _abi
@@ -242,3 +243,13 @@ def test_status_check_rejects_bad_workspace():
     L = _abi.load()
     assert L.tri_status_check(None, None, None) == _abi.TRI_ERR_INVALID_ARG
     assert L.tri_status_check(A + 16, None, None) == _abi.TRI_ERR_ALIGNMENT
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """A host pointer or a strided view must never reach a kernel."""
+    m = tri.model(1, 32, 8, 1e6)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tri.tri_calib(m, torch.zeros(1, 32, 8, 128, dtype=torch.bfloat16), 8, torch.zeros(1, 32, 64, 2),
+                      torch.zeros(1, 32, 64))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tri.kv_contig(1, torch.zeros(9, dtype=torch.int64), 0)
