@@ -432,8 +432,10 @@ def run_paged(a, tri, wl, B, rank, world, dev):
         max_row = int(np.max(cur))
         if fused:
             def call(st):
+                # with a score buffer the library fuses the short rounds and runs round 0's
+                # long prefills through the two-call path
                 tri.tri_score_compact(m, kv, K, V, P, c, n, pn, wl.offsets, tri.TRI_KEYS_POST_ROPE, B, W, max_row,
-                                      tri.out_paged(tables[o], bs, n_out), Ko, Vo, Po, kept, None, None, ws, st)
+                                      tri.out_paged(tables[o], bs, n_out), Ko, Vo, Po, kept, None, scores, ws, st)
         else:
             def call(st):
                 tri.tri_score(m, kv, K, P, c, n, pn, wl.offsets, tri.TRI_KEYS_POST_ROPE, scores, ws, st)

@@ -289,20 +289,23 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
 
 /*
  * tri_score followed by tri_compact in one call (digest, 流程详解 steps 2-4),
- * with the scoring and the selection fused when every row fits on chip:
- *   max_row_len <= TRI_FUSED_MAX_ROW: one CTA per row keeps the row's scores
- *     in shared memory, selects from there and writes the kept slots; K, V and
- *     pos are then gathered.  The scores are bit-identical to tri_score's, so
- *     the kept sets and outputs are those of tri_score + tri_compact.  `scores`
- *     may be NULL (they are then never written to memory); a row longer than
+ * with the scoring and the selection fused on chip where that pays:
+ *   fused (max_row_len <= TRI_FUSED_PREFER_ROW, or `scores` NULL and
+ *     max_row_len <= TRI_FUSED_MAX_ROW): one CTA per row keeps the row's
+ *     scores in shared memory, selects from there and writes the kept slots;
+ *     K, V and pos are then gathered.  `scores`, when given, receives the
+ *     scores; when NULL they never leave the chip.  A row longer than
  *     max_row_len sets TRI_FLAG_ROW_OFFSETS and keeps nothing.
- *   max_row_len >  TRI_FUSED_MAX_ROW: exactly tri_score then tri_compact,
- *     `scores` (float [total_keys]) required.
+ *   otherwise: exactly tri_score then tri_compact, `scores` (float
+ *     [total_keys]) required.
+ * Both ways give the same results bit for bit (the fused kernel runs the
+ * score kernel's arithmetic in the same order), so the choice is only speed.
  * Arguments as for tri_score and tri_compact; max_row_len is the caller's
  * bound on the longest row (for the compacted rounds of a serving loop,
  * min(N, B) + the new tokens).  Same workspace as tri_compact.
  */
 #define TRI_FUSED_MAX_ROW 32768
+#define TRI_FUSED_PREFER_ROW 8192
 tri_status tri_score_compact(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,
                              const int32_t *pos, const float *centres, const float *mean_norm, const int64_t *p_now,
                              const int32_t *offsets, int32_t n_offsets, int32_t key_mode, int32_t B, int32_t W,

@@ -35,6 +35,7 @@ EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_siz
            "tri_calib_stats", "tri_key_centres_ws_size", "tri_key_centres", "tri_attention_ws_size",
            "tri_decode_attention", "tri_score_compact")
 TRI_FUSED_MAX_ROW = 32768
+TRI_FUSED_PREFER_ROW = 8192
 TRI_NOALLOC_MAX_ROWS = 4096
 
 

@@ -348,8 +348,11 @@ tri_status tri_score_compact(const tri_model *m, const tri_kv_desc *kv, const vo
     Geometry geo;
     if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
     if (max_row_len < 0) return TRI_ERR_INVALID_ARG;
-    if (max_row_len > kFusedMaxRow) {
-        // Rows too long to hold on chip: the two-call path, through the caller's score buffer.
+    // Fused for short rows (one CTA per row streams little and the selection
+    // launch is saved) and whenever no score buffer is given; long rows with a
+    // score buffer take the two-call path, which spreads a long row over many SMs.
+    const bool fused = max_row_len <= kFusedMaxRow && (max_row_len <= TRI_FUSED_PREFER_ROW || !scores);
+    if (!fused) {
         if (!scores) return TRI_ERR_INVALID_ARG;
         if ((st = tri_score(m, kv, K, pos, centres, mean_norm, p_now, offsets, n_offsets, key_mode, scores, ws,
                             ws_bytes, stream)) != TRI_OK)

@@ -13,11 +13,13 @@
 //     0 .. M-1 (M = N-W) by radix narrowing over the row's key range: at most
 //     three passes of 2048-bin shared-memory histograms, each over the keys
 //     still in range, one block scan per pass to find the bin.
-//  C. Marking and emission: thread t owns slots 64t .. 64t+63 (read in a
-//     rotated order so a warp's reads hit 32 distinct banks); keys above thr
-//     and the window are kept, and of the keys equal to thr the most recent
-//     ones (a block scan ranks the ties in slot order); a second block scan of
-//     the per-thread kept counts places every kept slot, ascending.
+//  C. Marking and emission: thread t owns slots ipt*t .. ipt*t+ipt-1, ipt =
+//     ceil(N / 512) (read in a rotated order; for ipt = 64 a warp's reads hit 32
+//     distinct banks); keys above thr and the window are kept, and of the keys
+//     equal to thr the most recent ones (a block scan ranks the ties in slot
+//     order); a second block scan of the per-thread kept counts places every
+//     kept slot, ascending.  Every pass is bounded by the row's length, so a
+//     short row costs little.
 // Blocks never wait on other blocks.  Rows longer than kFusedMaxRow are not
 // processed here (flagged; the host routes such calls to the unfused kernels).
 #include "score_common.cuh"
@@ -194,7 +196,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
             const int shift = nbits > 11 ? nbits - 11 : 0;
             for (int b = 0; b < kFBinsPerThread; b++) hist[tid * kFBinsPerThread + b] = 0u;
             __syncthreads();
-            for (int e = 0; e < kFItems; e++) {
+            const int passes = (M + kFThreads - 1) / kFThreads;
+            for (int e = 0; e < passes; e++) {
                 const int j = e * kFThreads + tid;
                 if (j < M) {
                     const uint32_t u = keys[j];
@@ -238,9 +241,12 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
 
     // ---- C. mark kept slots (rotated reads: lane l of a warp reads bank (e + l) % 32) and emit them ascending
     unsigned long long gt = 0, eq = 0, keep = 0;
-    for (int e = 0; e < kFItems; e++) {
-        const int pos = (e + tid) & (kFItems - 1);
-        const int j = kFItems * tid + pos;
+    const int ipt = (N + kFThreads - 1) / kFThreads;  // 1 .. kFItems slots per thread
+    const int rot = ipt ? tid % ipt : 0;               // rotation of the read order
+    for (int e = 0; e < ipt; e++) {
+        int pos = e + rot;
+        if (pos >= ipt) pos -= ipt;
+        const int j = ipt * tid + pos;
         if (j < N) {
             if (j >= M || K == 0 && N <= B) {
                 keep |= 1ull << pos;  // window slots, or every slot when N <= B
@@ -266,7 +272,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
     while (bits) {
         const int e = __ffsll((long long)bits) - 1;
         bits &= bits - 1;
-        if (o < (uint32_t)B) out[o] = kFItems * tid + e;
+        if (o < (uint32_t)B) out[o] = ipt * tid + e;
         o++;
     }
 }
