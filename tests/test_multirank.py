@@ -2,11 +2,9 @@
 independent cache shard, the step time is the max over ranks, and the
 whole-job throughput counts every rank's keys.  No data-path collective exists."""
 import hashlib
-import os
 import socket
 
 import numpy as np
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
