@@ -132,7 +132,8 @@ typedef struct {
 /* Human-readable name of a status code (static string). */
 const char *tri_status_str(tri_status s);
 
-/* Library version, (major << 16) | minor. */
+/* Library version, (major << 16) | minor.  0.2: tri_model carries rope_style and
+ * tri_kv_desc elem_type (both zero by default: rotate-half RoPE, bf16). */
 uint32_t tri_version(void);
 
 /* After a call returned TRI_ERR_CUDA: which CUDA call failed on this thread,

@@ -115,7 +115,7 @@ const char *tri_status_str(tri_status s) {
     return "TRI_ERR_UNKNOWN";
 }
 
-uint32_t tri_version(void) { return (0u << 16) | 1u; }
+uint32_t tri_version(void) { return (0u << 16) | 2u; }
 
 const char *tri_last_error(void) { return g_last_error; }
 
