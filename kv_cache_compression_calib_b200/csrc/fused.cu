@@ -28,7 +28,8 @@ namespace tri {
 
 constexpr int kFThreads = 512;
 constexpr int kFWarps = kFThreads / 32;
-constexpr int kFItems = kFusedMaxRow / kFThreads;  // 64 slots per thread
+constexpr int kFItems = kFusedMaxRow / kFThreads;  // most slots per thread (64)
+static_assert(kFusedMaxRow % kFThreads == 0 && kFItems <= 64, "a thread's slots fit its 64-bit masks");
 constexpr int kFBins = 2048;
 constexpr int kFBinsPerThread = kFBins / kFThreads;
 constexpr size_t kFusedSmem = (size_t)kFusedMaxRow * 4 + kFBins * 4;
