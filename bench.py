@@ -165,26 +165,35 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.fh.close()
-        rows = []
         with open(self.path) as fh:
-            for line in fh:
-                p = [x.strip() for x in line.split(",")]
-                if len(p) < 9:
-                    continue
-                try:
-                    ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                    rows.append((ts, float(p[1]), float(p[2]), p[5:9]))
-                except ValueError:
-                    continue
+            lines = fh.readlines()
         os.unlink(self.path)
-        pad = 0.0 if t_end - t_begin >= 0.3 else 0.12
-        win = [r for r in rows if t_begin - pad <= r[0] <= t_end + pad]
-        if not win:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
-                    "note": "timed region shorter than the sampling interval"}
-        reasons = sorted({self.REASONS[i] for r in win for i in range(4) if r[3][i].lower() == "active"})
-        return {"sm_mhz": statistics.median(r[1] for r in win), "sm_max_mhz": max(r[2] for r in win),
-                "reasons": reasons, "samples": len(win)}
+        return summarize_clock_samples(lines, t_begin, t_end)
+
+
+def summarize_clock_samples(lines, t_begin, t_end):
+    """Median SM clock, maximum clock and active throttle reasons of the nvidia-smi
+    samples (lines of ClockSampler.FIELDS, csv without units) stamped inside
+    [t_begin, t_end] (widened by 0.12 s when the region is shorter than 0.3 s);
+    malformed lines are skipped."""
+    rows = []
+    for line in lines:
+        p = [x.strip() for x in line.split(",")]
+        if len(p) < 9:
+            continue
+        try:
+            ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            rows.append((ts, float(p[1]), float(p[2]), p[5:9]))
+        except ValueError:
+            continue
+    pad = 0.0 if t_end - t_begin >= 0.3 else 0.12
+    win = [r for r in rows if t_begin - pad <= r[0] <= t_end + pad]
+    if not win:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                "note": "timed region shorter than the sampling interval"}
+    reasons = sorted({ClockSampler.REASONS[i] for r in win for i in range(4) if r[3][i].lower() == "active"})
+    return {"sm_mhz": statistics.median(r[1] for r in win), "sm_max_mhz": max(r[2] for r in win),
+            "reasons": reasons, "samples": len(win)}
 
 
 # ------------------------------------------------------- multi-rank logic
