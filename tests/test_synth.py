@@ -72,3 +72,33 @@ def test_seq_lengths_in_range():
     L = wl.seq_lengths()
     assert L.shape == (64,) and L.min() >= 4096 and L.max() <= 65536
     np.testing.assert_array_equal(L, wl.seq_lengths())
+
+
+def test_fp8_conversion_is_nearest_e4m3_of_the_clamped_value():
+    """to_fp8: every value becomes the e4m3 code nearest to it after clamping to
+    +-448, a tie between two representable values going to the code with the even
+    mantissa - checked by exhaustive search over the finite codes, decoded with the
+    oracle's definition of the format."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import synth
+
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_bits_to_f64(codes)
+    finite = ~np.isnan(vals)
+    cv, cc = vals[finite], codes[finite]
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.standard_normal(4000) * np.exp(rng.uniform(-12, 7, 4000)),
+                        [0.0, 448.0, -448.0, 1000.0, -1e9, 2.0 ** -10, 2.0 ** -9 * 1.5, 1.0625, 3.0 * 2.0 ** -9]])
+    x = x.astype(np.float32).astype(np.float64)  # the generator converts from fp32
+    got = synth.to_fp8(torch.tensor(x, dtype=torch.float32)).view(torch.uint8).numpy()
+    got_v = oracle.e4m3_bits_to_f64(got)
+    xc = np.clip(x, -448.0, 448.0)
+    for xi, gi, gv in zip(xc, got, got_v):
+        d = np.abs(cv - xi)
+        near = np.unique(cv[d == d.min()])
+        assert gv in near, (xi, gi, near)
+        if len(near) == 2:  # an exact tie between two values: the even mantissa wins
+            assert gi & 1 == 0, (xi, gi, near)
