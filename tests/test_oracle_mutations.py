@@ -66,6 +66,45 @@ MUTATIONS = [
     ("gather off by one",
      [("memcpy(dst + t * width, src + idx[t] * width, (size_t)width);",
        "memcpy(dst + t * width, src + (idx[t] > 0 ? idx[t] - 1 : 0) * width, (size_t)width);")]),
+    # slips confined to one form of the score (the collapsed form is the one the
+    # kernels are compared with), to the single series term, and to the diagnostics
+    ("collapsed: sine term added",
+     [("ldbl trig = cosl(x) * sr[f] - sinl(x) * si[f];", "ldbl trig = cosl(x) * sr[f] + sinl(x) * si[f];")]),
+    ("collapsed: offset phasor sum of cosines only",
+     [("si[f] += sinl(w[f] * (ldbl)offsets[e]);", "si[f] += cosl(w[f] * (ldbl)offsets[e]);")]),
+    ("collapsed: key phase added",
+     [("(ldbl)(p_now - pos[j]) + qa[g * F + f] - atan2l(ki, kr);",
+       "(ldbl)(p_now - pos[j]) + qa[g * F + f] + atan2l(ki, kr);")]),
+    ("absorbed: key not conjugated",
+     [("s += br * kr + bi * ki + cf[f] * hypotl(kr, ki);", "s += br * kr - bi * ki + cf[f] * hypotl(kr, ki);")]),
+    ("absorbed: rotation to p_now backwards",
+     [("ar[f] = tr * ec - ti * es;\n            ai[f] = tr * es + ti * ec;",
+       "ar[f] = tr * ec + ti * es;\n            ai[f] = ti * ec - tr * es;")]),
+    ("absorbed: norm coefficient summed over the group",
+     [("cf[f] = c / (ldbl)G;", "cf[f] = c;")]),
+    ("absorbed: pre-RoPE distance reversed",
+     [("ldbl a = w[f] * (ldbl)(p_now - pos[j]), ec", "ldbl a = w[f] * (ldbl)(pos[j] - p_now), ec")]),
+    ("series term: key phase added",
+     [("ldbl phi = atan2l(qi, qr) - atan2l(ki, kr);", "ldbl phi = atan2l(qi, qr) + atan2l(ki, kr);")]),
+    ("key centres: cached keys left rotated",
+     [("key_pair(d, il, keys + j * d, f, post_rope, w, pos[j], &kr, &ki);",
+       "key_pair(d, il, keys + j * d, f, 0, w, pos[j], &kr, &ki);")]),
+    ("key centres: mean norm as the norm of the mean",
+     [("mnorm[f] = n ? (double)(sn / (ldbl)n) : 0.0;", "mnorm[f] = n ? (double)(hypotl(sr, si) / (ldbl)n) : 0.0;")]),
+    ("key centres: imaginary part from the real dimension",
+     [("si += ki;", "si += kr;")]),
+    ("stats: centre magnitudes squared",
+     [("sc += a;", "sc += a * a;")]),
+    ("stats: drift relative to the current norms",
+     [("rm += ref_mnorm[f];", "rm += mnorm[f];")]),
+    ("online: magnitudes not weighted",
+     [("sn += w * hypotl(xr, xi);", "sn += hypotl(xr, xi);")]),
+    ("attention: lse without the maximum",
+     [("*lse = (double)(m + logl(den));", "*lse = (double)logl(den);")]),
+    ("attention: weights applied to the keys",
+     [("acc[t] += p * (ldbl)values[j * d + t];", "acc[t] += p * (ldbl)keys[j * d + t];")]),
+    ("select: NaN ranks first",
+     [("if (an != bn) return an ? 1 : -1;", "if (an != bn) return an ? -1 : 1;")]),
 ]
 
 PIN_FUNCS = [
@@ -87,6 +126,12 @@ PIN_FUNCS = [
     lambda: pins.test_key_centres_undo_rope(False),
     lambda: pins.test_calib_stats_closed_forms(),
     lambda: pins.test_attention_matches_torch_sdpa_and_closed_forms(),
+    lambda: pins.test_trig_series_negative_distance(),
+    lambda: pins.test_identical_queries_logit_sum_other_layouts(True, 64, True),
+    lambda: pins.test_identical_queries_logit_sum_other_layouts(False, 256, False),
+    lambda: pins.test_key_centres_undo_rope(True),
+    lambda: pins.test_select_nan_ranks_last_and_bad_args(),
+    lambda: pins.test_calib_interleaved_pairs(),
 ]
 
 
