@@ -684,8 +684,9 @@ def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, 
 # ------------------------------------------------------- CPU oracle leg
 
 def oracle_sample(wl, B, K_rows, V_rows, pos_rows, cs, ms, rows_meta, seconds, max_rows):
-    """K_rows/V_rows hold the stored bits (int16 for bf16, uint8 for fp8)."""
-    """Time the oracle (collapsed score + select + gather) on rows until `seconds` pass."""
+    """Time the oracle (collapsed score + select + gather) on rows until `seconds` pass.
+
+    K_rows/V_rows hold the stored bits (int16 for bf16, uint8 for fp8)."""
     import oracle
 
     keys = 0
