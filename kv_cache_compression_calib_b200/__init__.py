@@ -19,7 +19,8 @@ import torch
 
 from . import _abi
 from ._abi import (TRI_ELEM_BF16, TRI_ELEM_FP8_E4M3, TRI_FLAG_BLOCK_TABLE,  # noqa: F401
-                   TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS, TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
+                   TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS, TRI_FLAG_STAGE_TIMEOUT,
+                   TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
                    TRI_MAX_OFFSETS, TRI_ROPE_HALF, TRI_ROPE_INTERLEAVED, TriKvDesc, TriModel, TriOutDesc)
 
 _L = _abi.load()

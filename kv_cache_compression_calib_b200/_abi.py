@@ -18,6 +18,7 @@ TRI_ERR_DEVICE_FLAG = 6
 TRI_FLAG_ROW_OFFSETS = 0x1
 TRI_FLAG_NONFINITE = 0x2
 TRI_FLAG_BLOCK_TABLE = 0x4
+TRI_FLAG_STAGE_TIMEOUT = 0x8
 
 TRI_MAX_OFFSETS = 64
 TRI_ROPE_HALF = 0
