@@ -61,7 +61,7 @@ typedef enum {
 #define TRI_FLAG_ROW_OFFSETS 0x1u /* row_off not non-decreasing from 0 to total_keys */
 #define TRI_FLAG_NONFINITE 0x2u   /* a NaN score reached selection (ranked last) */
 #define TRI_FLAG_BLOCK_TABLE 0x4u /* paged: block id out of [0, n_blocks) or row too long for the table; the key is skipped */
-#define TRI_FLAG_STAGE_TIMEOUT 0x8u /* a staged copy of keys did not land within 2 s; that warp's remaining keys were not scored */
+#define TRI_FLAG_STAGE_TIMEOUT 0x8u /* a staged copy of keys did not land within 2 s; the warp that waited skipped its remaining keys */
 
 #define TRI_MAX_OFFSETS 64
 

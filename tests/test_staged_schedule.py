@@ -165,3 +165,84 @@ def test_large_totals_last_batches():
             n = min(st["kb"], end - b0)
             assert 0 < n <= st["kb"] and b0 + n == total
             assert (b0 + n) * st["rb"] <= total * st["rb"] and b0 * st["rb"] % 16 == 0
+
+
+# ---------------------------------------------------------------- key centres
+
+KC_CHUNKS = 16
+
+
+def kc_staging(post, elem, lpk):
+    ng, u, f = 32 // lpk, 4, 8 * lpk
+    kb, rb = ng * u, 2 * f * elem
+    key_bytes = kb * rb
+    pos_cap = kb + 4 if post else 0
+    slot = key_bytes + pos_cap * 4
+    acc = 24 * WARPS * lpk * 8
+    header = 256
+    per_cta = (228 * 1024 - 2 * 1024) // 2
+    fit = (per_cta - acc - header) // (WARPS * slot)
+    stages = max(2, min(4, fit))
+    smem = header + acc + WARPS * stages * slot
+    return dict(ng=ng, u=u, kb=kb, rb=rb, key_bytes=key_bytes, pos_cap=pos_cap, slot=slot, acc=acc,
+                header=header, stages=stages, smem=smem)
+
+
+KC_CONFIGS = [(post, elem, lpk) for lpk in (4, 8, 16) for post in (True, False) for elem in (2, 1)]
+
+
+@pytest.mark.parametrize("post,elem,lpk", KC_CONFIGS)
+def test_key_centre_shared_memory(post, elem, lpk):
+    st = kc_staging(post, elem, lpk)
+    assert st["slot"] % 16 == 0 and st["acc"] % 16 == 0 and st["kb"] % 4 == 0
+    assert WARPS * st["stages"] * 8 <= st["header"]
+    assert 2 * (st["smem"] + RESERVED_PER_CTA) <= SMEM_PER_SM, st
+
+
+def kc_batches(lo, hi, chunk, warp, st):
+    n = hi - lo
+    beg = lo + n * chunk // KC_CHUNKS
+    end = lo + n * (chunk + 1) // KC_CHUNKS
+    first = beg + warp * st["kb"]
+    nbw = (end - first + WARPS * st["kb"] - 1) // (WARPS * st["kb"]) if first < end else 0
+    for t in range(nbw):
+        b0 = first + t * WARPS * st["kb"]
+        yield t, b0, min(st["kb"], end - b0), beg, end
+
+
+@pytest.mark.parametrize("post,elem,lpk", KC_CONFIGS)
+@pytest.mark.parametrize("rows", [[0], [1], [5], [17, 0, 3], [4096, 4097, 33], [1000, 2049, 7, 65536 + 3]])
+def test_key_centre_copies_in_bounds_and_cover_rows(post, elem, lpk, rows):
+    st = kc_staging(post, elem, lpk)
+    offs = [0]
+    for n in rows:
+        offs.append(offs[-1] + n)
+    total = offs[-1]
+    seen = bytearray(total)
+    for r in range(len(rows)):
+        lo, hi = offs[r], offs[r + 1]
+        for chunk in range(KC_CHUNKS):
+            for warp in range(WARPS):
+                slots = {}
+                for t, b0, n, beg, end in kc_batches(lo, hi, chunk, warp, st):
+                    assert beg <= b0 and b0 + n <= end and n > 0
+                    # records
+                    assert (b0 * st["rb"]) % 16 == 0 and (n * st["rb"]) % 16 == 0
+                    assert b0 * st["rb"] + n * st["rb"] <= total * st["rb"]
+                    ring = st["header"] + st["acc"] + (warp * st["stages"] + t % st["stages"]) * st["slot"]
+                    assert ring % 16 == 0 and ring + st["slot"] <= st["smem"]
+                    # the positions window [a0, a1) inside the array, 16-byte aligned
+                    if post:
+                        a0 = b0 & ~3
+                        a1 = min((b0 + n + 3) & ~3, total & ~3)
+                        if a1 > a0:
+                            assert (a0 * 4) % 16 == 0 and ((a1 - a0) * 4) % 16 == 0
+                            assert 0 <= a0 and a1 <= total and a1 - a0 <= st["pos_cap"]
+                        # every key k of the batch reads spos[k - a0] when k < a1, else global memory
+                        for k in range(b0, b0 + n):
+                            if k < a1:
+                                assert 0 <= k - a0 < a1 - a0
+                    for k in range(b0, b0 + n):
+                        seen[k] += 1
+                    slots[t % st["stages"]] = t
+    assert all(c == 1 for c in seen)
