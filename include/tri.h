@@ -371,6 +371,26 @@ tri_status tri_score_noalloc(const tri_model *m, const tri_kv_desc *kv, const vo
                              const int32_t *offsets, int32_t n_offsets, int32_t key_mode, float *scores,
                              tri_stream_t stream);
 
+/*
+ * tri_selftest_wait_timeout - exercises the bounded wait of the staged kernels.
+ *
+ * Kernels that stage keys in shared memory wait on a barrier that their bulk
+ * copies complete; the wait gives up after a time limit and the kernel sets
+ * TRI_FLAG_STAGE_TIMEOUT instead of hanging.  This call launches one warp that
+ * waits on a barrier nothing ever completes, with the same wait and the limit
+ * given here, so a caller can see that path end: after the stream reaches it,
+ * tri_status_check(ws) returns TRI_ERR_DEVICE_FLAG with TRI_FLAG_STAGE_TIMEOUT
+ * set, and the context remains usable.  No memory is accessed out of bounds
+ * and nothing faults.
+ *   ws, ws_bytes: a workspace of at least 256 bytes, 256-byte aligned (only its
+ *             flag word is written).
+ *   limit_ns:  the wait's limit, 1 us .. 10 s.
+ * Returns TRI_OK once the kernel is enqueued; TRI_ERR_INVALID_ARG,
+ * TRI_ERR_ALIGNMENT or TRI_ERR_WORKSPACE_TOO_SMALL for bad arguments (nothing
+ * launched); TRI_ERR_CUDA when the launch fails.
+ */
+tri_status tri_selftest_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, tri_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

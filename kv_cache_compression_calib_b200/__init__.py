@@ -242,6 +242,14 @@ def tri_status_check(ws: torch.Tensor, stream=None):
     return st, int(flags.value)
 
 
+def tri_selftest_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Enqueue the self-test of the staged kernels' bounded wait: one warp waits
+    `limit_ns` on a barrier nothing completes and sets TRI_FLAG_STAGE_TIMEOUT
+    (read it with ``tri_status_check``)."""
+    _check(_L.tri_selftest_wait_timeout(_p(ws), ws.numel() * ws.element_size(), int(limit_ns), _s(stream)),
+           "tri_selftest_wait_timeout")
+
+
 def tri_score_noalloc(m: TriModel, kv: TriKvDesc, K: torch.Tensor, pos, centres: torch.Tensor,
                       mean_norm: torch.Tensor, p_now: torch.Tensor, offsets, key_mode: int,
                       scores: torch.Tensor, stream=None) -> None:

@@ -50,13 +50,14 @@ __device__ __forceinline__ unsigned long long global_ns() {
 }
 
 // Waits until the phase with parity `parity` of `bar` has completed.  Returns
-// false, without waiting further, after kStageWaitNs or kStageWaitIters tries.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// false, without waiting further, after limit_ns or kStageWaitIters tries.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          unsigned long long limit_ns = kStageWaitNs) {
     if (mbar_test(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (uint32_t it = 0; it < kStageWaitIters; it++) {
         if (mbar_test(bar, parity)) return true;
-        if (global_ns() - t0 > kStageWaitNs) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
     return false;
 }

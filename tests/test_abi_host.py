@@ -245,6 +245,16 @@ def test_status_check_rejects_bad_workspace():
     assert L.tri_status_check(A + 16, None, None) == _abi.TRI_ERR_ALIGNMENT
 
 
+def test_selftest_wait_rejects_bad_arguments():
+    """Checked before any launch, so no device is needed."""
+    L = _abi.load()
+    f = L.tri_selftest_wait_timeout
+    assert f(None, 256, 10**6, None) == _abi.TRI_ERR_INVALID_ARG
+    assert f(A, 255, 10**6, None) == _abi.TRI_ERR_WORKSPACE_TOO_SMALL
+    assert f(A + 16, 256, 10**6, None) == _abi.TRI_ERR_ALIGNMENT
+    assert f(A, 256, 999, None) == _abi.TRI_ERR_INVALID_ARG
+    assert f(A, 256, 10**10 + 1, None) == _abi.TRI_ERR_INVALID_ARG
+
 def test_binding_refuses_host_and_strided_tensors():
     """A host pointer or a strided view must never reach a kernel."""
     m = tri.model(1, 32, 8, 1e6)
