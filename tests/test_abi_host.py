@@ -254,6 +254,8 @@ def test_selftest_wait_rejects_bad_arguments():
     assert f(A + 16, 256, 10**6, None) == _abi.TRI_ERR_ALIGNMENT
     assert f(A, 256, 999, None) == _abi.TRI_ERR_INVALID_ARG
     assert f(A, 256, 10**10 + 1, None) == _abi.TRI_ERR_INVALID_ARG
+
+
 def test_header_constants_match_the_binding():
     """Every numeric #define, enum member and status code of include/tri.h has the
     same value in the Python binding, and the binding defines no TRI_ constant the
@@ -268,6 +270,7 @@ def test_header_constants_match_the_binding():
     assert len(header) >= 20
     binding = {k: v for k, v in vars(_abi).items() if k.startswith("TRI_") and isinstance(v, int)}
     assert header == binding
+
 
 def test_binding_refuses_host_and_strided_tensors():
     """A host pointer or a strided view must never reach a kernel."""
