@@ -214,6 +214,12 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
  *   kept_idx:   optional int32 [R][B]: kept slots of row r at r*B .. r*B+cnt-1
  *   kept_count: optional int32 [R]: min(N, B) per row
  *   ws:         workspace of tri_workspace_size bytes
+ * V, K_out, V_out and pos_out may also be page-locked host memory that the
+ * device addresses at the same pointer (cudaHostAlloc, or cudaHostRegister
+ * with cudaHostRegisterMapped, under unified addressing): only the kept
+ * records of V then cross the host link, and the compacted cache is written
+ * straight to host memory.  Pageable host memory must not be passed; the
+ * library cannot tell it from device memory.
  */
 tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *scores, int32_t B,
                        int32_t W, const void *K, const void *V, const int32_t *pos,
@@ -302,9 +308,10 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
  *     [total_keys]) required.
  * Both ways give the same results bit for bit (the fused kernel runs the
  * score kernel's arithmetic in the same order), so the choice is only speed.
- * Arguments as for tri_score and tri_compact; max_row_len is the caller's
- * bound on the longest row (for the compacted rounds of a serving loop,
- * min(N, B) + the new tokens).  Same workspace as tri_compact.
+ * Arguments as for tri_score and tri_compact (V and the outputs may be mapped
+ * page-locked host memory, as there); max_row_len is the caller's bound on the
+ * longest row (for the compacted rounds of a serving loop, min(N, B) + the new
+ * tokens).  Same workspace as tri_compact.
  */
 #define TRI_FUSED_MAX_ROW 32768
 #define TRI_FUSED_PREFER_ROW 8192

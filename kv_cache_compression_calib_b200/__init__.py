@@ -53,6 +53,21 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _pd(t):
+    """Pointer of a tensor the gather reads or writes record by record (V and the
+    compacted outputs): a contiguous CUDA tensor, or a contiguous page-locked host
+    tensor, which the device addresses at the same pointer under unified
+    addressing - the kept records then cross the host link directly.  Pageable
+    host memory is refused: the device cannot address it."""
+    if t is not None and not t.is_cuda:
+        if not t.is_pinned():
+            raise ValueError("expected a CUDA tensor or a pinned (page-locked) host tensor")
+        if not t.is_contiguous():
+            raise ValueError("expected a contiguous tensor (call .contiguous())")
+        return ctypes.c_void_p(t.data_ptr())
+    return _p(t)
+
+
 def _s(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -158,7 +173,7 @@ def tri_compact(m: TriModel, kv: TriKvDesc, scores: torch.Tensor, B: int, W: int
                 V_out: torch.Tensor, pos_out, kept_idx, kept_count, ws: torch.Tensor,
                 stream=None) -> None:
     _check(_L.tri_compact(ctypes.byref(m), ctypes.byref(kv), _p(scores), int(B), int(W), _p(K),
-                          _p(V), _p(pos), ctypes.byref(out), _p(K_out), _p(V_out), _p(pos_out),
+                          _pd(V), _p(pos), ctypes.byref(out), _pd(K_out), _pd(V_out), _pd(pos_out),
                           _p(kept_idx), _p(kept_count), _p(ws), ws.numel() * ws.element_size(),
                           _s(stream)), "tri_compact")
 
@@ -228,9 +243,9 @@ def tri_score_compact(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.Tens
                       kept_idx, kept_count, scores, ws: torch.Tensor, stream=None) -> None:
     """tri_score + tri_compact in one call, fused on chip when max_row_len <= TRI_FUSED_MAX_ROW."""
     offs = (ctypes.c_int32 * max(len(offsets), 1))(*[int(o) for o in offsets])
-    _check(_L.tri_score_compact(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(V), _p(pos), _p(centres),
+    _check(_L.tri_score_compact(ctypes.byref(m), ctypes.byref(kv), _p(K), _pd(V), _p(pos), _p(centres),
                                 _p(mean_norm), _p(p_now), offs, len(offsets), int(key_mode), int(B), int(W),
-                                int(max_row_len), ctypes.byref(out), _p(K_out), _p(V_out), _p(pos_out),
+                                int(max_row_len), ctypes.byref(out), _pd(K_out), _pd(V_out), _pd(pos_out),
                                 _p(kept_idx), _p(kept_count), _p(scores), _p(ws), ws.numel() * ws.element_size(),
                                 _s(stream)), "tri_score_compact")
 

@@ -272,6 +272,15 @@ def test_header_constants_match_the_binding():
     assert header == binding
 
 
+def test_binding_refuses_pageable_host_records():
+    """V and the compacted outputs may be pinned host tensors (the device addresses
+    them); pageable host memory is refused before anything is called."""
+    t = torch.zeros(64, 128, dtype=torch.bfloat16)
+    assert not t.is_pinned()
+    with pytest.raises(ValueError, match="pinned"):
+        tri._pd(t)
+    assert tri._pd(None) is None
+
 def test_binding_refuses_host_and_strided_tensors():
     """A host pointer or a strided view must never reach a kernel."""
     m = tri.model(1, 32, 8, 1e6)
