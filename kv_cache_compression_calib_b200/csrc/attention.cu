@@ -5,18 +5,20 @@
 //   s_j = scale * (q . k_j),  out = sum_j e^{s_j} v_j / sum_j e^{s_j},  lse = log sum_j e^{s_j}.
 //
 // A batched GEMV with G = Hq/H queries per KV head: 4 G flops per 2 d bytes of
-// K and V, bound by HBM, so CUDA cores, not tensor cores.  Pass 1: `chunks`
-// CTAs per row (about one wave over the SMs), each over a contiguous slice of
-// the row's keys in tiles of TK keys (64, or 32 for 512-byte records).  K and V
-// tiles are staged in shared memory with cp.async (16-byte copies,
-// double-buffered, rows padded by 16 bytes so lane-per-key reads hit distinct
-// banks).  QK: lane = key, warps split the tile's keys into 32-key halves and
-// the head dims into slices, partial dot products for all G queries (q
-// pre-scaled by scale * log2 e, broadcast from shared memory), added over the
-// dim slices in a fixed order.  Online softmax in base 2, one warp per query.
-// PV: each thread owns a pair of dims for all G queries over a group of the
-// tile's keys.  The slice's unnormalised output,
-// running maximum and sum go to the workspace.  Pass 2 merges a row's slices.
+// K and V, bound by HBM.  Pass 1 cuts every row into slices and writes each
+// slice's unnormalised output, running maximum and sum to the workspace; pass 2
+// (attn_combine_kernel) merges a row's slices.  Pass 1 has two kernels:
+// attn_partial_mma (d <= 128, warp-level tensor-core MMAs, below) and
+// attn_partial_simt (d = 256, CUDA cores), described here.  `chunks` CTAs per
+// row (about one wave over the SMs), each over a contiguous slice of the row's
+// keys in tiles of TK keys (64, or 32 for 512-byte records).  K and V tiles are
+// staged in shared memory with cp.async (16-byte copies, double-buffered, rows
+// padded by 16 bytes so lane-per-key reads hit distinct banks).  QK: lane =
+// key, warps split the tile's keys into 32-key halves and the head dims into
+// slices, partial dot products for all G queries (q pre-scaled by scale * log2
+// e, broadcast from shared memory), added over the dim slices in a fixed order.
+// Online softmax in base 2, one warp per query.  PV: each thread owns a pair of
+// dims for all G queries over a group of the tile's keys.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -306,16 +308,18 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_simt(const AttnPara
 // of tcgen05, and the op is HBM-bound, so the tensor pipe only takes the
 // multiply-adds off the CUDA cores.  bf16 caches use bf16 MMAs (the q and key
 // products are exact in fp32); fp8 caches use f16 MMAs with e4m3 converted to
-// f16 exactly and q rounded to f16 (exact for |q| in [2^-14, 65504]).  Each of
-// the 4 warps streams its own 16-key tiles (keys 16 (w + 4 i) .. of the CTA's
-// slice) through a private double buffer: no CTA barrier in the loop.
+// f16 exactly and q rounded to f16 (exact for |q| in [2^-14, 65504]).  A
+// persistent grid of the resident CTAs (4 warps each): every warp is a worker
+// that takes work items (row, slice) wid, wid + workers, ... and streams their
+// 16-key tiles through a private double buffer, prefetching across the end of
+// one item into the next, so there is no CTA barrier anywhere.
 //   S = Q K^T: K rows as the col-major B operand (ldmatrix, or e4m3 pairs
 //     converted in registers); scores scaled into base 2, masked past the slice.
 //   Online softmax per query row (4 lanes per row, shuffles).
 //   O += P V: the S accumulator fragments are the A fragments of the PV MMA;
 //     P is split into hi + lo halves (two MMAs) so P keeps ~16 bits; V via
 //     ldmatrix.trans (or e4m3 pairs gathered by key).
-// At the end the warps' (m, l, O) are merged in shared memory in warp order.
+// At the end of an item its worker writes the slice's (O, m, l) for the G rows.
 constexpr int kMmaWarps = 4;
 constexpr int kMmaThreads = 32 * kMmaWarps;
 constexpr int kMmaKeys = 16;  // keys per warp tile
