@@ -30,10 +30,12 @@
 // frequency pairs (with rotate-half RoPE: 8 consecutive real parts and the 8
 // matching imaginary parts d/2 elements later; with interleaved RoPE: 16
 // consecutive elements), so a warp instruction covers 32 / (d/16) keys'
-// records.  Every lane keeps U keys' loads in flight (U = 4 for d = 64, else
-// 8), accumulates its 8 pairs in fp32, and a butterfly reduce-scatter over the
-// lanes of a key leaves one full score per lane; a shuffle orders them for one
-// coalesced store per batch (32 keys, 16 for d = 256).
+// records.  Every lane keeps U keys' loads in flight (U = 4 for d = 64 and for
+// pre-RoPE caches, else 8), accumulates its 8 pairs in fp32, and a butterfly
+// reduce-scatter over the lanes of a key leaves one full score per lane; a
+// shuffle orders them for one coalesced store per batch (KB = 32 / (d/16) x U
+// keys).  Contiguous pre-RoPE and fp8 caches take score_staged_kernel (below),
+// which stages the same batches in shared memory.
 #include "score_common.cuh"
 #include "stage.cuh"
 
