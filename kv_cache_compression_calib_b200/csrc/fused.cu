@@ -6,9 +6,10 @@
 // the selection's re-reads happen, and no separate selection launch is made.
 //
 //  A. Scores: the streaming score kernel's lane layout and arithmetic (the same
-//     device functions, the same reduction order: bit-identical scores), the
-//     16 warps taking the row's 32-key batches in turn.  Optionally the fp32
-//     scores are also written to global memory.
+//     device functions, the same reduction order, and batches of KB keys on the
+//     same grid of multiples of KB in the concatenated key space, so the scores
+//     are bit-identical), the 16 warps taking the row's batches in turn.
+//     Optionally the fp32 scores are also written to global memory.
 //  B. Threshold: for N > B, the exact (B-W)-th best key value thr of slots
 //     0 .. M-1 (M = N-W) by radix narrowing over the row's key range: at most
 //     three passes of 2048-bin shared-memory histograms, each over the keys
