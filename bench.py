@@ -629,6 +629,11 @@ def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
 
 def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream, world,
             dev, fused_max_row=None):
+    """End to end through the public calls with the cache on the host: every step
+    copies K, pos, the row offsets, p_now and the centres from pinned host memory,
+    scores and compacts, with V and the compacted outputs left in pinned host memory
+    (the gather reads only the kept records of V over the link and writes the
+    compacted cache straight to the host), and reads the kept indices back."""
     try:
         hK = cache.K.cpu().pin_memory()
         hV = cache.V.cpu().pin_memory()
@@ -643,24 +648,28 @@ def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, 
         ok = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
     except RuntimeError as e:
         return {"value": None, "unit": UNIT, "skipped": f"pinned host buffers: {e}"[:200]}
-    ins = [(cache.K, hK), (cache.V, hV), (cache.pos, hpos), (cache.row_off, hro), (cache.p_now, hpn),
-           (centres, hc), (mnorm, hm)]
-    outs = [(oK, Ko), (oV, Vo), (op, po), (ok, kept)]
-    h2d = sum(h.numel() * h.element_size() for _, h in ins)
-    d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+    ins = [(cache.K, hK), (cache.pos, hpos), (cache.row_off, hro), (cache.p_now, hpn), (centres, hc), (mnorm, hm)]
+    outs = [(ok, kept)]
+    lens = np.diff(np.asarray(cache.row_off_np, dtype=np.int64))
+    n_kept = int(np.minimum(lens, B).sum())
+    rb = Ko.shape[-1] * Ko.element_size()
+    # bytes over the host link: the copies, the kept V records read in place, and the
+    # compacted K, V and positions written in place
+    h2d = sum(h.numel() * h.element_size() for _, h in ins) + n_kept * rb
+    d2h = sum(h.numel() * h.element_size() for h, _ in outs) + n_kept * (2 * rb + 4)
     steps = max(3, min(a.steps, 10))
 
     def step():
         for d, h in ins:
             d.copy_(h, non_blocking=True)
         if fused_max_row is not None:
-            tri.tri_score_compact(m, kv, cache.K, cache.V, cache.pos, centres, mnorm, cache.p_now, wl.offsets,
-                                  key_mode, B, wl.window, fused_max_row, tri.out_contig(), Ko, Vo, po, kept, None,
+            tri.tri_score_compact(m, kv, cache.K, hV, cache.pos, centres, mnorm, cache.p_now, wl.offsets,
+                                  key_mode, B, wl.window, fused_max_row, tri.out_contig(), oK, oV, op, kept, None,
                                   None, ws, stream)
         else:
             tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, wl.offsets, key_mode, scores, ws,
                           stream)
-            tri.tri_compact(m, kv, scores, B, wl.window, cache.K, cache.V, cache.pos, tri.out_contig(), Ko, Vo, po,
+            tri.tri_compact(m, kv, scores, B, wl.window, cache.K, hV, cache.pos, tri.out_contig(), oK, oV, op,
                             kept, None, ws, stream)
         for h, d in outs:
             h.copy_(d, non_blocking=True)
@@ -678,7 +687,8 @@ def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, 
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     return {"value": throughput(cache.total, world, ms / steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps}
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
+            "host_records": "V read and the compacted cache written in pinned host memory by the gather"}
 
 
 # ------------------------------------------------------- CPU oracle leg

@@ -61,6 +61,7 @@ typedef enum {
 #define TRI_FLAG_ROW_OFFSETS 0x1u /* row_off not non-decreasing from 0 to total_keys */
 #define TRI_FLAG_NONFINITE 0x2u   /* a NaN score reached selection (ranked last) */
 #define TRI_FLAG_BLOCK_TABLE 0x4u /* paged: block id out of [0, n_blocks) or row too long for the table; the key is skipped */
+#define TRI_FLAG_STAGE_TIMEOUT 0x8u /* a staged copy of keys did not land within 2 s; the warp that waited skipped its remaining keys */
 
 #define TRI_MAX_OFFSETS 64
 
@@ -213,6 +214,12 @@ tri_status tri_score(const tri_model *m, const tri_kv_desc *kv, const void *K, c
  *   kept_idx:   optional int32 [R][B]: kept slots of row r at r*B .. r*B+cnt-1
  *   kept_count: optional int32 [R]: min(N, B) per row
  *   ws:         workspace of tri_workspace_size bytes
+ * V, K_out, V_out and pos_out may also be page-locked host memory that the
+ * device addresses at the same pointer (cudaHostAlloc, or cudaHostRegister
+ * with cudaHostRegisterMapped, under unified addressing): only the kept
+ * records of V then cross the host link, and the compacted cache is written
+ * straight to host memory.  Pageable host memory must not be passed; the
+ * library cannot tell it from device memory.
  */
 tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *scores, int32_t B,
                        int32_t W, const void *K, const void *V, const int32_t *pos,
@@ -301,9 +308,10 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
  *     [total_keys]) required.
  * Both ways give the same results bit for bit (the fused kernel runs the
  * score kernel's arithmetic in the same order), so the choice is only speed.
- * Arguments as for tri_score and tri_compact; max_row_len is the caller's
- * bound on the longest row (for the compacted rounds of a serving loop,
- * min(N, B) + the new tokens).  Same workspace as tri_compact.
+ * Arguments as for tri_score and tri_compact (V and the outputs may be mapped
+ * page-locked host memory, as there); max_row_len is the caller's bound on the
+ * longest row (for the compacted rounds of a serving loop, min(N, B) + the new
+ * tokens).  Same workspace as tri_compact.
  */
 #define TRI_FUSED_MAX_ROW 32768
 #define TRI_FUSED_PREFER_ROW 8192
@@ -369,6 +377,26 @@ tri_status tri_score_noalloc(const tri_model *m, const tri_kv_desc *kv, const vo
                              const float *centres, const float *mean_norm, const int64_t *p_now,
                              const int32_t *offsets, int32_t n_offsets, int32_t key_mode, float *scores,
                              tri_stream_t stream);
+
+/*
+ * tri_selftest_wait_timeout - exercises the bounded wait of the staged kernels.
+ *
+ * Kernels that stage keys in shared memory wait on a barrier that their bulk
+ * copies complete; the wait gives up after a time limit and the kernel sets
+ * TRI_FLAG_STAGE_TIMEOUT instead of hanging.  This call launches one warp that
+ * waits on a barrier nothing ever completes, with the same wait and the limit
+ * given here, so a caller can see that path end: after the stream reaches it,
+ * tri_status_check(ws) returns TRI_ERR_DEVICE_FLAG with TRI_FLAG_STAGE_TIMEOUT
+ * set, and the context remains usable.  No memory is accessed out of bounds
+ * and nothing faults.
+ *   ws, ws_bytes: a workspace of at least 256 bytes, 256-byte aligned (only its
+ *             flag word is written).
+ *   limit_ns:  the wait's limit, 1 us .. 10 s.
+ * Returns TRI_OK once the kernel is enqueued; TRI_ERR_INVALID_ARG,
+ * TRI_ERR_ALIGNMENT or TRI_ERR_WORKSPACE_TOO_SMALL for bad arguments (nothing
+ * launched); TRI_ERR_CUDA when the launch fails.
+ */
+tri_status tri_selftest_wait_timeout(void *ws, size_t ws_bytes, uint64_t limit_ns, tri_stream_t stream);
 
 #ifdef __cplusplus
 }

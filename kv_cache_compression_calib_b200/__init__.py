@@ -19,7 +19,8 @@ import torch
 
 from . import _abi
 from ._abi import (TRI_ELEM_BF16, TRI_ELEM_FP8_E4M3, TRI_FLAG_BLOCK_TABLE,  # noqa: F401
-                   TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS, TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
+                   TRI_FLAG_NONFINITE, TRI_FLAG_ROW_OFFSETS, TRI_FLAG_STAGE_TIMEOUT,
+                   TRI_KEYS_POST_ROPE, TRI_KEYS_PRE_ROPE, TRI_KV_CONTIG, TRI_KV_PAGED,
                    TRI_MAX_OFFSETS, TRI_ROPE_HALF, TRI_ROPE_INTERLEAVED, TriKvDesc, TriModel, TriOutDesc)
 
 _L = _abi.load()
@@ -50,6 +51,21 @@ def _p(t):
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor (call .contiguous())")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _pd(t):
+    """Pointer of a tensor the gather reads or writes record by record (V and the
+    compacted outputs): a contiguous CUDA tensor, or a contiguous page-locked host
+    tensor, which the device addresses at the same pointer under unified
+    addressing - the kept records then cross the host link directly.  Pageable
+    host memory is refused: the device cannot address it."""
+    if t is not None and not t.is_cuda:
+        if not t.is_pinned():
+            raise ValueError("expected a CUDA tensor or a pinned (page-locked) host tensor")
+        if not t.is_contiguous():
+            raise ValueError("expected a contiguous tensor (call .contiguous())")
+        return ctypes.c_void_p(t.data_ptr())
+    return _p(t)
 
 
 def _s(stream):
@@ -157,7 +173,7 @@ def tri_compact(m: TriModel, kv: TriKvDesc, scores: torch.Tensor, B: int, W: int
                 V_out: torch.Tensor, pos_out, kept_idx, kept_count, ws: torch.Tensor,
                 stream=None) -> None:
     _check(_L.tri_compact(ctypes.byref(m), ctypes.byref(kv), _p(scores), int(B), int(W), _p(K),
-                          _p(V), _p(pos), ctypes.byref(out), _p(K_out), _p(V_out), _p(pos_out),
+                          _pd(V), _p(pos), ctypes.byref(out), _pd(K_out), _pd(V_out), _pd(pos_out),
                           _p(kept_idx), _p(kept_count), _p(ws), ws.numel() * ws.element_size(),
                           _s(stream)), "tri_compact")
 
@@ -227,9 +243,9 @@ def tri_score_compact(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.Tens
                       kept_idx, kept_count, scores, ws: torch.Tensor, stream=None) -> None:
     """tri_score + tri_compact in one call, fused on chip when max_row_len <= TRI_FUSED_MAX_ROW."""
     offs = (ctypes.c_int32 * max(len(offsets), 1))(*[int(o) for o in offsets])
-    _check(_L.tri_score_compact(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(V), _p(pos), _p(centres),
+    _check(_L.tri_score_compact(ctypes.byref(m), ctypes.byref(kv), _p(K), _pd(V), _p(pos), _p(centres),
                                 _p(mean_norm), _p(p_now), offs, len(offsets), int(key_mode), int(B), int(W),
-                                int(max_row_len), ctypes.byref(out), _p(K_out), _p(V_out), _p(pos_out),
+                                int(max_row_len), ctypes.byref(out), _pd(K_out), _pd(V_out), _pd(pos_out),
                                 _p(kept_idx), _p(kept_count), _p(scores), _p(ws), ws.numel() * ws.element_size(),
                                 _s(stream)), "tri_score_compact")
 
@@ -239,6 +255,14 @@ def tri_status_check(ws: torch.Tensor, stream=None):
     flags = ctypes.c_uint32(0)
     st = _L.tri_status_check(_p(ws), ctypes.byref(flags), _s(stream))
     return st, int(flags.value)
+
+
+def tri_selftest_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Enqueue the self-test of the staged kernels' bounded wait: one warp waits
+    `limit_ns` on a barrier nothing completes and sets TRI_FLAG_STAGE_TIMEOUT
+    (read it with ``tri_status_check``)."""
+    _check(_L.tri_selftest_wait_timeout(_p(ws), ws.numel() * ws.element_size(), int(limit_ns), _s(stream)),
+           "tri_selftest_wait_timeout")
 
 
 def tri_score_noalloc(m: TriModel, kv: TriKvDesc, K: torch.Tensor, pos, centres: torch.Tensor,

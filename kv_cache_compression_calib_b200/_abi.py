@@ -18,6 +18,7 @@ TRI_ERR_DEVICE_FLAG = 6
 TRI_FLAG_ROW_OFFSETS = 0x1
 TRI_FLAG_NONFINITE = 0x2
 TRI_FLAG_BLOCK_TABLE = 0x4
+TRI_FLAG_STAGE_TIMEOUT = 0x8
 
 TRI_MAX_OFFSETS = 64
 TRI_ROPE_HALF = 0
@@ -33,7 +34,7 @@ TRI_KEYS_PRE_ROPE = 1
 EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_size", "tri_workspace_init", "tri_calib",
            "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc", "tri_calib_update",
            "tri_calib_stats", "tri_key_centres_ws_size", "tri_key_centres", "tri_attention_ws_size",
-           "tri_decode_attention", "tri_score_compact")
+           "tri_decode_attention", "tri_score_compact", "tri_selftest_wait_timeout")
 TRI_FUSED_MAX_ROW = 32768
 TRI_FUSED_PREFER_ROW = 8192
 TRI_NOALLOC_MAX_ROWS = 4096
@@ -113,6 +114,8 @@ def load(path: str = LIB_PATH):
                               _P, _P, ctypes.c_size_t, _P]
     L.tri_status_check.restype = ctypes.c_int
     L.tri_status_check.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), _P]
+    L.tri_selftest_wait_timeout.restype = ctypes.c_int
+    L.tri_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint64, _P]
     L.tri_score_noalloc.restype = ctypes.c_int
     L.tri_score_noalloc.argtypes = [ctypes.POINTER(TriModel), ctypes.POINTER(TriKvDesc), _P, _P, _P, _P,
                                     _P, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, ctypes.c_int32,

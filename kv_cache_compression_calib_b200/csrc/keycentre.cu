@@ -16,6 +16,7 @@
 // so results are deterministic.  It reads every key once: an HBM-bound pass like
 // the scoring one (plus one sin/cos per (key, pair) for a RoPE cache).
 #include "score_common.cuh"
+#include "stage.cuh"
 
 namespace tri {
 
@@ -153,6 +154,202 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
     }
 }
 
+// Contiguous caches: the same pass with each warp's batches staged in shared
+// memory by bulk copies, STAGES batches ahead (see stage.cuh), so the bytes in
+// flight do not depend on registers.  A chunk may start at any key, so each
+// batch also stages the 16-byte-aligned window of positions around its keys.
+// To leave room for the ring, a flush folds the lanes' fp32 runs in fp64
+// across the lanes of the warp that hold the same pairs (a fixed shuffle
+// tree) into one column per (warp, lane group); the final sum runs over warps
+// in order.  Deterministic, like the unstaged pass.
+template <bool POST, int ELEM, int LPK>
+struct KcStaging {
+    static constexpr int kWarps = kKcThreads / 32;
+    static constexpr int NG = 32 / LPK, U = 4, KB = NG * U, F = 8 * LPK;
+    static constexpr int RB = 2 * F * ELEM;
+    static constexpr int KEY_BYTES = KB * RB;
+    static constexpr int POS_CAP = POST ? KB + 4 : 0;  // aligned window of a batch's positions
+    static constexpr int SLOT = KEY_BYTES + POS_CAP * 4;
+    static constexpr int ACC_BYTES = 24 * kWarps * LPK * 8;
+    static constexpr int HEADER = 256;  // the barriers (at most 8 warps x 4 stages)
+    // Two CTAs per SM: 228 KB less 1 KB reserved per CTA.
+    static constexpr int PER_CTA = (228 * 1024 - 2 * 1024) / 2;
+    static constexpr int FIT = (PER_CTA - ACC_BYTES - HEADER) / (kWarps * SLOT);
+    static constexpr int STAGES = FIT < 2 ? 2 : (FIT > 4 ? 4 : FIT);
+    static constexpr size_t SMEM = (size_t)HEADER + ACC_BYTES + (size_t)kWarps * STAGES * SLOT;
+    static_assert(KB % 4 == 0 && SLOT % 16 == 0 && KEY_BYTES % 16 == 0 && ACC_BYTES % 16 == 0, "16-byte units");
+    static_assert(kWarps * STAGES * 8 <= HEADER, "barriers fit the header");
+    static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+};
+
+// Issues batch t of a warp (keys b0 .. b0 + n - 1) into slot t % STAGES: its
+// records, and the positions [a0, a1) of the 16-byte-aligned window around
+// them that lies inside the array.  One thread per warp.
+template <typename St>
+__device__ __forceinline__ void kc_stage_batch(const KeyCentreParams &p, int64_t b0, int n, unsigned char *ring,
+                                               uint64_t *bar, int t, unsigned long long pol) {
+    unsigned char *slot = ring + (t % St::STAGES) * St::SLOT;
+    uint64_t *b = &bar[t % St::STAGES];
+    const uint32_t kbytes = (uint32_t)n * St::RB;
+    uint32_t pbytes = 0;
+    int64_t a0 = 0;
+    if (St::POS_CAP) {
+        a0 = b0 & ~int64_t(3);
+        const int64_t a1 = min((b0 + n + 3) & ~int64_t(3), p.geo.total & ~int64_t(3));
+        if (a1 > a0) pbytes = (uint32_t)(a1 - a0) * 4u;
+    }
+    mbar_arrive_expect_tx(b, kbytes + pbytes);
+    bulk_load(slot, p.K + b0 * St::RB, kbytes, b, pol);
+    if (pbytes) bulk_load(slot + St::KEY_BYTES, p.pos + a0, pbytes, b, pol);
+}
+
+template <bool POST, int ELEM, bool IL, int LPK>
+__global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const KeyCentreParams p) {
+    using St = KcStaging<POST, ELEM, LPK>;
+    constexpr int NG = St::NG, U = St::U, KB = St::KB, F = St::F, RB = St::RB, W = St::kWarps;
+    constexpr int STAGES = St::STAGES;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+    double *acc = reinterpret_cast<double *>(smem + St::HEADER);  // [24][W * LPK]
+    unsigned char *rings = smem + St::HEADER + St::ACC_BYTES;
+    const Geometry &geo = p.geo;
+    const int64_t r = blockIdx.x / kKeyCentreChunks;
+    const int chunk = (int)(blockIdx.x % kKeyCentreChunks);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int q = lane / LPK, gl = lane % LPK;
+    int64_t lo = geo.row_off[r], hi = geo.row_off[r + 1];
+    if (lo < 0 || hi < lo || hi > geo.total) {
+        if (threadIdx.x == 0 && chunk == 0) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
+        lo = hi = 0;
+    }
+    const int64_t n = hi - lo;
+    const int64_t beg = lo + n * chunk / kKeyCentreChunks;
+    const int64_t end = lo + n * (chunk + 1) / kKeyCentreChunks;
+    // This warp's batches: keys beg + (warp + t W) KB ..., t = 0 .. nbw - 1.
+    const int64_t first0 = beg + (int64_t)warp * KB;
+    const int nbw = first0 < end ? (int)((end - first0 + (int64_t)W * KB - 1) / ((int64_t)W * KB)) : 0;
+
+    unsigned long long T[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        T[i] = POST ? __double2ull_rn(pow(p.theta, -2.0 * (double)(8 * gl + i) / (double)(2 * F)) * kKcTurnScale)
+                    : 0ull;
+    float stc[8], sts[8];
+    if (POST) phasors(T, (int64_t)NG, stc, sts);
+    const unsigned long long pol = policy_evict_first();
+    uint64_t *bar = bars + warp * STAGES;
+    unsigned char *ring = rings + (size_t)warp * STAGES * St::SLOT;
+
+    for (int e = threadIdx.x; e < 24 * W * LPK; e += kKcThreads) acc[e] = 0.0;
+    if (lane == 0) {
+#pragma unroll
+        for (int k = 0; k < STAGES; k++) mbar_init(&bar[k], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (lane == 0)
+        for (int t = 0; t < min(nbw, STAGES); t++) {
+            const int64_t b0 = first0 + (int64_t)t * W * KB;
+            kc_stage_batch<St>(p, b0, (int)min((int64_t)KB, end - b0), ring, bar, t, pol);
+        }
+
+    float fr[8], fi[8], fn[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) fr[i] = fi[i] = fn[i] = 0.f;
+    // Adds the lanes' runs into this warp's columns: fp64 tree over the NG lanes
+    // of each lane group, then lane group gl's column.
+    auto fold = [&]() {
+#pragma unroll
+        for (int c3 = 0; c3 < 3; c3++)
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                double v = (double)(c3 == 0 ? fr[i] : c3 == 1 ? fi[i] : fn[i]);
+#pragma unroll
+                for (int o = LPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (q == 0) acc[(c3 * 8 + i) * (W * LPK) + warp * LPK + gl] += v;
+            }
+#pragma unroll
+        for (int i = 0; i < 8; i++) fr[i] = fi[i] = fn[i] = 0.f;
+    };
+
+    int run = 0;
+    for (int t = 0; t < nbw; t++) {
+        const int64_t b0 = first0 + (int64_t)t * W * KB;
+        const int nk = (int)min((int64_t)KB, end - b0);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar[t % STAGES], (uint32_t)(t / STAGES) & 1u))) {
+            // A copy did not land: flag it, wait once more (bounded) for every copy
+            // still in flight into this warp's ring, and skip the warp's other keys.
+            if (lane == 0) atomicOr(p.flags, TRI_FLAG_STAGE_TIMEOUT);
+            for (int j = t; j < min(nbw, t + STAGES); j++) mbar_wait(&bar[j % STAGES], (uint32_t)(j / STAGES) & 1u);
+            break;
+        }
+        const unsigned char *slot = ring + (t % STAGES) * St::SLOT;
+        const int32_t *spos = reinterpret_cast<const int32_t *>(slot + St::KEY_BYTES);
+        const int64_t a0 = b0 & ~int64_t(3);
+        const int64_t a1 = POST ? min((b0 + nk + 3) & ~int64_t(3), geo.total & ~int64_t(3)) : 0;
+        KeyChunk<ELEM, IL, F> kc[U];
+        int32_t kpos[U];
+        bool valid[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int idx = NG * u + q;
+            const int64_t k = b0 + idx;
+            valid[u] = idx < nk;
+            kpos[u] = 0;
+            if (valid[u]) {
+                kc[u].lds(slot + idx * RB, gl);
+                if (POST) kpos[u] = k < a1 ? spos[k - a0] : __ldg(p.pos + k);
+            } else {
+                kc[u].zero();
+            }
+        }
+        float cs[8], sn[8];
+        if (POST) phasors(T, (int64_t)kpos[0], cs, sn);
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            if (POST && u > 0) {
+                if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
+                else phasors(T, (int64_t)kpos[u], cs, sn);
+            }
+            if (!valid[u]) continue;
+            float x[8], y[8];
+            kc[u].unpack(x, y);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                float xr = x[i], xi = y[i];
+                if (POST) {
+                    xr = x[i] * cs[i] + y[i] * sn[i];
+                    xi = y[i] * cs[i] - x[i] * sn[i];
+                }
+                fr[i] += xr;
+                fi[i] += xi;
+                fn[i] += sqrt_approx(fmaf(x[i], x[i], y[i] * y[i]));
+            }
+        }
+        if (t + STAGES < nbw) {  // the slot's bytes are consumed: refill it
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int64_t bn = first0 + (int64_t)(t + STAGES) * W * KB;
+                kc_stage_batch<St>(p, bn, (int)min((int64_t)KB, end - bn), ring, bar, t + STAGES, pol);
+            }
+        }
+        if (++run == kFlush) {
+            run = 0;
+            fold();
+        }
+    }
+    fold();
+    __syncthreads();
+    for (int e = threadIdx.x; e < 3 * F; e += kKcThreads) {
+        const int f = e % F, comp = e / F;
+        const int g = f >> 3, i = f & 7;
+        double v = 0.0;
+        for (int w = 0; w < W; w++) v += acc[(comp * 8 + i) * (W * LPK) + w * LPK + g];
+        p.partial[((r * kKeyCentreChunks + chunk) * F + f) * 3 + comp] = v;
+    }
+}
+
 template <int F>
 __global__ void __launch_bounds__(F) key_centre_finalize(const KeyCentreParams p) {
     const int64_t r = blockIdx.x;
@@ -181,11 +378,30 @@ static cudaError_t launch_kc_t(const KeyCentreParams &p, int64_t R, cudaStream_t
     return cudaGetLastError();
 }
 
+template <bool POST, int ELEM, bool IL, int LPK>
+static cudaError_t launch_kc_staged_t(const KeyCentreParams &p, int64_t R, cudaStream_t s) {
+    using St = KcStaging<POST, ELEM, LPK>;
+    auto kern = key_centre_staged_kernel<POST, ELEM, IL, LPK>;
+    static bool set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!set[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)St::SMEM);
+        if (e != cudaSuccess) return e;
+        set[dev & 63] = true;
+    }
+    kern<<<(unsigned)(R * kKeyCentreChunks), kKcThreads, St::SMEM, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    key_centre_finalize<8 * LPK><<<(unsigned)R, 8 * LPK, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <int ELEM, bool IL, int LPK>
 static cudaError_t launch_kc_d(const KeyCentreParams &p, int64_t R, cudaStream_t s) {
     const bool paged = p.geo.layout == TRI_KV_PAGED;
     if (paged) return p.post_rope ? launch_kc_t<true, true, ELEM, IL, LPK>(p, R, s) : launch_kc_t<true, false, ELEM, IL, LPK>(p, R, s);
-    return p.post_rope ? launch_kc_t<false, true, ELEM, IL, LPK>(p, R, s) : launch_kc_t<false, false, ELEM, IL, LPK>(p, R, s);
+    return p.post_rope ? launch_kc_staged_t<true, ELEM, IL, LPK>(p, R, s) : launch_kc_staged_t<false, ELEM, IL, LPK>(p, R, s);
 }
 
 template <int ELEM, bool IL>

@@ -39,7 +39,8 @@ __device__ __forceinline__ void unpack_bf16_pairs(const uint4 a, const uint4 b, 
 // 8gl..8gl+7, imaginary parts F dims later - 2 x 16 bytes for bf16, 2 x 8 bytes
 // for fp8.  Interleaved (IL = true): dims 16gl..16gl+15, (re, im) adjacent -
 // 32 bytes for bf16, 16 for fp8.  Every load is naturally aligned: records are
-// 64..512 bytes long and start at multiples of their length from K.
+// 64..512 bytes long and start at multiples of their length from K.  `lds`
+// reads the same bytes of a record staged in shared memory.
 template <int ELEM, bool IL, int F>
 struct KeyChunk;
 
@@ -49,6 +50,10 @@ struct KeyChunk<2, false, F> {
     __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
         re = ld_stream16(key + 16 * gl, pol);
         im = ld_stream16(key + 2 * F + 16 * gl, pol);
+    }
+    __device__ __forceinline__ void lds(const unsigned char *key, int gl) {
+        re = *reinterpret_cast<const uint4 *>(key + 16 * gl);
+        im = *reinterpret_cast<const uint4 *>(key + 2 * F + 16 * gl);
     }
     __device__ __forceinline__ void zero() { re = im = make_uint4(0u, 0u, 0u, 0u); }
     __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
@@ -64,6 +69,10 @@ struct KeyChunk<1, false, F> {
         re = ld_stream8(key + 8 * gl, pol);
         im = ld_stream8(key + F + 8 * gl, pol);
     }
+    __device__ __forceinline__ void lds(const unsigned char *key, int gl) {
+        re = *reinterpret_cast<const uint2 *>(key + 8 * gl);
+        im = *reinterpret_cast<const uint2 *>(key + F + 8 * gl);
+    }
     __device__ __forceinline__ void zero() { re = im = make_uint2(0u, 0u); }
     __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {
         unpack_e4m3x8(re, x);
@@ -78,6 +87,10 @@ struct KeyChunk<2, true, F> {
         a = ld_stream16(key + 32 * gl, pol);
         b = ld_stream16(key + 32 * gl + 16, pol);
     }
+    __device__ __forceinline__ void lds(const unsigned char *key, int gl) {
+        a = *reinterpret_cast<const uint4 *>(key + 32 * gl);
+        b = *reinterpret_cast<const uint4 *>(key + 32 * gl + 16);
+    }
     __device__ __forceinline__ void zero() { a = b = make_uint4(0u, 0u, 0u, 0u); }
     __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const { unpack_bf16_pairs(a, b, x, y); }
 };
@@ -87,6 +100,9 @@ struct KeyChunk<1, true, F> {
     uint4 v;
     __device__ __forceinline__ void load(const char *key, int gl, unsigned long long pol) {
         v = ld_stream16(key + 16 * gl, pol);
+    }
+    __device__ __forceinline__ void lds(const unsigned char *key, int gl) {
+        v = *reinterpret_cast<const uint4 *>(key + 16 * gl);
     }
     __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
     __device__ __forceinline__ void unpack(float (&x)[8], float (&y)[8]) const {

@@ -245,6 +245,17 @@ def test_status_check_rejects_bad_workspace():
     assert L.tri_status_check(A + 16, None, None) == _abi.TRI_ERR_ALIGNMENT
 
 
+def test_selftest_wait_rejects_bad_arguments():
+    """Checked before any launch, so no device is needed."""
+    L = _abi.load()
+    f = L.tri_selftest_wait_timeout
+    assert f(None, 256, 10**6, None) == _abi.TRI_ERR_INVALID_ARG
+    assert f(A, 255, 10**6, None) == _abi.TRI_ERR_WORKSPACE_TOO_SMALL
+    assert f(A + 16, 256, 10**6, None) == _abi.TRI_ERR_ALIGNMENT
+    assert f(A, 256, 999, None) == _abi.TRI_ERR_INVALID_ARG
+    assert f(A, 256, 10**10 + 1, None) == _abi.TRI_ERR_INVALID_ARG
+
+
 def test_header_constants_match_the_binding():
     """Every numeric #define, enum member and status code of include/tri.h has the
     same value in the Python binding, and the binding defines no TRI_ constant the
@@ -259,6 +270,17 @@ def test_header_constants_match_the_binding():
     assert len(header) >= 20
     binding = {k: v for k, v in vars(_abi).items() if k.startswith("TRI_") and isinstance(v, int)}
     assert header == binding
+
+
+def test_binding_refuses_pageable_host_records():
+    """V and the compacted outputs may be pinned host tensors (the device addresses
+    them); pageable host memory is refused before anything is called."""
+    t = torch.zeros(64, 128, dtype=torch.bfloat16)
+    assert not t.is_pinned()
+    with pytest.raises(ValueError, match="pinned"):
+        tri._pd(t)
+    assert tri._pd(None) is None
+
 
 def test_binding_refuses_host_and_strided_tensors():
     """A host pointer or a strided view must never reach a kernel."""

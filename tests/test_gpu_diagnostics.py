@@ -129,6 +129,35 @@ def test_key_centres_contig(d, style, elem, mode):
         assert err < 0.1, (h, err)
 
 
+
+@pytest.mark.parametrize("elem,mode", [("bf16", "post"), ("fp8", "post"), ("bf16", "pre")])
+def test_key_centres_short_rows_ragged_total(elem, mode):
+    """One KV head, rows of 1001, 2, 37, 0 and 5 keys: chunks start at unaligned keys,
+    rows shorter than a batch, and a total (1045) that is not a multiple of 4, so the
+    last positions sit past the array's last whole 16-byte group."""
+    wl = synth.WORKLOADS["single_layer_4k"].with_(name="kc1", n_q_heads=4, n_kv_heads=1, batch=5, n_calib=8)
+    post = mode == "post"
+    lens = [1001, 2, 37, 0, 5]
+    host = synth.make_contig(wl, "cpu", lens=lens, rotate=post)
+    if elem == "fp8":
+        host.K = synth.to_fp8(host.K)
+    assert host.total == 1045
+    m = model_of(wl, 1)
+    kv = tri.kv_contig(len(lens), host.row_off.to(DEV), host.total, tri.elem_type_of(host.K))
+    R, F = host.n_rows, 64
+    kmode = tri.TRI_KEYS_POST_ROPE if post else tri.TRI_KEYS_PRE_ROPE
+    far = host.pos + 123457
+    c, n = run_key_centres(m, kv, host.K.to(DEV), far.to(DEV) if post else None, kmode, R, F, len(lens))
+    K = H.to_f64(host.K)
+    pos = far.numpy().astype(np.int64)
+    for r in range(R):
+        a, b = host.row_off_np[r], host.row_off_np[r + 1]
+        if b == a:
+            assert np.all(c[r] == 0) and np.all(n[r] == 0)
+            continue
+        rc, rm = oracle.key_centres(wl.theta, K[a:b], pos[a:b], post, wl.interleaved)
+        check_centres(c[r], n[r], rc, rm)
+
 def test_key_centres_paged():
     wl = synth.WORKLOADS["paged_16seq"].with_(name="kcp", batch=3, n_calib=8)
     lens = np.array([300, 2100, 1024])

@@ -150,3 +150,20 @@ def test_single_key_budgets(B, W):
     res = gpu_compact(dev, torch.tensor(ref32, dtype=torch.float32, device=DEV), B, W)
     assert res["status"] == 0
     check_compaction_exact(host, res, ref32, B, W)
+
+
+@pytest.mark.parametrize("elem,mode", [("bf16", PRE), ("fp8", PRE), ("fp8", POST)])
+def test_scores_with_a_total_not_a_multiple_of_four(elem, mode):
+    """One KV head, rows of 1001, 2, 37, 0 and 5 keys (1045 in all): the last batch's
+    final positions lie past the array's last whole 16-byte group, and rows shorter
+    than a batch sit between longer ones."""
+    wl = synth.WORKLOADS["single_layer_4k"].with_(name="odd", n_q_heads=4, n_kv_heads=1, batch=5, n_calib=32)
+    host = synth.make_contig(wl, "cpu", lens=[1001, 2, 37, 0, 5], rotate=(mode == POST))
+    if elem == "fp8":
+        host.K, host.V = synth.to_fp8(host.K), synth.to_fp8(host.V)
+    assert host.total == 1045
+    cs, ms = oracle_centres(host)
+    dev = to_dev(host)
+    got = gpu_score(dev, cs, ms, key_mode=mode).cpu().numpy().astype(np.float64)
+    ref, bound = oracle_scores(host, cs, ms, post_rope=(mode == POST), tier="collapsed")
+    assert H.score_error(got[:host.total], ref, bound) <= 1e-4

@@ -63,7 +63,9 @@ def assert_identical(a, b, scores=True):
 
 @pytest.mark.parametrize("d,style,elem,mode", [(128, "half", "bf16", POST), (128, "half", "bf16", PRE),
                                                (128, "half", "fp8", POST), (64, "interleaved", "bf16", POST),
-                                               (256, "half", "bf16", POST), (256, "interleaved", "fp8", PRE)])
+                                               (256, "half", "bf16", POST), (256, "interleaved", "fp8", PRE),
+                                               (64, "half", "bf16", PRE), (64, "interleaved", "fp8", POST),
+                                               (256, "half", "bf16", PRE)])
 def test_fused_equals_two_calls_and_meets_the_oracle(d, style, elem, mode):
     wl = synth.WORKLOADS["single_layer_4k"].with_(name=f"fz{d}{style}", head_dim=d, rope_style=style, batch=6,
                                                   n_calib=64, theta=1e6 if d == 128 else 1e4)
