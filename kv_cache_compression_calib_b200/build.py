@@ -12,8 +12,11 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtri.so")
 
+BUILD_DIR = os.path.join(ROOT, "_build")
+
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-              "-Xcompiler", "-fPIC,-O2,-Wall", "-shared", "--expt-relaxed-constexpr"]
+              "-Xcompiler", "-fPIC,-O2,-Wall", "--expt-relaxed-constexpr"]
+LINK_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC"]
 
 
 def nvcc() -> str:
@@ -35,13 +38,27 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    cmd = [nvcc()] + NVCC_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp"] + sources()
+def _compile(src: str, obj: str, verbose: bool) -> None:
+    cmd = [nvcc()] + NVCC_FLAGS + ["-c", "-I", INCLUDE, "-I", CSRC, "-o", obj, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source file to an object in _build/ (in parallel: the files
+    share no device code, so no device link is needed), then link libtri.so."""
+    if not force and not _stale():
+        return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    srcs = sources()
+    objs = [os.path.join(BUILD_DIR, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        for f in [ex.submit(_compile, s, o, verbose) for s, o in zip(srcs, objs)]:
+            f.result()
+    subprocess.run([nvcc()] + LINK_FLAGS + ["-o", LIB + ".tmp"] + objs, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 
