@@ -22,7 +22,9 @@
 //     kept slot, ascending.  Every pass is bounded by the row's length, so a
 //     short row costs little.
 // Blocks never wait on other blocks.  Rows longer than kFusedMaxRow are not
-// processed here (flagged; the host routes such calls to the unfused kernels).
+// processed here: they are flagged and their kept entries set to -1 (the host
+// routes calls whose bound on the row length exceeds kFusedMaxRow to the
+// unfused kernels, so only a caller's understated bound gets here).
 #include "score_common.cuh"
 
 namespace tri {
@@ -89,6 +91,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
             atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
             if (fp.kept_count) fp.kept_count[r] = 0;
         }
+        // The row keeps nothing: every kept entry is marked empty (-1), so the
+        // gather that follows leaves the row's output records untouched.
+        for (int i = tid; i < B; i += kFThreads) out[i] = -1;
         return;
     }
     const int N = (int)N64;

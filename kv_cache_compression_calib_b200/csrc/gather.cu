@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
         pv[it] = 0;
         if (i >= cnt) continue;
         const int64_t j = p.kept[r * p.B + i];
+        if (j == -1) continue;  // an entry the fused kernel emptied (its row was flagged there)
         int64_t src = -1;
         if (j >= 0 && j < N) {
             if (geo.layout == TRI_KV_PAGED) {

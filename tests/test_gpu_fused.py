@@ -121,14 +121,19 @@ def test_fused_fallback_and_long_rows():
     Ko = torch.zeros(dev.n_rows, 2048, 128, dtype=torch.bfloat16, device=DEV)
     Vo = torch.zeros_like(Ko)
     cnt = torch.full((dev.n_rows,), -1, dtype=torch.int32, device=DEV)
+    kept = torch.full((dev.n_rows, 2048), 12345, dtype=torch.int32, device=DEV)
     tri.tri_score_compact(m, kv, dev.K, dev.V, None, torch.tensor(cs, dtype=torch.float32, device=DEV),
                           torch.tensor(ms, dtype=torch.float32, device=DEV), dev.p_now, wl.offsets, POST, 2048, 128,
-                          32768, tri.out_contig(), Ko, Vo, None, None, cnt, None, ws)
+                          32768, tri.out_contig(), Ko, Vo, None, kept, cnt, None, ws)
     st, flags = tri.tri_status_check(ws)
-    assert st == tri._abi.TRI_ERR_DEVICE_FLAG and flags & tri.TRI_FLAG_ROW_OFFSETS
+    assert st == tri._abi.TRI_ERR_DEVICE_FLAG and flags == tri.TRI_FLAG_ROW_OFFSETS
     c = cnt.cpu().numpy()
     assert np.all(c[:8] == 0) and np.all(c[8:] == 2048)
+    # the flagged rows keep nothing: kept entries emptied, output records untouched
+    assert np.all(kept[:8].cpu().numpy() == -1)
+    assert not Ko[:8].any() and not Vo[:8].any()
     np.testing.assert_array_equal(H.raw_bits(Ko[8:].cpu()), plain_rows(plain, 8))
+    np.testing.assert_array_equal(kept[8:].cpu().numpy(), plain["kept"][8:])
 
 
 def plain_rows(res, r0):
