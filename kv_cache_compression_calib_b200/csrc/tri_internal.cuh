@@ -16,15 +16,15 @@ namespace tri {
 constexpr int kMaxD = 256;            // largest supported head dim
 constexpr int kMaxF = kMaxD / 2;      // its frequency pairs
 constexpr int kCoefPerGroup = 24;     // 8 pairs x (Re A, Im A, c)
-inline int coef_per_row(int D) { return (D / 16) * kCoefPerGroup; }  // 3 floats per pair
+constexpr int coef_per_row(int D) { return (D / 16) * kCoefPerGroup; }  // 3 floats per pair
 
 // Workspace layout (byte offsets from the 256-byte aligned base).
 constexpr size_t kWsFlags = 0;       // uint32 flag word
 constexpr size_t kWsTurns = 256;     // uint64 [d/2 <= 128]: w_f / 2pi in 0.64 fixed point
 constexpr size_t kWsCoef = 1280;     // float [R][d/16][24]
-inline size_t ws_coef_bytes(int64_t R, int D) { return ((size_t)R * coef_per_row(D) * 4 + 255) & ~size_t(255); }
-inline size_t ws_idx_offset(int64_t R, int D) { return kWsCoef + ws_coef_bytes(R, D); }
-inline size_t ws_total(int64_t R, int64_t B, int D) {
+constexpr size_t ws_coef_bytes(int64_t R, int D) { return ((size_t)R * coef_per_row(D) * 4 + 255) & ~size_t(255); }
+constexpr size_t ws_idx_offset(int64_t R, int D) { return kWsCoef + ws_coef_bytes(R, D); }  // what tri_score needs
+constexpr size_t ws_total(int64_t R, int64_t B, int D) {
     return ws_idx_offset(R, D) + (((size_t)R * (size_t)B * 4 + 255) & ~size_t(255));
 }
 
