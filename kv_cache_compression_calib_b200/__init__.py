@@ -257,6 +257,37 @@ def tri_status_check(ws: torch.Tensor, stream=None):
     return st, int(flags.value)
 
 
+def tri_calib_save(path: str, m: TriModel, nq: int, centres: torch.Tensor, mean_norm: torch.Tensor) -> None:
+    """Write a calibration file (model shape, nq and the centres bit for bit).  The
+    centres may be on any device; they are copied to contiguous host float32
+    tensors for the call (the library reads host memory here)."""
+    c = centres.detach().to("cpu", torch.float32).contiguous()
+    n = mean_norm.detach().to("cpu", torch.float32).contiguous()
+    F = m.head_dim // 2
+    if c.numel() != m.n_layers * m.n_q_heads * F * 2 or n.numel() != m.n_layers * m.n_q_heads * F:
+        raise ValueError("centres / mean_norm do not match the model shape")
+    _check(_L.tri_calib_save(str(path).encode(), ctypes.byref(m), int(nq), ctypes.c_void_p(c.data_ptr()),
+                             ctypes.c_void_p(n.data_ptr())), "tri_calib_save")
+
+
+def tri_calib_load(path: str, device=None):
+    """Read a calibration file -> (model, nq, centres [L][Hq][d/2][2], mean_norm
+    [L][Hq][d/2]) as float32 tensors on `device` (host when None)."""
+    m = TriModel()
+    nq = ctypes.c_int64(0)
+    _check(_L.tri_calib_load(str(path).encode(), ctypes.byref(m), ctypes.byref(nq), None, None, 0),
+           "tri_calib_load (header)")
+    F = m.head_dim // 2
+    c = torch.empty(m.n_layers, m.n_q_heads, F, 2, dtype=torch.float32)
+    n = torch.empty(m.n_layers, m.n_q_heads, F, dtype=torch.float32)
+    m2 = TriModel()
+    _check(_L.tri_calib_load(str(path).encode(), ctypes.byref(m2), ctypes.byref(nq), ctypes.c_void_p(c.data_ptr()),
+                             ctypes.c_void_p(n.data_ptr()), n.numel()), "tri_calib_load")
+    if device is not None:
+        c, n = c.to(device), n.to(device)
+    return m2, int(nq.value), c, n
+
+
 def tri_selftest_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
     """Enqueue the self-test of the staged kernels' bounded wait: one warp waits
     `limit_ns` on a barrier nothing completes and sets TRI_FLAG_STAGE_TIMEOUT

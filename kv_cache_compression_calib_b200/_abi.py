@@ -14,6 +14,7 @@ TRI_ERR_ALIGNMENT = 3
 TRI_ERR_WORKSPACE_TOO_SMALL = 4
 TRI_ERR_CUDA = 5
 TRI_ERR_DEVICE_FLAG = 6
+TRI_ERR_IO = 7
 
 TRI_FLAG_ROW_OFFSETS = 0x1
 TRI_FLAG_NONFINITE = 0x2
@@ -34,10 +35,12 @@ TRI_KEYS_PRE_ROPE = 1
 EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_size", "tri_workspace_init", "tri_calib",
            "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc", "tri_calib_update",
            "tri_calib_stats", "tri_key_centres_ws_size", "tri_key_centres", "tri_attention_ws_size",
-           "tri_decode_attention", "tri_score_compact", "tri_selftest_wait_timeout")
+           "tri_decode_attention", "tri_score_compact", "tri_selftest_wait_timeout", "tri_calib_save",
+           "tri_calib_load")
 TRI_FUSED_MAX_ROW = 32768
 TRI_FUSED_PREFER_ROW = 8192
 TRI_NOALLOC_MAX_ROWS = 4096
+TRI_CALIB_FILE_VERSION = 1
 
 
 class TriModel(ctypes.Structure):
@@ -114,6 +117,11 @@ def load(path: str = LIB_PATH):
                               _P, _P, ctypes.c_size_t, _P]
     L.tri_status_check.restype = ctypes.c_int
     L.tri_status_check.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), _P]
+    L.tri_calib_save.restype = ctypes.c_int
+    L.tri_calib_save.argtypes = [ctypes.c_char_p, ctypes.POINTER(TriModel), ctypes.c_int64, _P, _P]
+    L.tri_calib_load.restype = ctypes.c_int
+    L.tri_calib_load.argtypes = [ctypes.c_char_p, ctypes.POINTER(TriModel), ctypes.POINTER(ctypes.c_int64), _P, _P,
+                                 ctypes.c_size_t]
     L.tri_selftest_wait_timeout.restype = ctypes.c_int
     L.tri_selftest_wait_timeout.argtypes = [_P, ctypes.c_size_t, ctypes.c_uint64, _P]
     L.tri_score_noalloc.restype = ctypes.c_int

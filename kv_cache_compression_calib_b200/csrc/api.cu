@@ -111,11 +111,12 @@ const char *tri_status_str(tri_status s) {
         case TRI_ERR_WORKSPACE_TOO_SMALL: return "TRI_ERR_WORKSPACE_TOO_SMALL";
         case TRI_ERR_CUDA: return "TRI_ERR_CUDA";
         case TRI_ERR_DEVICE_FLAG: return "TRI_ERR_DEVICE_FLAG";
+        case TRI_ERR_IO: return "TRI_ERR_IO";
     }
     return "TRI_ERR_UNKNOWN";
 }
 
-uint32_t tri_version(void) { return (0u << 16) | 2u; }
+uint32_t tri_version(void) { return (0u << 16) | 3u; }
 
 const char *tri_last_error(void) { return g_last_error; }
 
