@@ -54,7 +54,8 @@ typedef enum {
     TRI_ERR_ALIGNMENT = 3,           /* a pointer is not aligned as documented */
     TRI_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < tri_workspace_size(...) */
     TRI_ERR_CUDA = 5,                /* a CUDA launch or copy failed */
-    TRI_ERR_DEVICE_FLAG = 6          /* tri_status_check found a flag set by a kernel */
+    TRI_ERR_DEVICE_FLAG = 6,         /* tri_status_check found a flag set by a kernel */
+    TRI_ERR_IO = 7                   /* a file could not be opened, read or written, or is not a valid calibration file */
 } tri_status;
 
 /* Flag bits that kernels OR into the workspace flag word. */
@@ -134,7 +135,8 @@ typedef struct {
 const char *tri_status_str(tri_status s);
 
 /* Library version, (major << 16) | minor.  0.2: tri_model carries rope_style and
- * tri_kv_desc elem_type (both zero by default: rotate-half RoPE, bf16). */
+ * tri_kv_desc elem_type (both zero by default: rotate-half RoPE, bf16).  0.3:
+ * calibration files (tri_calib_save / tri_calib_load) and TRI_ERR_IO. */
 uint32_t tri_version(void);
 
 /* After a call returned TRI_ERR_CUDA: which CUDA call failed on this thread,
@@ -167,6 +169,41 @@ tri_status tri_workspace_init(void *ws, size_t ws_bytes, tri_stream_t stream);
  */
 tri_status tri_calib(const tri_model *m, const void *qpre, int64_t nq, float *centres,
                      float *mean_norm, tri_stream_t stream);
+
+/*
+ * Calibration artefact on disk (digest, 流程详解 step 1: the centres are
+ * computed offline, ahead of serving; 复现注意事项: they depend on the
+ * calibration data, so the file records the model shape and the number of
+ * queries per head that produced them).  HOST pointers: the caller copies the
+ * centres from or to the device (they are tri_calib's outputs and
+ * tri_score's inputs).  The file is a 64-byte little-endian header (magic
+ * "TRICALIB", format version TRI_CALIB_FILE_VERSION, header size, head_dim,
+ * n_layers, n_q_heads, n_kv_heads, rope_style, a zero word, rope_theta as
+ * binary64, nq, and the FNV-1a 64-bit hash of the payload) followed by the
+ * payload: centres then mean_norm as little-endian binary32, in tri_calib's
+ * layouts.  Values are stored bit for bit.
+ *
+ * tri_calib_save: writes (or replaces) `path`.
+ *   m, nq:     the model and the calibration queries per head (>= 1)
+ *   centres:   host float [n_layers][n_q_heads][d/2][2]
+ *   mean_norm: host float [n_layers][n_q_heads][d/2]
+ *   Returns TRI_ERR_INVALID_ARG for null pointers, nq < 1 or an invalid
+ *   model, TRI_ERR_IO if the file cannot be written.
+ *
+ * tri_calib_load: reads `path` into *m and *nq and, when centres and mean_norm
+ *   are not NULL, the payload into them (capacity_pairs = the number of
+ *   (layer, query head, pair) entries they hold; it must be at least
+ *   n_layers * n_q_heads * d/2 of the file, else TRI_ERR_WORKSPACE_TOO_SMALL).
+ *   With both NULL only the header is read and checked, so a caller can size
+ *   its buffers first.  A missing or unreadable file, a wrong magic, version or
+ *   header, an invalid model, a truncated or over-long payload or a hash
+ *   mismatch return TRI_ERR_IO; nothing is written to the outputs then.
+ */
+#define TRI_CALIB_FILE_VERSION 1
+tri_status tri_calib_save(const char *path, const tri_model *m, int64_t nq, const float *centres,
+                          const float *mean_norm);
+tri_status tri_calib_load(const char *path, tri_model *m, int64_t *nq, float *centres, float *mean_norm,
+                          size_t capacity_pairs);
 
 /*
  * Score every cached key (digest, 流程详解 steps 2-3) with the rule in the
@@ -303,7 +340,11 @@ tri_status tri_key_centres(const tri_model *m, const tri_kv_desc *kv, const void
  *     scores in shared memory, selects from there and writes the kept slots;
  *     K, V and pos are then gathered.  `scores`, when given, receives the
  *     scores; when NULL they never leave the chip.  A row longer than
- *     max_row_len sets TRI_FLAG_ROW_OFFSETS and keeps nothing.
+ *     TRI_FUSED_MAX_ROW keys (possible only when max_row_len understates the
+ *     longest row) sets TRI_FLAG_ROW_OFFSETS and keeps nothing: its kept_count
+ *     is 0, its kept_idx entries are -1 and its output records are left
+ *     untouched.  Rows longer than max_row_len but within TRI_FUSED_MAX_ROW
+ *     are processed normally.
  *   otherwise: exactly tri_score then tri_compact, `scores` (float
  *     [total_keys]) required.
  * Both ways give the same results bit for bit (the fused kernel runs the
@@ -363,9 +404,11 @@ tri_status tri_decode_attention(const tri_model *m, const tri_kv_desc *kv, const
  * (n_layers * n_seqs * n_kv_heads); more rows return
  * TRI_ERR_WORKSPACE_TOO_SMALL before anything is launched.  The call
  * allocates nothing.
- *  - The first call on each device looks up the scratch's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture on the device.
+ *  - Each call made outside a stream capture looks up the scratch's device
+ *    address (cudaGetSymbolAddress) with the calling device current; a call
+ *    made while `stream` is being captured reuses the last address found on
+ *    that device.  Make the first call on each device before any stream
+ *    capture there, and again after a cudaDeviceReset.
  *  - All calls on a device share the one scratch array: calls whose kernels
  *    can overlap on the GPU (other streams, other threads) race and must be
  *    serialised by the caller.
