@@ -7,7 +7,7 @@ layer), inputs resident in HBM (larger than L2).  Calibration (tri_calib) is
 offline and timed separately.  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload qwen3_8b_32k] [--budget B] [--key-mode post|pre]
+                  [--workload qwen3_32b_128k] [--also qwen3_8b_32k|none] [--budget B] [--key-mode post|pre]
                   [--elem bf16|fp8] [--head-dim 64|128|256] [--rope half|interleaved]
 
 N > 1 (under torchrun): every rank compacts its own cache of the same shape
@@ -44,7 +44,7 @@ ELEM_BYTES = {"bf16": 2, "fp8": 1}
 
 
 def score_bytes_per_key(eb: int, d: int = 128) -> int:
-    return d * eb + 4  # read the key, write its fp32 score
+    return d * eb  # read the key (the fp32 score write is overhead: it shows in the measured traffic)
 
 
 def kept_bytes(eb: int, d: int = 128) -> int:
@@ -57,7 +57,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen3_8b_32k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="qwen3_32b_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--also", default="qwen3_8b_32k", choices=sorted(synth.WORKLOADS) + ["none"],
+                    help="a second workload timed in the same run (step timing only), reported under 'also'; "
+                         "skipped with --layers, --budget or when it equals --workload")
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--layers", type=int, default=None,
                     help="first N layers only (small cases for profiling; not a bench line)")
@@ -229,13 +232,15 @@ def throughput(keys_per_rank: int, world: int, ms_per_step: float) -> float:
 
 # ----------------------------------------------------------------- ours
 
-def run_ours(a, rank, world, local_rank):
+def run_ours(a, rank, world, local_rank, workload=None, light=False):
+    """One workload's bench line.  light: the step timing only (no end-to-end leg,
+    CPU baseline or off-step diagnostics), for the extra workload of a run."""
     import kv_cache_compression_calib_b200 as tri
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl0 = synth.WORKLOADS[a.workload]
-    B = a.budget or wl0.budget
+    wl0 = synth.WORKLOADS[workload or a.workload]
+    B = (a.budget if not light else None) or wl0.budget
     if a.layers:
         wl0 = wl0.with_(n_layers=min(a.layers, wl0.n_layers))
     wl0 = with_layout(wl0, a)
@@ -354,15 +359,20 @@ def run_ours(a, rank, world, local_rank):
     ms_step = ms / a.steps
     value = throughput(keys_step, world, ms_step)
 
-    diagnostics = time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream)
-    diagnostics.update(time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream))
+    diagnostics = {}
+    if not light:
+        diagnostics = time_diagnostics(tri, m, kv, cache, key_mode, wl, eb, dev, stream)
+        diagnostics.update(time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream))
 
     # ---- end to end through the public API: pinned host inputs, copies in the region
     e2e = None
-    if not a.no_e2e:
-        e2e = run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream,
-                      world, dev, max_row if fused else None)
+    if not a.no_e2e and not light:
+        e2e = run_e2e(a, tri, cache, centres, mnorm, key_mode, B, wl, stream, world, dev)
 
+    # prep + score + select (the selection kernel copies the records itself when rows
+    # average more than one 32768-slot chunk, else a gather kernel follows); fused:
+    # prep + fused score/select + gather
+    launches_per_step = 3 if fused or total > cache.n_rows * 32768 else 4
     peak, peak_kind = measured_peak()
     if fused:  # one call per step: its roofline is the whole path's
         score_bytes = alg_bytes
@@ -371,7 +381,8 @@ def run_ours(a, rank, world, local_rank):
     else:
         score_bytes = score_bytes_per_key(eb, D) * total
         kernel = "tri_score (prep + score kernels)"
-        traffic = recorded_traffic(total, a.elem) if (D, wl.rope_style) == (128, "half") else None
+        traffic = (recorded_traffic(total, a.elem) if (D, wl.rope_style, a.key_mode) == (128, "half", "post")
+                   else None)
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     path_gbs = alg_bytes / (ms_step / 1e3) / 1e9
     line = {
@@ -386,14 +397,21 @@ def run_ours(a, rank, world, local_rank):
                           "frac_of_measured": path_gbs / peak, "frac_of_8tbs": path_gbs / NOMINAL_HBM_GBS},
         "calib_ms": calib_ms,
         "diagnostics": diagnostics,
-        "gpu_launches": (3 if fused else 4) * a.steps,
+        "gpu_launches": launches_per_step * a.steps,
         "path": "fused" if fused else "split",
         "clocks": clocks,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and not light:
         line["cpu_baseline"] = cpu_baseline(wl, B, cache, a.cpu_seconds)
     return line
+
+
+def also_summary(line):
+    """The step figures of an extra workload's line (same clock, same run)."""
+    keep = ("value", "unit", "ms_per_step", "steps", "config", "roofline", "path_roofline", "clocks",
+            "gpu_launches", "path")
+    return {k: line[k] for k in keep if k in line}
 
 
 def run_paged(a, tri, wl, B, rank, world, dev):
@@ -540,7 +558,7 @@ def run_paged(a, tri, wl, B, rank, world, dev):
                           "frac_of_8tbs": alg_bytes / (ms_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
                           "round0_ms": r0_ms, "round_ms": r1_ms,
                           "round_frac_of_measured": bytes1 / (r1_ms / 1e3) / 1e9 / peak},
-        "gpu_launches": (3 if fused else 4) * (1 + wl.rounds) * a.steps,
+        "gpu_launches": 3 * (1 + wl.rounds) * a.steps,
         "clocks": clocks,
         "e2e": None,
         "path": "fused" if fused else "split",
@@ -627,68 +645,103 @@ def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
             if R * B * 2 * D * eb < 100e6 else "compacted K+V larger than L2"}
 
 
-def run_e2e(a, tri, m, kv, cache, centres, mnorm, scores, Ko, Vo, po, kept, ws, key_mode, B, wl, stream, world,
-            dev, fused_max_row=None):
-    """End to end through the public calls with the cache on the host: every step
-    copies K, pos, the row offsets, p_now and the centres from pinned host memory,
-    scores and compacts, with V and the compacted outputs left in pinned host memory
-    (the gather reads only the kept records of V over the link and writes the
-    compacted cache straight to the host), and reads the kept indices back."""
+HOST_CACHE_BYTES = 24 << 30  # pinned host memory the end-to-end leg may hold for the cache
+
+
+def run_e2e(a, tri, cache, centres, mnorm, key_mode, B, wl, stream, world, dev):
+    """End to end through the public calls with the cache on the host, streamed
+    layer by layer.  Every step, for every layer: K and the positions are copied
+    from pinned host memory into the layer's device region on a copy stream
+    (overlapping the previous layer's calls), then tri_score and tri_compact run
+    on the layer; the gather reads only the kept records of V from pinned host
+    memory and writes the compacted K, V and positions straight into pinned host
+    buffers; p_now is copied in at the start and the kept indices read back at
+    the end.  The calibration (offline, like the model's weights) stays on the
+    device.  The pinned host cache holds at most HOST_CACHE_BYTES of layers (the
+    host has far less RAM than a 128K cache): layer l streams from host layer
+    l mod h, so every byte of every layer still crosses the link each step."""
+    L, S, Hh, D = wl.n_layers, len(cache.lens), wl.n_kv_heads, wl.head_dim
+    rpl = S * Hh
+    ro = cache.row_off_np
+    eb = cache.K.element_size()
+    et = tri.elem_type_of(cache.K)
+    m1 = tri.model(1, wl.n_q_heads, Hh, wl.theta, head_dim=D,
+                   rope_style=tri.TRI_ROPE_INTERLEAVED if wl.interleaved else tri.TRI_ROPE_HALF)
+    spans = [(int(ro[l * rpl]), int(ro[(l + 1) * rpl])) for l in range(L)]
+    kvs = []
+    for l, (a0, a1) in enumerate(spans):
+        roff = torch.as_tensor(ro[l * rpl:(l + 1) * rpl + 1] - a0, device=dev)
+        kvs.append(tri.kv_contig(S, roff, a1 - a0, et))
+    layer_bytes = max(a1 - a0 for a0, a1 in spans) * (2 * D * eb + 4)
+    hl = int(max(1, min(L, HOST_CACHE_BYTES // max(layer_bytes, 1))))
     try:
-        hK = cache.K.cpu().pin_memory()
-        hV = cache.V.cpu().pin_memory()
-        hpos = cache.pos.cpu().pin_memory()
-        hro = cache.row_off.cpu().pin_memory()
+        hK, hV, hP = [], [], []
+        for a0, a1 in spans[:hl]:
+            for lst, src in ((hK, cache.K), (hV, cache.V), (hP, cache.pos)):
+                h = torch.empty(src[a0:a1].shape, dtype=src.dtype, pin_memory=True)
+                h.copy_(src[a0:a1])
+                lst.append(h)
+        oK = [torch.empty(rpl, B, D, dtype=cache.K.dtype, pin_memory=True) for _ in range(L)]
+        oV = [torch.empty(rpl, B, D, dtype=cache.K.dtype, pin_memory=True) for _ in range(L)]
+        oP = [torch.empty(rpl, B, dtype=torch.int32, pin_memory=True) for _ in range(L)]
         hpn = cache.p_now.cpu().pin_memory()
-        hc = centres.cpu().pin_memory()
-        hm = mnorm.cpu().pin_memory()
-        oK = torch.empty(Ko.shape, dtype=Ko.dtype).pin_memory()
-        oV = torch.empty(Vo.shape, dtype=Vo.dtype).pin_memory()
-        op = torch.empty(po.shape, dtype=po.dtype).pin_memory()
-        ok = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
+        kept = torch.empty(L * rpl, B, dtype=torch.int32, device=dev)
+        okept = torch.empty(kept.shape, dtype=kept.dtype, pin_memory=True)
     except RuntimeError as e:
         return {"value": None, "unit": UNIT, "skipped": f"pinned host buffers: {e}"[:200]}
-    ins = [(cache.K, hK), (cache.pos, hpos), (cache.row_off, hro), (cache.p_now, hpn), (centres, hc), (mnorm, hm)]
-    outs = [(ok, kept)]
-    lens = np.diff(np.asarray(cache.row_off_np, dtype=np.int64))
-    n_kept = int(np.minimum(lens, B).sum())
-    rb = Ko.shape[-1] * Ko.element_size()
-    # bytes over the host link: the copies, the kept V records read in place, and the
-    # compacted K, V and positions written in place
-    h2d = sum(h.numel() * h.element_size() for _, h in ins) + n_kept * rb
-    d2h = sum(h.numel() * h.element_size() for h, _ in outs) + n_kept * (2 * rb + 4)
-    steps = max(3, min(a.steps, 10))
+    scores = torch.empty(cache.total, dtype=torch.float32, device=dev)
+    ws = tri.alloc_workspace(m1, S, B, device=dev)
+    copy = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(L)]
+    done = [torch.cuda.Event() for _ in range(L)]
+    out_desc = tri.out_contig()
 
     def step():
-        for d, h in ins:
-            d.copy_(h, non_blocking=True)
-        if fused_max_row is not None:
-            tri.tri_score_compact(m, kv, cache.K, hV, cache.pos, centres, mnorm, cache.p_now, wl.offsets,
-                                  key_mode, B, wl.window, fused_max_row, tri.out_contig(), oK, oV, op, kept, None,
-                                  None, ws, stream)
-        else:
-            tri.tri_score(m, kv, cache.K, cache.pos, centres, mnorm, cache.p_now, wl.offsets, key_mode, scores, ws,
-                          stream)
-            tri.tri_compact(m, kv, scores, B, wl.window, cache.K, hV, cache.pos, tri.out_contig(), oK, oV, op,
-                            kept, None, ws, stream)
-        for h, d in outs:
-            h.copy_(d, non_blocking=True)
+        cache.p_now.copy_(hpn, non_blocking=True)
+        for l, (a0, a1) in enumerate(spans):
+            h = l % hl
+            with torch.cuda.stream(copy):
+                copy.wait_event(done[l])  # the previous step's calls on this layer are done
+                cache.K[a0:a1].copy_(hK[h], non_blocking=True)
+                cache.pos[a0:a1].copy_(hP[h], non_blocking=True)
+                ready[l].record(copy)
+            stream.wait_event(ready[l])
+            Kl, Pl = cache.K[a0:a1], cache.pos[a0:a1]
+            tri.tri_score(m1, kvs[l], Kl, Pl, centres[l:l + 1], mnorm[l:l + 1], cache.p_now, wl.offsets, key_mode,
+                          scores[a0:a1], ws, stream)
+            tri.tri_compact(m1, kvs[l], scores[a0:a1], B, wl.window, Kl, hV[h], Pl, out_desc, oK[l], oV[l], oP[l],
+                            kept[l * rpl:(l + 1) * rpl], None, ws, stream)
+            done[l].record(stream)
+        okept.copy_(kept, non_blocking=True)
 
-    for _ in range(2):
-        step()
+    lens = np.diff(np.asarray(ro, dtype=np.int64))
+    n_kept = int(np.minimum(lens, B).sum())
+    rb = D * eb
+    h2d = sum((a1 - a0) * (rb + 4) for a0, a1 in spans) + hpn.numel() * 8 + n_kept * rb
+    d2h = okept.numel() * 4 + n_kept * (2 * rb + 4)
+    est_s = h2d / 40e9
+    steps = max(2, min(a.steps, 10, int(8.0 / max(est_s, 1e-3))))
+    step()
     torch.cuda.synchronize()
+    st, flags = tri.tri_status_check(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device flags {flags:#x} in the end-to-end leg")
     if world > 1:
         torch.distributed.barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    copy.wait_event(t0)
     for _ in range(steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     return {"value": throughput(cache.total, world, ms / steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
-            "host_records": "V read and the compacted cache written in pinned host memory by the gather"}
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps, "copies_declared": True,
+            "host_cache": f"{hl} of {L} layers of K, V and positions in pinned host memory; layer l streams from "
+                          f"host layer l mod {hl}",
+            "host_records": "V read and the compacted cache written in pinned host memory by the gather",
+            "calls_per_step": f"tri_score + tri_compact per layer ({L} layers)"}
 
 
 # ------------------------------------------------------- CPU oracle leg
@@ -800,6 +853,12 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     try:
         line = run_ours(a, rank, world, local_rank)
+        if a.also != "none" and a.also != a.workload and not a.layers and not a.budget:
+            import gc
+
+            gc.collect()
+            torch.cuda.empty_cache()
+            line["also"] = also_summary(run_ours(a, rank, world, local_rank, workload=a.also, light=True))
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

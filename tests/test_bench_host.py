@@ -39,10 +39,34 @@ def test_clock_summary_short_region_and_empty():
 
 
 def test_algorithmic_bytes():
-    # read the key and write its fp32 score; K and V read and written per kept key, plus pos
-    assert bench.score_bytes_per_key(2, 128) == 260 and bench.score_bytes_per_key(1, 128) == 132
+    # scoring reads every key once (the fp32 score write is overhead, counted in the
+    # measured traffic, not in the algorithmic bytes); K and V read and written per
+    # kept key, plus its position read and written
+    assert bench.score_bytes_per_key(2, 128) == 256 and bench.score_bytes_per_key(1, 128) == 128
     assert bench.kept_bytes(2, 128) == 1032 and bench.kept_bytes(1, 64) == 264
-    assert bench.score_bytes_per_key(2, 256) == 516
+    assert bench.score_bytes_per_key(2, 256) == 512
+
+
+def test_default_line_is_the_largest_single_gpu_workload():
+    import sys
+    argv = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        a = bench.parse()
+    finally:
+        sys.argv = argv
+    assert a.workload == "qwen3_32b_128k" and a.also == "qwen3_8b_32k"
+    keys = {n: w.n_layers * w.batch * w.n_kv_heads * w.seq_len[1] for n, w in synth.WORKLOADS.items()
+            if w.layout == "contig" and not n.startswith("sweep")}
+    assert max(keys, key=keys.get) == a.workload
+
+
+def test_also_summary_keeps_the_step_figures():
+    line = {"value": 1.0, "unit": "keys/s", "ms_per_step": 0.5, "steps": 3, "config": {"workload": "x"},
+            "roofline": {}, "path_roofline": {}, "clocks": {}, "gpu_launches": 12, "path": "split",
+            "e2e": None, "diagnostics": {"a": 1}}
+    got = bench.also_summary(line)
+    assert "e2e" not in got and "diagnostics" not in got and got["value"] == 1.0
 
 
 def test_workload_overrides_and_rank_shards():
