@@ -236,7 +236,6 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
     sp.kept = kept;
     sp.kept_count = kept_count;
     sp.flags = (unsigned *)(w + kWsFlags);
-    if ((st = cuda_status(launch_select(sp, s), "select_kernel launch")) != TRI_OK) return st;
 
     GatherParams gp;
     std::memset(&gp, 0, sizeof(gp));
@@ -255,7 +254,7 @@ tri_status tri_compact(const tri_model *m, const tri_kv_desc *kv, const float *s
     gp.V_out = (char *)V_out;
     gp.pos_out = pos_out;
     gp.flags = sp.flags;
-    return cuda_status(launch_gather(gp, s), "gather_kernel launch");
+    return cuda_status(launch_select_gather(sp, gp, s), "select_kernel launch");
 }
 
 tri_status tri_calib_update(const tri_model *m, const void *qpre, int64_t nq, double decay, double *sums,
@@ -404,19 +403,17 @@ tri_status tri_score_compact(const tri_model *m, const tri_kv_desc *kv, const vo
     pp.n_off = n_offsets;
     pp.pre_rope = key_mode == TRI_KEYS_PRE_ROPE;
     for (int i = 0; i < n_offsets; i++) pp.offsets[i] = offsets[i];
-    pp.coef = (float *)(w + kWsCoef);
-    pp.turns = (unsigned long long *)(w + kWsTurns);
     pp.flags = (unsigned *)(w + kWsFlags);
-    if ((st = cuda_status(launch_prep(pp, s), "prep_kernel launch")) != TRI_OK) return st;
 
+    // No prep launch: every CTA of the fused kernel forms its own row's
+    // coefficients with the prep kernel's steps.
     FusedParams fp;
     std::memset(&fp, 0, sizeof(fp));
+    fp.pp = pp;
     fp.sp.geo = geo;
     fp.sp.K = (const char *)K;
     fp.sp.pos = pos;
     fp.sp.p_now = p_now;
-    fp.sp.coef = pp.coef;
-    fp.sp.turns = pp.turns;
     fp.sp.scores = scores;
     fp.sp.flags = pp.flags;
     fp.B = B;

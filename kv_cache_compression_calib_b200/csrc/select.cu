@@ -33,7 +33,7 @@
 // thr of the K-th best, then an in-order pass with one block scan of packed
 // (greater, equal) counts marks the keys above thr and the most recent ties.
 // Blocks never wait on other blocks.
-#include "tri_internal.cuh"
+#include "gather_chunk.cuh"
 
 namespace tri {
 
@@ -244,7 +244,276 @@ __device__ __forceinline__ void emit_bitmap(const uint32_t *bm_words, int64_t c0
     base += tot;
 }
 
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectParams p) {
+// All kept records of row r (cnt of them), moved by the whole CTA in chunks of
+// GatherChunk<RB, kSelThreads, 2>::kSlots slots (two K and two V vectors in flight per
+// thread: 64 KB per SM with two CTAs, within the select path's registers).
+template <int RB>
+__device__ __forceinline__ void gather_row(const GatherParams &g, int64_t r, int64_t row_lo, int64_t N, int cnt) {
+    using Chunk = GatherChunk<RB, kSelThreads, 2>;
+    for (int base = 0; base < cnt; base += Chunk::kSlots) Chunk::move(g, r, row_lo, N, cnt, base);
+}
+
+// ------------------------------------------------------------------ one pass
+//
+// Rows of more than one chunk and at most kOpMaxRow candidate slots first try
+// a single streaming pass (the general passes re-read a multi-chunk row, whose
+// scores no longer sit in L2, three times).  The value range of a sample (512 runs of 8 consecutive slots, evenly
+// spaced) sets the same clamped linear 2048-bin map as above; the sample's own
+// histogram gives a band of bins [b_lo, b_hi] that holds the K-th best key
+// unless the sample misleads by more than kOpZ standard deviations of a
+// binomial count (bins above b_hi hold fewer than pS - kOpZ sd sampled keys,
+// bins from b_lo up more than pS + kOpZ sd, p = K/M, S = 4096).  One pass over
+// the row then sets the keep-bit of every key above the band (bitmap words
+// assembled with shuffles, each written once) and appends the band's keys and
+// slots to a shared-memory list (one warp scan per 16 slots a thread reads);
+// the band is held as two fp32 values, so a slot costs three comparisons.  If the band did hold the
+// K-th best key (A keys above it, A <= K <= A + C with the C band keys all
+// held), the rest runs on chip: radix narrowing of the C keys to the exact
+// threshold key thr, keep-bits for keys above thr, tie-bits for keys equal to
+// it, the most recent ties chosen by a block scan in slot order, and the kept
+// slots emitted ascending by a block scan of the keep words.  Otherwise nothing
+// has been written and the general passes run.  The result is identical
+// either way: the band only decides which keys are resolved on chip.
+constexpr int kOpRuns = kSelThreads;             // sample runs, one per thread
+constexpr int kOpRun = 8;                        // consecutive slots per run
+constexpr int kOpSample = kOpRuns * kOpRun;      // 4096 sampled slots
+constexpr int64_t kOpMinRow = kChunk + 1;        // one-chunk rows: the general passes (from L2, cheaper)
+constexpr int64_t kOpMaxRow = 4 * kChunk;        // 131072 slots: the bitmaps' capacity
+constexpr int kOpWords = (int)(kOpMaxRow / 32);  // words per bitmap
+constexpr int kOpCand = 8192;                    // band keys held on chip
+constexpr float kOpZ = 5.f;                      // band half-width in binomial standard deviations
+constexpr int kOpUnroll = 4;                     // 16-byte loads in flight per thread
+constexpr size_t kSelDynSmem = (size_t)(2 * kOpWords + 2 * kOpCand) * sizeof(uint32_t);
+
+__device__ __forceinline__ bool one_pass_select(const float *sc, int M, uint32_t K, bool vec, int32_t *out,
+                                                unsigned *flags, uint32_t *dyn, uint32_t *hist, uint32_t *scan_sm,
+                                                uint32_t *sh_bin, uint32_t *sh_above, uint32_t *sh_count,
+                                                float *red_fa, float *red_fb, uint32_t *red_a, uint32_t *red_b) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t *keepw = dyn;                     // [kOpWords] keep-bits of the row
+    uint32_t *tiew = dyn + kOpWords;           // [kOpWords] keys equal to thr
+    uint32_t *cand_u = dyn + 2 * kOpWords;     // [kOpCand] band keys
+    uint32_t *cand_s = cand_u + kOpCand;       // [kOpCand] their slots
+    const int nwords = (M + 31) >> 5;
+
+    // Sample: run `tid` starts at slot (tid * M / 512) rounded down to a multiple
+    // of 8, and ends at most at M - 8 (M >= kOpMinRow).
+    const int r0 = (int)(((int64_t)tid * M / kOpRuns) & ~(int64_t)7);
+    float x[kOpRun];
+    float fmn = INFINITY, fmx = -INFINITY;
+    int snan = 0;
+#pragma unroll
+    for (int i = 0; i < kOpRun; i++) {
+        x[i] = __ldg(sc + r0 + i);
+        fmn = fminf(fmn, x[i]);
+        fmx = fmaxf(fmx, x[i]);
+        snan |= x[i] != x[i];
+    }
+    snan = __syncthreads_or(snan);
+    block_minmax(fmn, fmx, red_fa, red_fb);
+    BinMap bm;
+    const float vspan = fmx - fmn;
+    const float vlo = fmn - 0.0625f * vspan, vhi = fmx + 0.0625f * vspan;
+    bm.vmin = vlo;
+    bm.scale = vhi > vlo ? (float)kBins / (vhi - vlo) : 0.f;
+    bm.by_value = 1;
+    bm.lo = 0u;
+    bm.shift = 0;
+    if (snan || !isfinite(vspan) || !(vspan > 0.f) || !isfinite(vlo) || !isfinite(vhi) || !isfinite(bm.scale) ||
+        !(bm.scale > 0.f))
+        return false;  // no usable value range (block-uniform)
+
+    for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
+    for (int w = tid; w < nwords; w += kSelThreads) tiew[w] = 0u;
+    if (tid == 0) *sh_count = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kOpRun; i++) atomicAdd(&hist[bm(x[i])], 1u);
+    __syncthreads();
+    const float pk = (float)K / (float)M;
+    const float ps = pk * (float)kOpSample;
+    const float sd = sqrtf(ps * (1.f - pk));
+    const int r_hi = max(0, (int)floorf(ps - kOpZ * sd) - 1);        // sampled keys allowed above the band
+    const int r_lo = min(kOpSample, (int)ceilf(ps + kOpZ * sd) + 1);  // sampled keys from the band's low bin up
+    uint32_t b_hi = kBins - 1, b_lo, dummy;
+    if (r_hi > 0) find_bin(hist, (uint32_t)r_hi, scan_sm, sh_bin, sh_above, b_hi, dummy);
+    find_bin(hist, (uint32_t)r_lo, scan_sm, sh_bin, sh_above, b_lo, dummy);
+    // The band in value terms: T_hi = the largest sampled value in bin b_hi (no
+    // sampled value above it lies outside the bins above b_hi; +inf when nothing
+    // may be above), T_lo = the smallest sampled value in bin b_lo.  The map is
+    // monotone, so exactly the sampled keys of bins > b_hi exceed T_hi and those
+    // of bins >= b_lo are >= T_lo.  Comparisons in fp32 rank -0 with +0 and put
+    // NaN (every comparison false) below the band, as the order keys do.
+    float hmax = -INFINITY, lmin = INFINITY;
+#pragma unroll
+    for (int i = 0; i < kOpRun; i++) {
+        const int b = bm(x[i]);
+        if (b == (int)b_hi) hmax = fmaxf(hmax, x[i]);
+        if (b == (int)b_lo) lmin = fminf(lmin, x[i]);
+    }
+    block_minmax(lmin, hmax, red_fa, red_fb);
+    const float t_hi = r_hi > 0 ? hmax : INFINITY, t_lo = lmin;
+
+    // The pass: thread t takes slots 4v .. 4v+3 for v = k * 512 + t, kOpUnroll
+    // 16-byte loads in flight (4-byte loads when the row is not 16-byte aligned).
+    // Keep-bits of the keys above the band go to the bitmap; the band's slots of a
+    // group of kOpUnroll vectors are appended with one warp scan per group (their
+    // values are read again, from L1, when stored).
+    uint32_t above = 0;
+    int nan = 0;
+    const int nv = (M + 3) >> 2;
+    const int iters = (nv + kSelThreads - 1) / kSelThreads;
+    for (int k0 = 0; k0 < iters; k0 += kOpUnroll) {
+        float sv[kOpUnroll][4];
+#pragma unroll
+        for (int u = 0; u < kOpUnroll; u++) {
+            const int v = (k0 + u) * kSelThreads + tid;
+            if (vec && 4 * v + 3 < M) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(sc) + v);
+                sv[u][0] = f.x;
+                sv[u][1] = f.y;
+                sv[u][2] = f.z;
+                sv[u][3] = f.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; i++) sv[u][i] = 4 * v + i < M ? __ldg(sc + 4 * v + i) : 0.f;
+            }
+        }
+        uint32_t cmask = 0;  // bit 4u + i: slot 4 v_u + i lies in the band
+#pragma unroll
+        for (int u = 0; u < kOpUnroll; u++) {
+            const int v = (k0 + u) * kSelThreads + tid;
+            const int lim = M - 4 * v;  // valid slots of this vector (<= 0: none)
+            uint32_t nib = 0;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float sx = sv[u][i];
+                const bool valid = i < lim;
+                nib |= (uint32_t)(valid && sx > t_hi) << i;
+                cmask |= (uint32_t)(valid && sx >= t_lo && sx <= t_hi) << (4 * u + i);
+                nan |= valid && sx != sx;
+            }
+            above += __popc(nib);
+            uint32_t w = nib << (4 * (lane & 7));
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            w |= __shfl_xor_sync(0xffffffffu, w, 4);
+            if ((lane & 7) == 0 && lim > 0) keepw[v >> 3] = w;
+        }
+        const uint32_t c = __popc(cmask);
+        if (__ballot_sync(0xffffffffu, c != 0u)) {
+            uint32_t incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            uint32_t base = 0;
+            if (lane == 31) base = atomicAdd(sh_count, incl);
+            base = __shfl_sync(0xffffffffu, base, 31) + incl - c;
+            while (cmask) {
+                const int e = __ffs(cmask) - 1;
+                cmask &= cmask - 1;
+                const int j = 4 * ((k0 + (e >> 2)) * kSelThreads + tid) + (e & 3);
+                if (base < (uint32_t)kOpCand) {
+                    cand_u[base] = order_key(__ldg(sc + j));
+                    cand_s[base] = (uint32_t)j;
+                }
+                base++;
+            }
+        }
+    }
+    if (__syncthreads_or(nan) && tid == 0) atomicOr(flags, TRI_FLAG_NONFINITE);
+    uint32_t A;
+    block_exclusive_scan(above, scan_sm, &A);
+    const uint32_t C = *sh_count;
+    if (!(A <= K && A + C >= K && C <= (uint32_t)kOpCand)) return false;  // block-uniform
+
+    // The K - A best band keys: exact threshold key thr by radix narrowing over
+    // the band keys' range; need2 of the cand2 keys equal to thr are kept.
+    const uint32_t need = K - A;
+    uint32_t thr = 0xffffffffu, need2 = 0, cand2 = 0;
+    if (need > 0) {
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        for (int i = tid; i < (int)C; i += kSelThreads) {
+            lo = min(lo, cand_u[i]);
+            hi = max(hi, cand_u[i]);
+        }
+        block_minmax(lo, hi, red_a, red_b);
+        need2 = need;
+        cand2 = C;
+        for (;;) {
+            const uint32_t range = hi - lo;
+            if (range == 0) break;
+            const int nbits = 32 - __clz(range);
+            const int shift = nbits > 11 ? nbits - 11 : 0;
+            for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
+            __syncthreads();
+            for (int i = tid; i < (int)C; i += kSelThreads) {
+                const uint32_t u = cand_u[i];
+                if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> shift], 1u);
+            }
+            __syncthreads();
+            uint32_t b2, ab2;
+            find_bin(hist, need2, scan_sm, sh_bin, sh_above, b2, ab2);
+            need2 -= ab2;
+            cand2 = hist[b2];
+            const uint32_t nlo = lo + (b2 << shift);
+            const unsigned long long nhi = (unsigned long long)nlo + ((1ull << shift) - 1ull);
+            hi = nhi < (unsigned long long)hi ? (uint32_t)nhi : hi;
+            lo = nlo;
+            __syncthreads();
+            if (shift == 0) break;
+        }
+        thr = lo;
+        for (int i = tid; i < (int)C; i += kSelThreads) {
+            const uint32_t u = cand_u[i], j = cand_s[i];
+            if (u > thr) atomicOr(&keepw[j >> 5], 1u << (j & 31));
+            else if (u == thr) atomicOr(&tiew[j >> 5], 1u << (j & 31));
+        }
+    }
+    __syncthreads();
+
+    // Thread t owns words t*wpt .. t*wpt+wpt-1: keep the ties whose rank from the
+    // oldest is at least cand2 - need2, then emit the kept slots ascending.
+    const int wpt = (nwords + kSelThreads - 1) / kSelThreads;
+    const int w0 = tid * wpt;
+    uint32_t tcnt = 0;
+    for (int j = 0; j < wpt; j++)
+        if (w0 + j < nwords) tcnt += __popc(tiew[w0 + j]);
+    uint32_t ttot;
+    uint32_t trank = block_exclusive_scan(tcnt, scan_sm, &ttot);
+    const uint32_t tie_skip = cand2 - need2;
+    uint32_t kcnt = 0;
+    for (int j = 0; j < wpt; j++) {
+        if (w0 + j >= nwords) break;
+        uint32_t kw = keepw[w0 + j], tw = tiew[w0 + j];
+        while (tw) {
+            const int e = __ffs(tw) - 1;
+            tw &= tw - 1;
+            if (trank >= tie_skip) kw |= 1u << e;
+            trank++;
+        }
+        keepw[w0 + j] = kw;
+        kcnt += __popc(kw);
+    }
+    uint32_t ktot;
+    uint32_t o = block_exclusive_scan(kcnt, scan_sm, &ktot);
+    for (int j = 0; j < wpt; j++) {
+        if (w0 + j >= nwords) break;
+        uint32_t kw = keepw[w0 + j];
+        while (kw) {
+            const int e = __ffs(kw) - 1;
+            kw &= kw - 1;
+            if (o < K) out[o] = (w0 + j) * 32 + e;
+            o++;
+        }
+    }
+    return true;
+}
+
+template <bool GATHER>
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectParams p, const GatherParams g) {
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t bmw[kWords];  // keep-bitmap of the current chunk
     __shared__ uint32_t scan_sm[kSelWarps];
@@ -263,254 +532,302 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
     const int64_t N = p.geo.row_off[r + 1] - row_lo;
     const int32_t B = p.B, W = p.W;
     int32_t *out = p.kept + (int64_t)r * B;
-    if (N < 0 || N > 0x7fffffffLL || row_lo < 0 || row_lo + N > p.geo.total) {
-        if (tid == 0) {
-            atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
-            if (p.kept_count) p.kept_count[r] = 0;
+    // Selection (every exit is block-uniform and leaves the loop), then the
+    // row's kept records are copied by the same CTA: rows whose selection is
+    // latency-bound overlap other rows' copies, which keep HBM busy.
+    bool row_ok = true;
+    do {
+        if (N < 0 || N > 0x7fffffffLL || row_lo < 0 || row_lo + N > p.geo.total) {
+            if (tid == 0) {
+                atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
+                if (p.kept_count) p.kept_count[r] = 0;
+            }
+            row_ok = false;
+            break;
         }
-        return;
-    }
-    if (N <= B) {
-        for (int64_t i = tid; i < N; i += kSelThreads) out[i] = (int32_t)i;
-        if (tid == 0 && p.kept_count) p.kept_count[r] = (int32_t)N;
-        return;
-    }
-    const int64_t M = N - W;
-    const uint32_t K = (uint32_t)(B - W);
-    for (int i = tid; i < W; i += kSelThreads) out[K + i] = (int32_t)(M + i);
-    if (tid == 0 && p.kept_count) p.kept_count[r] = B;
-    if (K == 0) return;
-    const float *sc = p.scores + row_lo;
-    const bool vec = (((uintptr_t)sc) & 15) == 0;
-    const int nchunks = (int)((M + kChunk - 1) / kChunk);
-    if (tid == 0) {
-        sh_bin = 0;
-        sh_above = 0;
-        sh_count = 0;
-    }
+        if (N <= B) {
+            for (int64_t i = tid; i < N; i += kSelThreads) out[i] = (int32_t)i;
+            if (tid == 0 && p.kept_count) p.kept_count[r] = (int32_t)N;
+            break;
+        }
+        const int64_t M = N - W;
+        const uint32_t K = (uint32_t)(B - W);
+        for (int i = tid; i < W; i += kSelThreads) out[K + i] = (int32_t)(M + i);
+        if (tid == 0 && p.kept_count) p.kept_count[r] = B;
+        if (K == 0) break;
+        const float *sc = p.scores + row_lo;
+        const bool vec = (((uintptr_t)sc) & 15) == 0;
+        const int nchunks = (int)((M + kChunk - 1) / kChunk);
+        if (M >= kOpMinRow && M <= kOpMaxRow) {
+            extern __shared__ uint32_t sel_dyn[];
+            if (one_pass_select(sc, (int)M, K, vec, out, p.flags, sel_dyn, hist, scan_sm, &sh_bin, &sh_above, &sh_count,
+                                red_fa, red_fb, red_a, red_b))
+                break;
+            __syncthreads();  // every thread has read sh_count before it is cleared below
+        }
+        if (tid == 0) {
+            sh_bin = 0;
+            sh_above = 0;
+            sh_count = 0;
+        }
 
-    // Value range of an evenly spaced 1024-slot sample of the row, widened by
-    // 1/16 of its span on each side (two 4-byte loads per thread).
-    float fmn = INFINITY, fmx = -INFINITY;
-    int snan = 0;
-#pragma unroll
-    for (int k = 0; k < 2; k++) {
-        const int64_t j = ((int64_t)(2 * tid + k) * M) / (2 * kSelThreads);  // < M
-        const float s = __ldg(sc + j);
-        fmn = fminf(fmn, s);
-        fmx = fmaxf(fmx, s);
-        snan |= s != s;
-    }
-    const int any_snan = __syncthreads_or(snan);
-    block_minmax(fmn, fmx, red_fa, red_fb);
+        // Value range of an evenly spaced 1024-slot sample of the row, widened by
+        // 1/16 of its span on each side (two 4-byte loads per thread).
+        float fmn = INFINITY, fmx = -INFINITY;
+        int snan = 0;
+    #pragma unroll
+        for (int k = 0; k < 2; k++) {
+            const int64_t j = ((int64_t)(2 * tid + k) * M) / (2 * kSelThreads);  // < M
+            const float s = __ldg(sc + j);
+            fmn = fminf(fmn, s);
+            fmx = fmaxf(fmx, s);
+            snan |= s != s;
+        }
+        const int any_snan = __syncthreads_or(snan);
+        block_minmax(fmn, fmx, red_fa, red_fb);
 
-    BinMap bm;
-    const float vspan = fmx - fmn;
-    const float vlo = fmn - 0.0625f * vspan, vhi = fmx + 0.0625f * vspan;
-    bm.vmin = vlo;
-    bm.scale = vhi > vlo ? (float)kBins / (vhi - vlo) : 0.f;
-    bm.by_value = !any_snan && isfinite(vspan) && vspan > 0.f && isfinite(vlo) && isfinite(vhi) &&
-                  isfinite(bm.scale) && bm.scale > 0.f;
-    uint32_t umx = 0xffffffffu;
-    bm.lo = 0u;
-    bm.shift = 21;
-    if (!bm.by_value) {  // key-space bins over the row's key range
-        uint32_t umn = 0xffffffffu;
-        umx = 0u;
+        BinMap bm;
+        const float vspan = fmx - fmn;
+        const float vlo = fmn - 0.0625f * vspan, vhi = fmx + 0.0625f * vspan;
+        bm.vmin = vlo;
+        bm.scale = vhi > vlo ? (float)kBins / (vhi - vlo) : 0.f;
+        bm.by_value = !any_snan && isfinite(vspan) && vspan > 0.f && isfinite(vlo) && isfinite(vhi) &&
+                      isfinite(bm.scale) && bm.scale > 0.f;
+        uint32_t umx = 0xffffffffu;
+        bm.lo = 0u;
+        bm.shift = 21;
+        if (!bm.by_value) {  // key-space bins over the row's key range
+            uint32_t umn = 0xffffffffu;
+            umx = 0u;
+            for (int c = 0; c < nchunks; c++) {
+                const int64_t c0 = (int64_t)c * kChunk;
+                for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
+                    const uint32_t u = order_key(s);
+                    umn = min(umn, u);
+                    umx = max(umx, u);
+                });
+            }
+            block_minmax(umn, umx, red_a, red_b);
+            const uint32_t range = umx - umn;
+            const int nbits = range ? 32 - __clz(range) : 0;
+            bm.lo = umn;
+            bm.shift = nbits > 11 ? nbits - 11 : 0;
+        }
+
+        // Pass 1: histogram of the bins; b* and the keys above it.
+        for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
+        __syncthreads();
+        int nan = 0;
         for (int c = 0; c < nchunks; c++) {
             const int64_t c0 = (int64_t)c * kChunk;
             for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
-                const uint32_t u = order_key(s);
-                umn = min(umn, u);
-                umx = max(umx, u);
+                atomicAdd(&hist[bm(s)], 1u);
+                nan |= s != s;
             });
         }
-        block_minmax(umn, umx, red_a, red_b);
-        const uint32_t range = umx - umn;
-        const int nbits = range ? 32 - __clz(range) : 0;
-        bm.lo = umn;
-        bm.shift = nbits > 11 ? nbits - 11 : 0;
-    }
+        if (__syncthreads_or(nan) && tid == 0) atomicOr(p.flags, TRI_FLAG_NONFINITE);
+        uint32_t bin, above;
+        find_bin(hist, K, scan_sm, &sh_bin, &sh_above, bin, above);
+        const uint32_t need = K - above;  // keys to keep from b*
+        const uint32_t cand = hist[bin];  // keys in b*
+        const int ibin = (int)bin;
+        uint32_t out_base = 0;
 
-    // Pass 1: histogram of the bins; b* and the keys above it.
-    for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
-    __syncthreads();
-    int nan = 0;
-    for (int c = 0; c < nchunks; c++) {
-        const int64_t c0 = (int64_t)c * kChunk;
-        for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
-            atomicAdd(&hist[bm(s)], 1u);
-            nan |= s != s;
-        });
-    }
-    if (__syncthreads_or(nan) && tid == 0) atomicOr(p.flags, TRI_FLAG_NONFINITE);
-    uint32_t bin, above;
-    find_bin(hist, K, scan_sm, &sh_bin, &sh_above, bin, above);
-    const uint32_t need = K - above;  // keys to keep from b*
-    const uint32_t cand = hist[bin];  // keys in b*
-    const int ibin = (int)bin;
-    uint32_t out_base = 0;
-
-    if (cand <= (uint32_t)kCandMax) {
-        // Pass 2: gather b*'s members (and, for a one-chunk row, the bitmap of
-        // the higher bins on the same read).
-        for (int c = 0; c < nchunks; c++) {
-            const int64_t c0 = (int64_t)c * kChunk;
-            const int n = chunk_len(M, c0);
-            if (nchunks == 1) {
-                build_bitmap(sc, n, vec, bmw, [&](int j, float s) {
-                    const int b = bm(s);
-                    if (b == ibin) {
-                        const uint32_t i = atomicAdd(&sh_count, 1u);
-                        if (i < (uint32_t)kCandMax) {
-                            cand_key[i] = order_key(s);
-                            cand_slot[i] = j;
+        if (cand <= (uint32_t)kCandMax) {
+            // Pass 2: gather b*'s members (and, for a one-chunk row, the bitmap of
+            // the higher bins on the same read).
+            for (int c = 0; c < nchunks; c++) {
+                const int64_t c0 = (int64_t)c * kChunk;
+                const int n = chunk_len(M, c0);
+                if (nchunks == 1) {
+                    build_bitmap(sc, n, vec, bmw, [&](int j, float s) {
+                        const int b = bm(s);
+                        if (b == ibin) {
+                            const uint32_t i = atomicAdd(&sh_count, 1u);
+                            if (i < (uint32_t)kCandMax) {
+                                cand_key[i] = order_key(s);
+                                cand_slot[i] = j;
+                            }
                         }
-                    }
-                    return b > ibin;
-                });
-            } else {
-                for_each_score(sc + c0, n, vec, [&](int j, float s) {
-                    if (bm(s) == ibin) {
-                        const uint32_t i = atomicAdd(&sh_count, 1u);
-                        if (i < (uint32_t)kCandMax) {
-                            cand_key[i] = order_key(s);
-                            cand_slot[i] = c0 + j;
+                        return b > ibin;
+                    });
+                } else {
+                    for_each_score(sc + c0, n, vec, [&](int j, float s) {
+                        if (bm(s) == ibin) {
+                            const uint32_t i = atomicAdd(&sh_count, 1u);
+                            if (i < (uint32_t)kCandMax) {
+                                cand_key[i] = order_key(s);
+                                cand_slot[i] = c0 + j;
+                            }
                         }
-                    }
-                });
+                    });
+                }
             }
-        }
-        __syncthreads();
-        // Rank each member by (key desc, slot desc), 4 threads per member.
-        const int i = tid >> 2, q = tid & 3;
-        uint32_t rank = 0;
-        uint32_t ui = 0;
-        int64_t si = 0;
-        if (i < (int)cand) {
-            ui = cand_key[i];
-            si = cand_slot[i];
-            for (int j = q; j < (int)cand; j += 4) {
-                const uint32_t uj = cand_key[j];
-                rank += (uj > ui) | ((uj == ui) & (cand_slot[j] > si));
-            }
-        }
-        rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-        rank += __shfl_xor_sync(0xffffffffu, rank, 2);
-        if (i < (int)cand && q == 0) cand_keep[i] = rank < need;
-        __syncthreads();
-        for (int c = 0; c < nchunks; c++) {
-            const int64_t c0 = (int64_t)c * kChunk;
-            const int n = chunk_len(M, c0);
-            if (nchunks > 1) build_bitmap(sc + c0, n, vec, bmw, [&](int, float s) { return bm(s) > ibin; });
             __syncthreads();
-            if (tid < (int)cand && cand_keep[tid] && cand_slot[tid] >= c0 && cand_slot[tid] < c0 + n) {
-                const int j = (int)(cand_slot[tid] - c0);
-                atomicOr(&bmw[j >> 5], 1u << (j & 31));
+            // Rank each member by (key desc, slot desc), 4 threads per member.
+            const int i = tid >> 2, q = tid & 3;
+            uint32_t rank = 0;
+            uint32_t ui = 0;
+            int64_t si = 0;
+            if (i < (int)cand) {
+                ui = cand_key[i];
+                si = cand_slot[i];
+                for (int j = q; j < (int)cand; j += 4) {
+                    const uint32_t uj = cand_key[j];
+                    rank += (uj > ui) | ((uj == ui) & (cand_slot[j] > si));
+                }
             }
+            rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+            rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+            if (i < (int)cand && q == 0) cand_keep[i] = rank < need;
+            __syncthreads();
+            for (int c = 0; c < nchunks; c++) {
+                const int64_t c0 = (int64_t)c * kChunk;
+                const int n = chunk_len(M, c0);
+                if (nchunks > 1) build_bitmap(sc + c0, n, vec, bmw, [&](int, float s) { return bm(s) > ibin; });
+                __syncthreads();
+                if (tid < (int)cand && cand_keep[tid] && cand_slot[tid] >= c0 && cand_slot[tid] < c0 + n) {
+                    const int j = (int)(cand_slot[tid] - c0);
+                    atomicOr(&bmw[j >> 5], 1u << (j & 31));
+                }
+                __syncthreads();
+                emit_bitmap(bmw, c0, out, K, out_base, scan_sm);
+            }
+            break;
+        }
+
+        // Crowded b*: narrow in key space over its members, whose keys form the
+        // contiguous range [lo, hi], to the single key value thr.
+        uint32_t lo, hi;
+        if (bm.by_value) {
+            uint32_t cmn = 0xffffffffu, cmx = 0u;
+            for (int c = 0; c < nchunks; c++) {
+                const int64_t c0 = (int64_t)c * kChunk;
+                for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
+                    if (bm(s) == ibin) {
+                        const uint32_t u = order_key(s);
+                        cmn = min(cmn, u);
+                        cmx = max(cmx, u);
+                    }
+                });
+            }
+            block_minmax(cmn, cmx, red_a, red_b);
+            lo = cmn;
+            hi = cmx;
+        } else {
+            lo = bm.lo + (bin << bm.shift);
+            const unsigned long long h = (unsigned long long)lo + ((1ull << bm.shift) - 1ull);
+            hi = h < (unsigned long long)umx ? (uint32_t)h : umx;
+        }
+        uint32_t need2 = need, cand2 = cand;
+        for (;;) {
+            const uint32_t range = hi - lo;
+            if (range == 0) break;
+            const int nbits = 32 - __clz(range);
+            const int shift = nbits > 11 ? nbits - 11 : 0;
+            for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
+            __syncthreads();
+            for (int c = 0; c < nchunks; c++) {
+                const int64_t c0 = (int64_t)c * kChunk;
+                for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
+                    if (bm(s) == ibin) {
+                        const uint32_t u = order_key(s);
+                        if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> shift], 1u);
+                    }
+                });
+            }
+            __syncthreads();
+            uint32_t b2, ab2;
+            find_bin(hist, need2, scan_sm, &sh_bin, &sh_above, b2, ab2);
+            need2 -= ab2;
+            cand2 = hist[b2];
+            const uint32_t nlo = lo + (b2 << shift);
+            const unsigned long long nhi = (unsigned long long)nlo + ((1ull << shift) - 1ull);
+            hi = nhi < (unsigned long long)hi ? (uint32_t)nhi : hi;
+            lo = nlo;
+            __syncthreads();
+            if (shift == 0) break;
+        }
+        const uint32_t thr = lo;
+        const uint32_t tie_skip = cand2 - need2;  // ties at thr in the oldest slots are dropped
+        // In slot order (thread t: slots 64t .. 64t+63), mark the keys above thr and
+        // the ties whose rank from the oldest is at least tie_skip.
+        uint32_t tie_base = 0;
+        for (int c = 0; c < nchunks; c++) {
+            const int64_t c0 = (int64_t)c * kChunk;
+            const int n = chunk_len(M, c0);
+            const int j0 = tid * kItems;
+            unsigned long long gt_bits = 0, eq_bits = 0;
+            for (int e = 0; e < kItems; e++) {
+                const int j = j0 + e;
+                if (j < n) {
+                    const float s = __ldg(sc + c0 + j);
+                    const int b = bm(s);
+                    if (b > ibin) {
+                        gt_bits |= 1ull << e;
+                    } else if (b == ibin) {
+                        const uint32_t u = order_key(s);
+                        gt_bits |= (unsigned long long)(u > thr) << e;
+                        eq_bits |= (unsigned long long)(u == thr) << e;
+                    }
+                }
+            }
+            uint32_t tot;
+            uint32_t rank = tie_base + block_exclusive_scan((uint32_t)__popcll(eq_bits), scan_sm, &tot);
+            unsigned long long keep = gt_bits, eqs = eq_bits;
+            while (eqs) {
+                const int e = __ffsll((long long)eqs) - 1;
+                eqs &= eqs - 1;
+                if (rank >= tie_skip) keep |= 1ull << e;
+                rank++;
+            }
+            tie_base += tot;
+            bmw[2 * tid] = (uint32_t)keep;
+            bmw[2 * tid + 1] = (uint32_t)(keep >> 32);
             __syncthreads();
             emit_bitmap(bmw, c0, out, K, out_base, scan_sm);
         }
-        return;
-    }
-
-    // Crowded b*: narrow in key space over its members, whose keys form the
-    // contiguous range [lo, hi], to the single key value thr.
-    uint32_t lo, hi;
-    if (bm.by_value) {
-        uint32_t cmn = 0xffffffffu, cmx = 0u;
-        for (int c = 0; c < nchunks; c++) {
-            const int64_t c0 = (int64_t)c * kChunk;
-            for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
-                if (bm(s) == ibin) {
-                    const uint32_t u = order_key(s);
-                    cmn = min(cmn, u);
-                    cmx = max(cmx, u);
-                }
-            });
-        }
-        block_minmax(cmn, cmx, red_a, red_b);
-        lo = cmn;
-        hi = cmx;
-    } else {
-        lo = bm.lo + (bin << bm.shift);
-        const unsigned long long h = (unsigned long long)lo + ((1ull << bm.shift) - 1ull);
-        hi = h < (unsigned long long)umx ? (uint32_t)h : umx;
-    }
-    uint32_t need2 = need, cand2 = cand;
-    for (;;) {
-        const uint32_t range = hi - lo;
-        if (range == 0) break;
-        const int nbits = 32 - __clz(range);
-        const int shift = nbits > 11 ? nbits - 11 : 0;
-        for (int b = 0; b < kBinsPerThread; b++) hist[tid * kBinsPerThread + b] = 0u;
-        __syncthreads();
-        for (int c = 0; c < nchunks; c++) {
-            const int64_t c0 = (int64_t)c * kChunk;
-            for_each_score(sc + c0, chunk_len(M, c0), vec, [&](int, float s) {
-                if (bm(s) == ibin) {
-                    const uint32_t u = order_key(s);
-                    if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> shift], 1u);
-                }
-            });
-        }
-        __syncthreads();
-        uint32_t b2, ab2;
-        find_bin(hist, need2, scan_sm, &sh_bin, &sh_above, b2, ab2);
-        need2 -= ab2;
-        cand2 = hist[b2];
-        const uint32_t nlo = lo + (b2 << shift);
-        const unsigned long long nhi = (unsigned long long)nlo + ((1ull << shift) - 1ull);
-        hi = nhi < (unsigned long long)hi ? (uint32_t)nhi : hi;
-        lo = nlo;
-        __syncthreads();
-        if (shift == 0) break;
-    }
-    const uint32_t thr = lo;
-    const uint32_t tie_skip = cand2 - need2;  // ties at thr in the oldest slots are dropped
-    // In slot order (thread t: slots 64t .. 64t+63), mark the keys above thr and
-    // the ties whose rank from the oldest is at least tie_skip.
-    uint32_t tie_base = 0;
-    for (int c = 0; c < nchunks; c++) {
-        const int64_t c0 = (int64_t)c * kChunk;
-        const int n = chunk_len(M, c0);
-        const int j0 = tid * kItems;
-        unsigned long long gt_bits = 0, eq_bits = 0;
-        for (int e = 0; e < kItems; e++) {
-            const int j = j0 + e;
-            if (j < n) {
-                const float s = __ldg(sc + c0 + j);
-                const int b = bm(s);
-                if (b > ibin) {
-                    gt_bits |= 1ull << e;
-                } else if (b == ibin) {
-                    const uint32_t u = order_key(s);
-                    gt_bits |= (unsigned long long)(u > thr) << e;
-                    eq_bits |= (unsigned long long)(u == thr) << e;
-                }
-            }
-        }
-        uint32_t tot;
-        uint32_t rank = tie_base + block_exclusive_scan((uint32_t)__popcll(eq_bits), scan_sm, &tot);
-        unsigned long long keep = gt_bits, eqs = eq_bits;
-        while (eqs) {
-            const int e = __ffsll((long long)eqs) - 1;
-            eqs &= eqs - 1;
-            if (rank >= tie_skip) keep |= 1ull << e;
-            rank++;
-        }
-        tie_base += tot;
-        bmw[2 * tid] = (uint32_t)keep;
-        bmw[2 * tid + 1] = (uint32_t)(keep >> 32);
-        __syncthreads();
-        emit_bitmap(bmw, c0, out, K, out_base, scan_sm);
+    } while (0);
+    if (!GATHER || !row_ok) return;
+    __syncthreads();  // out[] of this row is complete and visible to the block
+    const int cnt = (int)(N < (int64_t)B ? N : (int64_t)B);
+    switch (g.geo.D * g.geo.elem_bytes) {
+        case 64: gather_row<64>(g, r, row_lo, N, cnt); break;
+        case 128: gather_row<128>(g, r, row_lo, N, cnt); break;
+        case 256: gather_row<256>(g, r, row_lo, N, cnt); break;
+        case 512: gather_row<512>(g, r, row_lo, N, cnt); break;
     }
 }
 
-cudaError_t launch_select(const SelectParams &p, cudaStream_t s) {
+template <bool GATHER>
+static cudaError_t launch_select_t(const SelectParams &p, const GatherParams &g, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
-    return launch_pdl(select_kernel, dim3((unsigned)R), dim3(kSelThreads), 0, s, p);
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr[dev & 63]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(select_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
+        if (e != cudaSuccess) return e;
+        attr[dev & 63] = true;
+    }
+    return launch_pdl(select_kernel<GATHER>, dim3((unsigned)R), dim3(kSelThreads), kSelDynSmem, s, p, g);
+}
+
+// Rows longer than one selection chunk on average: the selection kernel copies
+// its row's records itself (rows still selecting overlap rows already copying,
+// over several waves).  Shorter rows all select in one wave, where the gather
+// kernel, with more bytes in flight per thread, moves the records faster.  The
+// results are identical either way.
+cudaError_t launch_select_gather(const SelectParams &p, const GatherParams &g, cudaStream_t s) {
+    const int rb = g.geo.D * g.geo.elem_bytes;
+    if (rb != 64 && rb != 128 && rb != 256 && rb != 512) return cudaErrorInvalidValue;
+    const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
+    if (R > 0 && p.geo.total > R * kChunk) return launch_select_t<true>(p, g, s);
+    const cudaError_t e = launch_select_t<false>(p, g, s);
+    if (e != cudaSuccess) return e;
+    return launch_gather(g, s);
 }
 
 }  // namespace tri

@@ -144,7 +144,8 @@ struct AttnParams {
 constexpr int kFusedMaxRow = TRI_FUSED_MAX_ROW;  // longest row the fused score-and-select kernel holds on chip
 
 struct FusedParams {
-    ScoreParams sp;       // cache, coefficients, scores (may be null: kept on chip only)
+    PrepParams pp;        // calibration, positions, offsets: each CTA forms its row's coefficients
+    ScoreParams sp;       // cache, scores (may be null: kept on chip only)
     int32_t B, W;
     int32_t *kept;        // [R][B]
     int32_t *kept_count;  // [R] or null
@@ -158,7 +159,7 @@ cudaError_t launch_stats(const StatsParams &p, cudaStream_t s);
 cudaError_t launch_key_centres(const KeyCentreParams &p, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams &p, cudaStream_t s);
 cudaError_t launch_score(const ScoreParams &p, int pre_rope, cudaStream_t s);
-cudaError_t launch_select(const SelectParams &p, cudaStream_t s);
+cudaError_t launch_select_gather(const SelectParams &p, const GatherParams &g, cudaStream_t s);
 cudaError_t launch_gather(const GatherParams &p, cudaStream_t s);
 
 int sm_count();  // SMs of the current device (cached per device)
