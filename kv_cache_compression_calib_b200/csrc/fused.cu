@@ -25,6 +25,7 @@
 // processed here: they are flagged and their kept entries set to -1 (the host
 // routes calls whose bound on the row length exceeds kFusedMaxRow to the
 // unfused kernels, so only a caller's understated bound gets here).
+#include "coef.cuh"
 #include "score_common.cuh"
 
 namespace tri {
@@ -76,12 +77,19 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
     __shared__ uint32_t red_a[kFWarps], red_b[kFWarps];
     __shared__ uint32_t sh_bin, sh_above;
 
-    grid_dependency_wait();
-    grid_dependents_launch();
     const ScoreParams &p = fp.sp;
     const Geometry &geo = p.geo;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = blockIdx.x;
+    // The row's coefficients, step 1 (kernel parameters only) before the wait
+    // for the preceding kernel: threads tid < kPrepParts * F, as in the prep kernel.
+    constexpr int kCoefThreads = kPrepParts * F;
+    static_assert(kCoefThreads <= kFThreads, "the coefficient steps fit the block");
+    unsigned long long Tf = 0;
+    double osr = 0.0, osi = 0.0;
+    if (tid < kCoefThreads) coef_offsets<F>(fp.pp, tid % F, tid / F, Tf, osr, osi);
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int64_t lo = geo.row_off[r], hi = geo.row_off[r + 1];
     const int64_t N64 = hi - lo;
     const int32_t B = fp.B, W = fp.W;
@@ -100,16 +108,39 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
     const int M = N > B ? N - W : N;       // candidate slots (all slots when N <= B)
     const uint32_t K = N > B ? (uint32_t)(B - W) : 0u;
 
+    // Step 2 of the coefficients, staged in shared memory before the keys use it:
+    // partial sums in the histogram's space, the row's [d/16][24] coefficients and
+    // the T_f table at the start of the keys' space.
+    double(*part_re)[F] = reinterpret_cast<double(*)[F]>(hist);
+    double(*part_im)[F] = reinterpret_cast<double(*)[F]>(hist + 2 * kPrepParts * F);
+    float *coef_sm = reinterpret_cast<float *>(keys);
+    unsigned long long *turns_sm = reinterpret_cast<unsigned long long *>(keys + 3 * F);
+    if (tid < kCoefThreads) {
+        part_re[tid / F][tid % F] = osr;
+        part_im[tid / F][tid % F] = osi;
+    }
+    __syncthreads();
+    if (tid < F) {
+        coef_finish<F>(fp.pp, r, tid, Tf, part_re, part_im, coef_sm);
+        turns_sm[tid] = Tf;
+        if (r == 0 && tid == 0) {
+            const int64_t R = (int64_t)geo.L * geo.S * geo.H;
+            if (geo.row_off[0] != 0 || geo.row_off[R] != geo.total) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
+        }
+    }
+    __syncthreads();
+
     // ---- A. scores of the row into shared memory (and optionally global)
     const int q = lane / LPK, gl = lane % LPK;
     unsigned long long T[8];
 #pragma unroll
-    for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * gl + i] : 0ull;
+    for (int i = 0; i < 8; i++) T[i] = PRE ? turns_sm[8 * gl + i] : 0ull;
     float stc[8], sts[8];
     if (PRE) phasors(T, -(int64_t)NG, stc, sts);
     const unsigned long long pol = policy_evict_first();
     RowCtx c;
-    set_row(c, p, r, gl, LPK * kCoefPerGroup);
+    set_row_coef(c, p, r, gl, coef_sm + gl * kCoefPerGroup);
+    __syncthreads();  // the keys' space is rewritten below
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     int nan = 0;
     // Batches on the same grid as the score kernel's (multiples of KB in the

@@ -253,9 +253,9 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
             kc_stage_batch<St>(p, b0, (int)min((int64_t)KB, end - b0), ring, bar, t, pol);
         }
 
-    float fr[8], fi[8], fn[8];
+    unsigned long long fr2[4], fi2[4], fn2[4];  // fp32 runs, pairs (2k, 2k+1) packed
 #pragma unroll
-    for (int i = 0; i < 8; i++) fr[i] = fi[i] = fn[i] = 0.f;
+    for (int i = 0; i < 4; i++) fr2[i] = fi2[i] = fn2[i] = 0ull;
     // Adds the lanes' runs into this warp's columns: fp64 tree over the NG lanes
     // of each lane group, then lane group gl's column.
     auto fold = [&]() {
@@ -263,13 +263,14 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
         for (int c3 = 0; c3 < 3; c3++)
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                double v = (double)(c3 == 0 ? fr[i] : c3 == 1 ? fi[i] : fn[i]);
+                const float2 pr = f2split(c3 == 0 ? fr2[i >> 1] : c3 == 1 ? fi2[i >> 1] : fn2[i >> 1]);
+                double v = (double)((i & 1) ? pr.y : pr.x);
 #pragma unroll
                 for (int o = LPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
                 if (q == 0) acc[(c3 * 8 + i) * (W * LPK) + warp * LPK + gl] += v;
             }
 #pragma unroll
-        for (int i = 0; i < 8; i++) fr[i] = fi[i] = fn[i] = 0.f;
+        for (int i = 0; i < 4; i++) fr2[i] = fi2[i] = fn2[i] = 0ull;
     };
 
     int run = 0;
@@ -287,7 +288,6 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
         const int32_t *spos = reinterpret_cast<const int32_t *>(slot + St::KEY_BYTES);
         const int64_t a0 = b0 & ~int64_t(3);
         const int64_t a1 = POST ? min((b0 + nk + 3) & ~int64_t(3), geo.total & ~int64_t(3)) : 0;
-        KeyChunk<ELEM, IL, F> kc[U];
         int32_t kpos[U];
         bool valid[U];
 #pragma unroll
@@ -296,12 +296,7 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
             const int64_t k = b0 + idx;
             valid[u] = idx < nk;
             kpos[u] = 0;
-            if (valid[u]) {
-                kc[u].lds(slot + idx * RB, gl);
-                if (POST) kpos[u] = k < a1 ? spos[k - a0] : __ldg(p.pos + k);
-            } else {
-                kc[u].zero();
-            }
+            if (valid[u] && POST) kpos[u] = k < a1 ? spos[k - a0] : __ldg(p.pos + k);
         }
         float cs[8], sn[8];
         if (POST) phasors(T, (int64_t)kpos[0], cs, sn);
@@ -312,18 +307,26 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
                 else phasors(T, (int64_t)kpos[u], cs, sn);
             }
             if (!valid[u]) continue;
+            KeyChunk<ELEM, IL, F> kc;  // read from the slot as it is used
+            kc.lds(slot + (NG * u + q) * RB, gl);
             float x[8], y[8];
-            kc[u].unpack(x, y);
+            kc.unpack(x, y);
+            // Two pairs per packed instruction: the de-rotation by e^{-i w pos},
+            // the sums and the magnitudes.
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                float xr = x[i], xi = y[i];
+            for (int k2 = 0; k2 < 4; k2++) {
+                const unsigned long long X = f2(x[2 * k2], x[2 * k2 + 1]), Y = f2(y[2 * k2], y[2 * k2 + 1]);
+                unsigned long long XR = X, XI = Y;
                 if (POST) {
-                    xr = x[i] * cs[i] + y[i] * sn[i];
-                    xi = y[i] * cs[i] - x[i] * sn[i];
+                    const unsigned long long CS = f2(cs[2 * k2], cs[2 * k2 + 1]);
+                    const unsigned long long SN = f2(sn[2 * k2], sn[2 * k2 + 1]);
+                    XR = fma2(X, CS, mul2(Y, SN));   // x cs + y sn
+                    XI = fma2(Y, CS, mul2(X, neg2(SN)));  // y cs - x sn
                 }
-                fr[i] += xr;
-                fi[i] += xi;
-                fn[i] += sqrt_approx(fmaf(x[i], x[i], y[i] * y[i]));
+                fr2[k2] = add2(fr2[k2], XR);
+                fi2[k2] = add2(fi2[k2], XI);
+                const float2 qq = f2split(fma2(X, X, mul2(Y, Y)));
+                fn2[k2] = add2(fn2[k2], f2(sqrt_approx(qq.x), sqrt_approx(qq.y)));
             }
         }
         if (t + STAGES < nbw) {  // the slot's bytes are consumed: refill it

@@ -287,18 +287,17 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE) ? 3 : 2) sc
         }
         float part[U];
         if (bend == b0 + KB && b0 >= c.lo && bend <= c.hi) {
-            // Whole batch inside the current row (npos = KB when positions were staged).
-            KeyChunk<ELEM, IL, F> kc[U];
+            // Whole batch inside the current row (npos = KB when positions were staged):
+            // each key is read from the slot as it is scored.
             int32_t kpos[U];
-            bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; u++) {
                 const int idx = NG * u + q;
-                kc[u].lds(slot + idx * RB, gl);
                 kpos[u] = PRE ? (pos_bulk ? spos[idx] : __ldg(p.pos + b0 + idx)) : 0;
-                ok[u] = true;
             }
-            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, stc, sts, part);
+            batch_partials_lazy<PRE, U, NG, KeyChunk<ELEM, IL, F>>(
+                [&](int u, KeyChunk<ELEM, IL, F> &kc) { kc.lds(slot + (NG * u + q) * RB, gl); }, kpos, c, T, stc,
+                sts, part);
         } else {
             // Batch crosses a row boundary or the span end: one segment per row,
             // each key read from the slot as it is scored.

@@ -18,7 +18,9 @@ struct RowCtx {
     float ar[8], ai[8], cc[8];
 };
 
-__device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, int gl, int coef_per_row) {
+// Row context of row r with lane group gl's 24 coefficients at `cg` (global or
+// shared memory, 16-byte aligned).
+__device__ __forceinline__ void set_row_coef(RowCtx &c, const ScoreParams &p, int r, int gl, const float *cg) {
     const Geometry &geo = p.geo;
     c.r = r;
     c.lo = geo.row_off[r];
@@ -30,7 +32,7 @@ __device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, 
     c.table = geo.block_table + (int64_t)s * geo.max_blocks;
     c.layer_blk = (int64_t)l * geo.n_blocks;
     c.p_now = p.p_now[s];
-    const float4 *cp = reinterpret_cast<const float4 *>(p.coef + (int64_t)r * coef_per_row + gl * kCoefPerGroup);
+    const float4 *cp = reinterpret_cast<const float4 *>(cg);
     const float4 v0 = cp[0], v1 = cp[1], v2 = cp[2], v3 = cp[3], v4 = cp[4], v5 = cp[5];
     c.ar[0] = v0.x; c.ar[1] = v0.y; c.ar[2] = v0.z; c.ar[3] = v0.w;
     c.ar[4] = v1.x; c.ar[5] = v1.y; c.ar[6] = v1.z; c.ar[7] = v1.w;
@@ -38,6 +40,10 @@ __device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, 
     c.ai[4] = v3.x; c.ai[5] = v3.y; c.ai[6] = v3.z; c.ai[7] = v3.w;
     c.cc[0] = v4.x; c.cc[1] = v4.y; c.cc[2] = v4.z; c.cc[3] = v4.w;
     c.cc[4] = v5.x; c.cc[5] = v5.y; c.cc[6] = v5.z; c.cc[7] = v5.w;
+}
+
+__device__ __forceinline__ void set_row(RowCtx &c, const ScoreParams &p, int r, int gl, int coef_per_row) {
+    set_row_coef(c, p, r, gl, p.coef + (int64_t)r * coef_per_row + gl * kCoefPerGroup);
 }
 
 // Slot index (in units of one (slot, head) record) of global key k in row c,
@@ -72,6 +78,13 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// Both lanes negated (sign bits flipped: exact).
+__device__ __forceinline__ unsigned long long neg2(unsigned long long a) { return a ^ 0x8000000080000000ull; }
 __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
     unsigned long long d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -178,6 +191,40 @@ __device__ __forceinline__ void batch_partials(const Chunk (&kc)[U], const int32
         float x[8], y[8];
         kc[u].unpack(x, y);
         part[u] = ok[u] ? partial_pre_rot(x, y, c, cs, sn) : 0.f;
+    }
+}
+
+// batch_partials for keys read as they are scored (from shared memory, where a
+// staged batch already sits), so no key waits in registers: load(u, chunk)
+// fetches key u.  The same arithmetic in the same order, so the same bits.
+template <bool PRE, int U, int NG, typename Chunk, typename Load>
+__device__ __forceinline__ void batch_partials_lazy(Load &&load, const int32_t (&kpos)[U], const RowCtx &c,
+                                                    const unsigned long long (&T)[8], const float (&stc)[8],
+                                                    const float (&sts)[8], float (&part)[U]) {
+    if (!PRE) {
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            Chunk kc;
+            load(u, kc);
+            float x[8], y[8];
+            kc.unpack(x, y);
+            part[u] = partial_post(x, y, c);
+        }
+        return;
+    }
+    float cs[8], sn[8];
+    phasors(T, c.p_now - (int64_t)kpos[0], cs, sn);
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+        if (u > 0) {
+            if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
+            else phasors(T, c.p_now - (int64_t)kpos[u], cs, sn);
+        }
+        Chunk kc;
+        load(u, kc);
+        float x[8], y[8];
+        kc.unpack(x, y);
+        part[u] = partial_pre_rot(x, y, c, cs, sn);
     }
 }
 
