@@ -638,11 +638,21 @@ def time_attention(tri, m, cache, Ko, Vo, wl, B, eb, dev, stream, reps=10):
         raise RuntimeError(f"device flags {flags:#x} in decode attention")
     nbytes = float(R) * B * 2 * D * eb + q.numel() * 2 + out.numel() * 4 + lse.numel() * 4
     peak, _ = measured_peak()
-    return {"decode_attention_ms": ms, "decode_attention_bytes": nbytes,
-            "decode_attention_gbs": nbytes / (ms / 1e3) / 1e9,
-            "decode_attention_frac": nbytes / (ms / 1e3) / 1e9 / peak,
-            "decode_attention_l2": "the compacted K+V (%.0f MB) fit in L2: timed warm" % (R * B * 2 * D * eb / 1e6)
-            if R * B * 2 * D * eb < 100e6 else "compacted K+V larger than L2"}
+    res = {"decode_attention_ms": ms, "decode_attention_bytes": nbytes,
+           "decode_attention_gbs": nbytes / (ms / 1e3) / 1e9,
+           "decode_attention_frac": nbytes / (ms / 1e3) / 1e9 / peak,
+           "decode_attention_l2": "the compacted K+V (%.0f MB) fit in L2: timed warm" % (R * B * 2 * D * eb / 1e6)
+           if R * B * 2 * D * eb < 100e6 else "compacted K+V larger than L2"}
+    if eb == 2 and D == 128 and wl.group <= 16:
+        # the tensor-memory kernel on the same cache and queries, timed beside it
+        ms_tc = graph_time(lambda s: tri.tri_decode_attention_tc(m, kvc, Ko, Vo, q, scale, out, lse, ws, s),
+                           stream, reps)
+        st, flags = tri.tri_status_check(ws, stream)
+        if st != 0:
+            raise RuntimeError(f"device flags {flags:#x} in tensor-memory decode attention")
+        res.update({"decode_attention_tc_ms": ms_tc,
+                    "decode_attention_tc_frac": nbytes / (ms_tc / 1e3) / 1e9 / peak})
+    return res
 
 
 HOST_CACHE_BYTES = 24 << 30  # pinned host memory the end-to-end leg may hold for the cache

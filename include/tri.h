@@ -391,6 +391,25 @@ tri_status tri_decode_attention(const tri_model *m, const tri_kv_desc *kv, const
                                 size_t ws_bytes, tri_stream_t stream);
 
 /*
+ * tri_decode_attention on the 5th-generation tensor cores: the same result
+ * (within fp32 rounding of a different summation order), for bf16 caches of
+ * head dim 128 in the contiguous layout with G <= 16 and total_keys < 2^31;
+ * anything else returns TRI_ERR_UNSUPPORTED before any launch.  Per 128-key
+ * tile the keys fill the M side of tcgen05.mma (S^T = K Q^T, then O^T = V^T P^T
+ * with the head dims on M, the queries padded to 16 columns on N), accumulators
+ * in tensor memory, K and V tiles brought by TMA; softmax, its maximum and sums
+ * as in tri_decode_attention.  On the workloads measured here it is slower than
+ * tri_decode_attention (one 4-warp CTA per SM keeps too few tiles in flight;
+ * the warp-level kernel runs 12 independent warps per SM), so
+ * tri_decode_attention does not use it.  Same arguments, workspace and flags;
+ * a copy or product that does not complete within 2 s sets
+ * TRI_FLAG_STAGE_TIMEOUT.
+ */
+tri_status tri_decode_attention_tc(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,
+                                   const void *q, float softmax_scale, float *out, float *lse, void *ws,
+                                   size_t ws_bytes, tri_stream_t stream);
+
+/*
  * tri_score without a workspace argument, for callers that cannot allocate
  * device memory where they score: code running inside another framework's
  * memory pool that forbids foreign allocations, plugins whose host process

@@ -237,6 +237,14 @@ def tri_decode_attention(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.T
            "tri_decode_attention")
 
 
+def tri_decode_attention_tc(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor,
+                            softmax_scale: float, out: torch.Tensor, lse, ws: torch.Tensor, stream=None) -> None:
+    """tri_decode_attention on the tensor-memory (tcgen05) kernel: bf16 contiguous caches, head dim 128, G <= 16."""
+    _check(_L.tri_decode_attention_tc(ctypes.byref(m), ctypes.byref(kv), _p(K), _p(V), _p(q), float(softmax_scale),
+                                      _p(out), _p(lse), _p(ws), ws.numel() * ws.element_size(), _s(stream)),
+           "tri_decode_attention_tc")
+
+
 def tri_score_compact(m: TriModel, kv: TriKvDesc, K: torch.Tensor, V: torch.Tensor, pos, centres: torch.Tensor,
                       mean_norm: torch.Tensor, p_now: torch.Tensor, offsets, key_mode: int, B: int, W: int,
                       max_row_len: int, out: TriOutDesc, K_out: torch.Tensor, V_out: torch.Tensor, pos_out,

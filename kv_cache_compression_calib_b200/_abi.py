@@ -36,7 +36,7 @@ EXPORTS = ("tri_status_str", "tri_version", "tri_last_error", "tri_workspace_siz
            "tri_score", "tri_compact", "tri_status_check", "tri_score_noalloc", "tri_calib_update",
            "tri_calib_stats", "tri_key_centres_ws_size", "tri_key_centres", "tri_attention_ws_size",
            "tri_decode_attention", "tri_score_compact", "tri_selftest_wait_timeout", "tri_calib_save",
-           "tri_calib_load")
+           "tri_calib_load", "tri_decode_attention_tc")
 TRI_FUSED_MAX_ROW = 32768
 TRI_FUSED_PREFER_ROW = 8192
 TRI_NOALLOC_MAX_ROWS = 4096
@@ -102,6 +102,8 @@ def load(path: str = LIB_PATH):
     L.tri_decode_attention.restype = ctypes.c_int
     L.tri_decode_attention.argtypes = [ctypes.POINTER(TriModel), ctypes.POINTER(TriKvDesc), _P, _P, _P,
                                        ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
+    L.tri_decode_attention_tc.restype = ctypes.c_int
+    L.tri_decode_attention_tc.argtypes = L.tri_decode_attention.argtypes
     L.tri_key_centres_ws_size.restype = ctypes.c_size_t
     L.tri_key_centres_ws_size.argtypes = [ctypes.POINTER(TriModel), ctypes.c_int32]
     L.tri_key_centres.restype = ctypes.c_int

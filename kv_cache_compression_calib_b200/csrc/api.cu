@@ -475,6 +475,37 @@ tri_status tri_decode_attention(const tri_model *m, const tri_kv_desc *kv, const
     return cuda_status(launch_attention(p, (cudaStream_t)stream), "attention kernel launch");
 }
 
+tri_status tri_decode_attention_tc(const tri_model *m, const tri_kv_desc *kv, const void *K, const void *V,
+                                   const void *q, float softmax_scale, float *out, float *lse, void *ws,
+                                   size_t ws_bytes, tri_stream_t stream) {
+    tri_status st = check_model(m);
+    if (st != TRI_OK) return st;
+    Geometry geo;
+    if ((st = check_kv(m, kv, &geo)) != TRI_OK) return st;
+    if (geo.G > 16 || geo.D != 128 || geo.elem_bytes != 2 || geo.layout != TRI_KV_CONTIG) return TRI_ERR_UNSUPPORTED;
+    if (kv->total_keys < 1 || kv->total_keys > 0x7fffffffLL) return TRI_ERR_UNSUPPORTED;
+    if (!K || !V || !q || !out) return TRI_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f)) return TRI_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(q, 2) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+        return TRI_ERR_ALIGNMENT;
+    if ((st = check_ws(ws, ws_bytes, tri_attention_ws_size(m, kv->n_seqs))) != TRI_OK) return st;
+    const int64_t R = rows_of(m, kv->n_seqs);
+    if (R * kAttnMaxChunks > 0x7fffffffLL || R * geo.G > 0x7fffffffLL) return TRI_ERR_UNSUPPORTED;
+    AttnParams p;
+    p.geo = geo;
+    p.K = (const char *)K;
+    p.V = (const char *)V;
+    p.q = (const uint16_t *)q;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.part = (float *)((char *)ws + 256);
+    p.out = out;
+    p.lse = lse;
+    p.flags = (unsigned *)((char *)ws + kWsFlags);
+    const cudaError_t e = launch_attention_tc(p, R, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return TRI_ERR_UNSUPPORTED;
+    return cuda_status(e, "tensor-memory attention kernel launch");
+}
+
 tri_status tri_status_check(void *ws, uint32_t *flags, tri_stream_t stream) {
     tri_status st = check_ws(ws, 256, 256);
     if (st != TRI_OK) return st;

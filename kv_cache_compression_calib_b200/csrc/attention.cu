@@ -778,15 +778,11 @@ cudaError_t launch_attn_combine(const AttnParams &p, int64_t R, cudaStream_t s) 
     return cudaGetLastError();
 }
 
-cudaError_t launch_attention_tc(const AttnParams &p, int64_t R, cudaStream_t s);
-
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
     if (R * kAttnMaxChunks > 0x7fffffffLL || R * p.geo.G > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    // bf16 contiguous caches of head dim 128: the tcgen05 kernel (attention_tc.cu).
-    const cudaError_t e = launch_attention_tc(p, R, s);
-    if (e != cudaErrorNotSupported) return e;
+
     const bool paged = p.geo.layout == TRI_KV_PAGED;
     if (p.geo.elem_bytes == 1) return paged ? launch_attn_d<1, true>(p, R, s) : launch_attn_d<1, false>(p, R, s);
     return paged ? launch_attn_d<2, true>(p, R, s) : launch_attn_d<2, false>(p, R, s);

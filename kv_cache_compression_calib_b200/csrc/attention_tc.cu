@@ -23,8 +23,8 @@
 // (~16-bit weights), per-thread fp32 partial sums rescaled as the maximum
 // grows.  The output of tile i is read from TMEM and added to the registers
 // while tile i+1 runs (O double-buffered), and the QK product of tile i+1 is
-// issued before tile i's softmax (S double-buffered); K tiles are fetched two
-// ahead, V tiles one ahead.  A persistent grid of one CTA per SM takes (row,
+// issued before tile i's softmax (S double-buffered); K and V tiles are fetched
+// up to three tiles ahead (three stages each).  A persistent grid of one CTA per SM takes (row,
 // slice) items in turn and writes each slice's unnormalised output, maximum and
 // sum; attn_combine_kernel merges a row's slices.  Every wait is bounded
 // (TRI_FLAG_STAGE_TIMEOUT); tensor memory is released before the CTA exits.
@@ -51,14 +51,22 @@ constexpr int kTcTileBytes = 2 * kTcBoxBytes;          // 32 KB: a K or V tile
 constexpr int kTcBBytes = kTcN * kTcD * 2;             // 4 KB: Q, or one P part
 constexpr int kTcTmemCols = 64;                        // S[2], O[2]: 16 columns each
 
+// P (a B operand, [16 queries][128 keys]) uses a padded core-matrix layout: the
+// core matrices of 8 keys are 144 bytes apart (not 128), so the four key groups a
+// warp's 32 lanes write for one query fall on different banks.
+constexpr int kPLbo = 144;               // between core matrices along the keys
+constexpr int kPSbo = 16 * kPLbo;        // between the two groups of 8 queries
+constexpr int kPBytes = 2 * kPSbo;       // one P part: 4608 bytes
+constexpr int kTcStages = 3;             // K and V tiles in flight per CTA
+
 // Shared memory, from a 1024-byte aligned base (swizzle atoms need it).
-constexpr int kSmK = 0;                                 // K tiles [2]
-constexpr int kSmV = kSmK + 2 * kTcTileBytes;           // V tiles [2]
-constexpr int kSmP = kSmV + 2 * kTcTileBytes;           // P [2 stages][hi, lo]
-constexpr int kSmQ = kSmP + 4 * kTcBBytes;              // Q
+constexpr int kSmK = 0;                                 // K tiles [kTcStages]
+constexpr int kSmV = kSmK + kTcStages * kTcTileBytes;   // V tiles [kTcStages]
+constexpr int kSmP = kSmV + kTcStages * kTcTileBytes;   // P [2 buffers][hi, lo]
+constexpr int kSmQ = kSmP + 4 * kPBytes;                // Q
 constexpr int kSmRed = kSmQ + kTcBBytes;                // float [16][4] per-warp reductions
-constexpr int kSmBar = kSmRed + kTcN * 4 * 4;           // 8 mbarriers
-constexpr int kSmTmem = kSmBar + 8 * 8;                 // allocated TMEM base
+constexpr int kSmBar = kSmRed + kTcN * 4 * 4;           // 10 mbarriers
+constexpr int kSmTmem = kSmBar + 10 * 8;                // allocated TMEM base
 constexpr int kSmAbort = kSmTmem + 4;                   // 1 after a wait ran out
 constexpr size_t kTcSmem = kSmAbort + 4 + 1024;         // + alignment slack
 
@@ -83,9 +91,9 @@ constexpr uint32_t kIdescQK = idesc_bf16(kTcKeys, kTcN, 0);
 constexpr uint32_t kIdescPV = idesc_bf16(kTcD, kTcN, 1);
 
 // K-major B operand without swizzle: core matrix (row group i of 8 rows, column
-// group j of 8 elements) at i * 2048 + j * 128 bytes, rows 16 bytes apart.
-__device__ __forceinline__ uint32_t b_core_offset(int row, int col) {
-    return (uint32_t)((row >> 3) * 2048 + (col >> 3) * 128 + (row & 7) * 16 + (col & 7) * 2);
+// group j of 8 elements) at i * sbo + j * lbo bytes, its rows 16 bytes apart.
+__device__ __forceinline__ uint32_t b_core_offset(int row, int col, int lbo = 128, int sbo = 2048) {
+    return (uint32_t)((row >> 3) * sbo + (col >> 3) * lbo + (row & 7) * 16 + (col & 7) * 2);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
@@ -135,17 +143,19 @@ __device__ __forceinline__ void tma_tile(unsigned char *dst, const CUtensorMap *
     tma_box(dst + kTcBoxBytes, map, kTcBoxDims, (int)key0, bar);
 }
 
-// Maximum (MAX = true) or sum over the warp of each of 16 values: a
-// reduce-scatter over lane bits 4..1, then bit 0.  Lane l ends with the result
-// for value index ((l >> 1) & 15), which is returned.
-template <bool MAX>
-__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
-    float a[16];
+// Maximum (MAX = true) or sum over the warp of each of the first N values (N =
+// 4, 8 or 16): a reduce-scatter over the top log2(N) lane bits (lane bit 16 >> s
+// decides which half of the remaining values a lane keeps at stage s), then
+// butterflies over the other lane bits.  Lane l ends with the result for value
+// index reduced_index<N>(l), which is returned.
+template <int N, bool MAX>
+__device__ __forceinline__ float warp_reduce(const float (&v)[16]) {
+    float a[N];
 #pragma unroll
-    for (int i = 0; i < 16; i++) a[i] = v[i];
+    for (int i = 0; i < N; i++) a[i] = v[i];
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int half = 8; half >= 1; half >>= 1) {
-        const int bit = half << 1;  // lane bit 16, 8, 4, 2 for half 8, 4, 2, 1
+    for (int half = N / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
         const bool up = (lane & bit) != 0;
 #pragma unroll
         for (int i = 0; i < half; i++) {
@@ -155,27 +165,68 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
             a[i] = MAX ? fmaxf(keep, other) : keep + other;
         }
     }
-    const float o = __shfl_xor_sync(0xffffffffu, a[0], 1);
-    return MAX ? fmaxf(a[0], o) : a[0] + o;
+#pragma unroll
+    for (int bit = 32 / N / 2; bit >= 1; bit >>= 1) {
+        const float o = __shfl_xor_sync(0xffffffffu, a[0], bit);
+        a[0] = MAX ? fmaxf(a[0], o) : a[0] + o;
+    }
+    return a[0];
 }
 
-// The value index lane l holds after warp_reduce16.
+template <int N>
 __device__ __forceinline__ int reduced_index(int lane) {
-    // Stage with half h keeps the upper half of the values when lane bit 2h is set.
-    return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+    int idx = 0;
+#pragma unroll
+    for (int half = N / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1)
+        if (lane & bit) idx += half;
+    return idx;
+}
+
+// Waits on bar[st] for the parity in bit st of ph (then flips that bit); false,
+// with the abort flag and TRI_FLAG_STAGE_TIMEOUT set, if the wait ran out.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t &ph, int st, volatile uint32_t *abort_flag,
+                                        unsigned *flags) {
+    const bool ok = mbar_wait(bar + st, (ph >> st) & 1u);
+    ph ^= 1u << st;
+    if (!ok) {
+        *abort_flag = 1u;
+        atomicOr(flags, TRI_FLAG_STAGE_TIMEOUT);
+    }
+    return ok;
+}
+
+// The QK product of a tile (one thread): K stage ks against Q, into TMEM
+// columns t_s, once the stage's copy has landed (bar_k[ks]); completion
+// arrives on bar_s[sb].
+__device__ __forceinline__ void tc_issue_qk(int ks, int sb, uint32_t sm_base, uint32_t t_s, uint64_t *bar_k,
+                                            uint64_t *bar_s, uint32_t &ph_k, volatile uint32_t *abort_flag,
+                                            unsigned *flags) {
+    if (!tc_wait(bar_k, ph_k, ks, abort_flag, flags)) return;
+    tc_fence_after();
+    const uint32_t kb = sm_base + kSmK + ks * kTcTileBytes;
+#pragma unroll
+    for (int k = 0; k < kTcD / 16; k++) {
+        const uint64_t a = smem_desc(kb + (k >> 2) * kTcBoxBytes + (k & 3) * 32, 16, 1024, 2);
+        const uint64_t b = smem_desc(sm_base + kSmQ + k * 256, 128, 2048, 0);
+        mma_bf16(t_s, a, b, kIdescQK, k > 0);
+    }
+    mma_commit(&bar_s[sb]);
 }
 
 }  // namespace
 
+// GQ: the query columns the softmax works on (4, 8 or 16; G <= GQ).  The MMAs
+// always run 16 columns; P rows GQ..15 stay zero.
+template <int GQ>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_partial_tc(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV) {
     extern __shared__ unsigned char smraw[];
     unsigned char *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
-    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + kSmBar);  // K tile landed [2]
-    uint64_t *bar_v = bar_k + 2;                                    // V tile landed [2]
-    uint64_t *bar_s = bar_k + 4;                                    // QK product done [2]
-    uint64_t *bar_o = bar_k + 6;                                    // PV product done [2]
+    uint64_t *bar_k = reinterpret_cast<uint64_t *>(sm + kSmBar);  // K tile landed [kTcStages]
+    uint64_t *bar_v = bar_k + kTcStages;                            // V tile landed [kTcStages]
+    uint64_t *bar_s = bar_v + kTcStages;                            // QK product done [2]
+    uint64_t *bar_o = bar_s + 2;                                    // PV product done [2]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSmTmem);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(sm + kSmAbort);
     float *red = reinterpret_cast<float *>(sm + kSmRed);  // [16][4]
@@ -184,10 +235,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
 
     if (t == 0) {
-        for (int i = 0; i < 8; i++) mbar_init(&bar_k[i], 1);
+        for (int i = 0; i < 2 * kTcStages + 4; i++) mbar_init(&bar_k[i], 1);
         mbar_init_fence();
         *abort_flag = 0u;
     }
+    // P rows of the padded queries are read by the PV products and must be zero.
+    for (int e = t; e < 4 * kPBytes / 16; e += kTcThreads)
+        reinterpret_cast<uint4 *>(sm + kSmP)[e] = make_uint4(0u, 0u, 0u, 0u);
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTcTmemCols)
@@ -200,25 +254,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tbase = *tmem_slot;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     // TMEM columns: S of stage st at tbase + 16 st, O of stage st at tbase + 32 + 16 st.
-    auto t_s = [&](int st) { return tbase + 16u * (uint32_t)st; };
-    auto t_o = [&](int st) { return tbase + 32u + 16u * (uint32_t)st; };
+#define t_s(st) (tbase + 16u * (uint32_t)(st))
+#define t_o(st) (tbase + 32u + 16u * (uint32_t)(st))
     // Parities of the next phase to wait for: bit st of each word, per barrier pair
     // (thread 0 alone waits on bar_k).
     uint32_t ph_k = 0u, ph_v = 0u, ph_s = 0u, ph_o = 0u;
     const uint32_t sm_base = smem_u32(sm);
     const int64_t n_items = (int64_t)geo.L * geo.S * geo.H * p.chunks;
-
-    // Waits on bar[st] for the parity in bit st of ph (then flips it); false (and
-    // the abort flag set) if it ran out.
-    auto wait = [&](uint64_t *bar, uint32_t &ph, int st) -> bool {
-        const bool ok = mbar_wait(bar + st, (ph >> st) & 1u);
-        ph ^= 1u << st;
-        if (!ok) {
-            *abort_flag = 1u;
-            atomicOr(p.flags, TRI_FLAG_STAGE_TIMEOUT);
-        }
-        return ok;
-    };
 
     for (int64_t item = blockIdx.x; item < n_items && !*abort_flag; item += gridDim.x) {
         const int64_t r = item / p.chunks;
@@ -267,47 +309,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
         // Prologue: K and V of tiles 0 and 1, then the QK product of tile 0.
         if (t == 0 && ntiles > 0) {
-            for (int j = 0; j < 2 && j < ntiles; j++) {
+            for (int j = 0; j < kTcStages && j < ntiles; j++) {
                 tma_tile(sm + kSmK + j * kTcTileBytes, &tmK, key0 + (int64_t)j * kTcKeys, &bar_k[j]);
                 tma_tile(sm + kSmV + j * kTcTileBytes, &tmV, key0 + (int64_t)j * kTcKeys, &bar_v[j]);
             }
         }
 
-        // The QK product of tile j (thread 0): K stage j % 2 against Q, into S[j % 2].
-        auto issue_qk = [&](int j) {
-            const int st = j & 1;
-            if (!wait(bar_k, ph_k, st)) return;
-            tc_fence_after();
-            const uint32_t kb = sm_base + kSmK + st * kTcTileBytes;
-#pragma unroll
-            for (int k = 0; k < kTcD / 16; k++) {
-                const uint64_t a = smem_desc(kb + (k >> 2) * kTcBoxBytes + (k & 3) * 32, 16, 1024, 2);
-                const uint64_t b = smem_desc(sm_base + kSmQ + k * 256, 128, 2048, 0);
-                mma_bf16(t_s(st), a, b, kIdescQK, k > 0);
-            }
-            mma_commit(&bar_s[st]);
-        };
-        if (t == 0 && ntiles > 0) issue_qk(0);
+        if (t == 0 && ntiles > 0) tc_issue_qk(0, 0, sm_base, t_s(0), bar_k, bar_s, ph_k, abort_flag, p.flags);
 
         for (int i = 0; i < ntiles; i++) {
-            const int st = i & 1;
-            if (t == 0 && i + 1 < ntiles) issue_qk(i + 1);
+            const int st = i & 1;          // S, O and P buffers
+            const int ks = i % kTcStages;  // K and V stages
+            if (t == 0 && i + 1 < ntiles)
+                tc_issue_qk((i + 1) % kTcStages, (i + 1) & 1, sm_base, t_s((i + 1) & 1), bar_k, bar_s, ph_k,
+                            abort_flag, p.flags);
             // ---- scores of tile i
-            wait(bar_s, ph_s, st);
+            tc_wait(bar_s, ph_s, st, abort_flag, p.flags);
             tc_fence_after();
-            if (t == 0 && i + 2 < ntiles)  // K stage st is free once the QK product of tile i is done
-                tma_tile(sm + kSmK + st * kTcTileBytes, &tmK, key0 + (int64_t)(i + 2) * kTcKeys, &bar_k[st]);
+            if (t == 0 && i + kTcStages < ntiles)  // K stage ks is free once the QK product of tile i is done
+                tma_tile(sm + kSmK + ks * kTcTileBytes, &tmK, key0 + (int64_t)(i + kTcStages) * kTcKeys, &bar_k[ks]);
             float x[16];
             tmem_ld16(t_s(st) + lane_off, x);
             const int64_t tile_beg = beg + (int64_t)i * kTcKeys;
             const int valid = (int)std::min<int64_t>(kTcKeys, end - tile_beg);
 #pragma unroll
-            for (int q = 0; q < 16; q++) x[q] = t < valid ? x[q] * p.scale_log2 : -INFINITY;
+            for (int q = 0; q < GQ; q++) x[q] = t < valid ? x[q] * p.scale_log2 : -INFINITY;
             // V of tile i has landed; the rows past the slice's end are zeroed (a
             // zero weight times whatever the box read there must give zero).
-            wait(bar_v, ph_v, st);
+            tc_wait(bar_v, ph_v, ks, abort_flag, p.flags);
             if (valid < kTcKeys && t >= valid) {
-                unsigned char *vrow = sm + kSmV + st * kTcTileBytes + t * 128;
+                unsigned char *vrow = sm + kSmV + ks * kTcTileBytes + t * 128;
 #pragma unroll
                 for (int b = 0; b < 2; b++)
 #pragma unroll
@@ -316,13 +347,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             // tile maximum of every query over the 128 keys
             {
-                const float wm = warp_reduce16<true>(x, lane);
-                if ((lane & 1) == 0) red[reduced_index(lane) * 4 + warp] = wm;
+                const float wm = warp_reduce<GQ, true>(x);
+                if ((lane & (32 / GQ - 1)) == 0) red[reduced_index<GQ>(lane) * 4 + warp] = wm;
             }
             __syncthreads();
             float pw[16];
 #pragma unroll
-            for (int q = 0; q < 16; q++) {
+            for (int q = 0; q < GQ; q++) {
                 const float4 mv = *reinterpret_cast<const float4 *>(red + q * 4);
                 const float tm = fmaxf(fmaxf(mv.x, mv.y), fmaxf(mv.z, mv.w));
                 const float mn = fmaxf(m_run[q], tm);
@@ -333,14 +364,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 x[q] = a;  // this tile's rescale factor, kept for its output
             }
             // P^T of tile i as bf16 hi + lo parts (B operands [16 queries][128 keys]).
-            unsigned char *ph = sm + kSmP + (2 * st) * kTcBBytes;
-            unsigned char *pl = ph + kTcBBytes;
+            unsigned char *ph = sm + kSmP + (2 * st) * kPBytes;
+            unsigned char *pl = ph + kPBytes;
 #pragma unroll
-            for (int q = 0; q < 16; q++) {
+            for (int q = 0; q < GQ; q++) {
                 const __nv_bfloat16 hb = __float2bfloat16_rn(pw[q]);
                 const __nv_bfloat16 lb = __float2bfloat16_rn(pw[q] - __bfloat162float(hb));
-                *reinterpret_cast<__nv_bfloat16 *>(ph + b_core_offset(q, t)) = hb;
-                *reinterpret_cast<__nv_bfloat16 *>(pl + b_core_offset(q, t)) = lb;
+                *reinterpret_cast<__nv_bfloat16 *>(ph + b_core_offset(q, t, kPLbo, kPSbo)) = hb;
+                *reinterpret_cast<__nv_bfloat16 *>(pl + b_core_offset(q, t, kPLbo, kPSbo)) = lb;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
@@ -350,14 +381,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             // ---- PV product of tile i into O[st] (fresh), hi then lo weights
             if (t == 0) {
-                const uint32_t vb = sm_base + kSmV + st * kTcTileBytes;
-                const uint32_t pb = sm_base + kSmP + (2 * st) * kTcBBytes;
+                const uint32_t vb = sm_base + kSmV + ks * kTcTileBytes;
+                const uint32_t pb = sm_base + kSmP + (2 * st) * kPBytes;
 #pragma unroll
                 for (int part = 0; part < 2; part++)
 #pragma unroll
                     for (int k = 0; k < kTcKeys / 16; k++) {
                         const uint64_t a = smem_desc(vb + k * 2048, kTcBoxBytes, 1024, 2);
-                        const uint64_t b = smem_desc(pb + part * kTcBBytes + k * 256, 128, 2048, 0);
+                        const uint64_t b = smem_desc(pb + part * kPBytes + k * 2 * kPLbo, kPLbo, kPSbo, 0);
                         mma_bf16(t_o(st), a, b, kIdescPV, part > 0 || k > 0);
                     }
                 mma_commit(&bar_o[st]);
@@ -365,34 +396,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // ---- output of tile i-1 (its PV product ran while this tile's scores were formed)
             if (i >= 1) {
                 const int sp = st ^ 1;
-                wait(bar_o, ph_o, sp);
+                tc_wait(bar_o, ph_o, sp, abort_flag, p.flags);
                 tc_fence_after();
-                if (t == 0 && i + 1 < ntiles)  // V stage sp is free once the PV product of tile i-1 is done
-                    tma_tile(sm + kSmV + sp * kTcTileBytes, &tmV, key0 + (int64_t)(i + 1) * kTcKeys, &bar_v[sp]);
+                // V stage (i-1) % kTcStages is free once the PV product of tile i-1 is
+                // done: it takes the tile kTcStages - 1 ahead of this one.
+                const int vs = (i - 1) % kTcStages;
+                if (t == 0 && i - 1 + kTcStages < ntiles)
+                    tma_tile(sm + kSmV + vs * kTcTileBytes, &tmV, key0 + (int64_t)(i - 1 + kTcStages) * kTcKeys,
+                             &bar_v[vs]);
                 float ot[16];
                 tmem_ld16(t_o(sp) + lane_off, ot);
 #pragma unroll
-                for (int q = 0; q < 16; q++) o_acc[q] = fmaf(o_acc[q], alpha_prev[q], ot[q]);
+                for (int q = 0; q < GQ; q++) o_acc[q] = fmaf(o_acc[q], alpha_prev[q], ot[q]);
             }
 #pragma unroll
-            for (int q = 0; q < 16; q++) alpha_prev[q] = x[q];
+            for (int q = 0; q < GQ; q++) alpha_prev[q] = x[q];
             tc_fence_before();
         }
         if (__syncthreads_or(*abort_flag)) break;
         // ---- the last tile's output, then (O, m, l) of queries < G
         if (ntiles > 0) {
             const int sp = (ntiles - 1) & 1;
-            wait(bar_o, ph_o, sp);
+            tc_wait(bar_o, ph_o, sp, abort_flag, p.flags);
             tc_fence_after();
             float ot[16];
             tmem_ld16(t_o(sp) + lane_off, ot);
 #pragma unroll
-            for (int q = 0; q < 16; q++) o_acc[q] = fmaf(o_acc[q], alpha_prev[q], ot[q]);
+            for (int q = 0; q < GQ; q++) o_acc[q] = fmaf(o_acc[q], alpha_prev[q], ot[q]);
         }
         {
-            const float ws = warp_reduce16<false>(l_part, lane);
+            const float ws = warp_reduce<GQ, false>(l_part);
             __syncthreads();  // red[] of the last tile maximum has been read
-            if ((lane & 1) == 0) red[reduced_index(lane) * 4 + warp] = ws;
+            if ((lane & (32 / GQ - 1)) == 0) red[reduced_index<GQ>(lane) * 4 + warp] = ws;
             __syncthreads();
         }
         float *out = p.part + item * (int64_t)G * (kTcD + 2);
@@ -409,9 +444,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // Teardown: after a wait ran out, give every copy and product still in flight
     // one more bounded wait, so nothing lands in memory that is released below.
     if (*abort_flag && t == 0) {
-        for (int b = 0; b < 2; b++) {
+        for (int b = 0; b < kTcStages; b++) {
             mbar_wait(&bar_k[b], (ph_k >> b) & 1u);
             mbar_wait(&bar_v[b], (ph_v >> b) & 1u);
+        }
+        for (int b = 0; b < 2; b++) {
             mbar_wait(&bar_s[b], (ph_s >> b) & 1u);
             mbar_wait(&bar_o[b], (ph_o >> b) & 1u);
         }
@@ -421,6 +458,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTcTmemCols) : "memory");
+#undef t_s
+#undef t_o
 }
 
 namespace {
@@ -464,13 +503,15 @@ cudaError_t launch_attention_tc(const AttnParams &p0, int64_t R, cudaStream_t s)
         return cudaErrorNotSupported;
     CUtensorMap mk, mv;
     if (!make_map(&mk, p0.K, geo.total) || !make_map(&mv, p0.V, geo.total)) return cudaErrorNotSupported;
-    static bool attr[64] = {false};
+    auto kern = geo.G <= 4 ? attn_partial_tc<4> : geo.G <= 8 ? attn_partial_tc<8> : attn_partial_tc<16>;
+    static bool attr[3][64] = {{false}};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!attr[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(attn_partial_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
+    const int ki = geo.G <= 4 ? 0 : geo.G <= 8 ? 1 : 2;
+    if (!attr[ki][dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
         if (e != cudaSuccess) return e;
-        attr[dev & 63] = true;
+        attr[ki][dev & 63] = true;
     }
     // Persistent grid, one CTA per SM; rows cut into slices so that every CTA
     // gets about four items (each slice costs (d + 2) G floats written and read back).
@@ -478,7 +519,7 @@ cudaError_t launch_attention_tc(const AttnParams &p0, int64_t R, cudaStream_t s)
     const int64_t ctas = sm_count();
     p.chunks = (int)std::min<int64_t>(kAttnMaxChunks, std::max<int64_t>(1, (4 * ctas + R - 1) / R));
     const int64_t grid = std::min<int64_t>(ctas, R * p.chunks);
-    attn_partial_tc<<<(unsigned)grid, kTcThreads, kTcSmem, s>>>(p, mk, mv);
+    kern<<<(unsigned)grid, kTcThreads, kTcSmem, s>>>(p, mk, mv);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_attn_combine(p, R, s);

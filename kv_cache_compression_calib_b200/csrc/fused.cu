@@ -135,8 +135,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
     unsigned long long T[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) T[i] = PRE ? turns_sm[8 * gl + i] : 0ull;
-    float stc[8], sts[8];
-    if (PRE) phasors(T, -(int64_t)NG, stc, sts);
+    unsigned long long TC[4], TS[4];
+    if (PRE) step_phasors(T, NG, TC, TS);
     const unsigned long long pol = policy_evict_first();
     RowCtx c;
     set_row_coef(c, p, r, gl, coef_sm + gl * kCoefPerGroup);
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
                 ok[u] = !PAGED || slot[u] >= 0;
                 if (!ok[u]) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
             }
-            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, stc, sts, part);
+            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, TC, TS, part);
         } else {
 #pragma unroll
             for (int u = 0; u < U; u++) {

@@ -68,8 +68,8 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE && !PAGED) ?
     unsigned long long T[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * gl + i] : 0ull;
-    float stc[8], sts[8];  // e^{-i w NG}: from one key's rotation to the next one's in a batch
-    if (PRE) phasors(T, -(int64_t)NG, stc, sts);
+    unsigned long long TC[4], TS[4];  // e^{-i w NG}: from one key's rotated coefficients to the next one's
+    if (PRE) step_phasors(T, NG, TC, TS);
     const unsigned long long pol = policy_evict_first();
 
     // Row holding key `beg`: the last r with row_off[r] <= beg.
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE && !PAGED) ?
                 ok[u] = !PAGED || slot[u] >= 0;
                 if (!ok[u]) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
             }
-            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, stc, sts, part);
+            batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, TC, TS, part);
         } else {
             // Batch crosses a row boundary or the span end: one segment per row.
 #pragma unroll
@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE) ? 3 : 2) sc
     unsigned long long T[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) T[i] = PRE ? p.turns[8 * gl + i] : 0ull;
-    float stc[8], sts[8];
-    if (PRE) phasors(T, -(int64_t)NG, stc, sts);
+    unsigned long long TC[4], TS[4];
+    if (PRE) step_phasors(T, NG, TC, TS);
 
     int rl = 0, rh = R;
     while (rh - rl > 1) {
@@ -296,8 +296,8 @@ __global__ void __launch_bounds__(kScoreThreads, (ELEM == 1 && !PRE) ? 3 : 2) sc
                 kpos[u] = PRE ? (pos_bulk ? spos[idx] : __ldg(p.pos + b0 + idx)) : 0;
             }
             batch_partials_lazy<PRE, U, NG, KeyChunk<ELEM, IL, F>>(
-                [&](int u, KeyChunk<ELEM, IL, F> &kc) { kc.lds(slot + (NG * u + q) * RB, gl); }, kpos, c, T, stc,
-                sts, part);
+                [&](int u, KeyChunk<ELEM, IL, F> &kc) { kc.lds(slot + (NG * u + q) * RB, gl); }, kpos, c, T, TC,
+                TS, part);
         } else {
             // Batch crosses a row boundary or the span end: one segment per row,
             // each key read from the slot as it is scored.

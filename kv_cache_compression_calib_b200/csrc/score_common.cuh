@@ -163,14 +163,101 @@ __device__ __forceinline__ float partial_pre(const float (&x)[8], const float (&
     return partial_pre_rot(x, y, c, cs, sn);
 }
 
-// Partials of one lane's U keys of a whole batch (keys NG slots apart).  Pre-RoPE:
-// the first key's phasors from the reduced phase, each next key's by one complex
-// step (stc, sts) = e^{-i w NG} when the positions advance by NG (any gap: the
-// key's own reduced phase).  Invalid (unplaceable) keys give 0.
+// The step e^{-i w NG} from one key of a lane's batch to the next (pre-RoPE),
+// two pairs per register: TC = cos, TS = sin.
+__device__ __forceinline__ void step_phasors(const unsigned long long (&T)[8], int NG, unsigned long long (&TC)[4],
+                                             unsigned long long (&TS)[4]) {
+    float cs[8], sn[8];
+    phasors(T, -(int64_t)NG, cs, sn);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        TC[k] = f2(cs[2 * k], cs[2 * k + 1]);
+        TS[k] = f2(sn[2 * k], sn[2 * k + 1]);
+    }
+}
+
+// Pre-RoPE, rotated coefficients of 8 pairs, two pairs per register:
+// B_i = A'_i (cs_i + i sn_i), formed exactly as partial_pre_rot forms them.
+__device__ __forceinline__ void rotate_coef(const RowCtx &c, const float (&cs)[8], const float (&sn)[8],
+                                            unsigned long long (&BR)[4], unsigned long long (&BI)[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const unsigned long long AR = f2(c.ar[2 * k], c.ar[2 * k + 1]), AI = f2(c.ai[2 * k], c.ai[2 * k + 1]);
+        const unsigned long long CS = f2(cs[2 * k], cs[2 * k + 1]), SN = f2(sn[2 * k], sn[2 * k + 1]);
+        BR[k] = fma2(AR, CS, mul2(neg2(AI), SN));
+        BI[k] = fma2(AR, SN, mul2(AI, CS));
+    }
+}
+
+// B <- B * e^{-i w NG} (TC, TS the step's cos and sin): the rotated
+// coefficients of the key NG slots further on.
+__device__ __forceinline__ void advance_coef(unsigned long long (&BR)[4], unsigned long long (&BI)[4],
+                                             const unsigned long long (&TC)[4], const unsigned long long (&TS)[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const unsigned long long r = fma2(BR[k], TC[k], mul2(BI[k], neg2(TS[k])));
+        BI[k] = fma2(BR[k], TS[k], mul2(BI[k], TC[k]));
+        BR[k] = r;
+    }
+}
+
+// Partial score of 8 pre-RoPE pairs given their rotated coefficients: the dot
+// product and the norm term in the order of partial_pre_rot.
+__device__ __forceinline__ float partial_rotated(const float (&x)[8], const float (&y)[8],
+                                                 const unsigned long long (&BR)[4],
+                                                 const unsigned long long (&BI)[4], const RowCtx &c) {
+    unsigned long long d = 0ull, e = 0ull;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const unsigned long long X = f2(x[2 * k], x[2 * k + 1]), Y = f2(y[2 * k], y[2 * k + 1]);
+        d = fma2(BR[k], X, d);
+        d = fma2(BI[k], Y, d);
+        const float2 q = f2split(fma2(X, X, mul2(Y, Y)));
+        e = fma2(f2(c.cc[2 * k], c.cc[2 * k + 1]), f2(sqrt_approx(q.x), sqrt_approx(q.y)), e);
+    }
+    const float2 dd = f2split(d), ee = f2split(e);
+    return (dd.x + dd.y) + (ee.x + ee.y);
+}
+
+// Pre-RoPE partials of a lane's U keys (NG slots apart): the first key's rotated
+// coefficients from its exactly reduced phase, each next key's by one complex
+// step of the coefficients themselves when the positions advance by NG (any
+// gap: from the key's own reduced phase).  key(u, x, y) unpacks key u.
+template <int U, int NG, typename Key>
+__device__ __forceinline__ void pre_partials(Key &&key, const int32_t (&kpos)[U], const bool (&ok)[U],
+                                             const RowCtx &c, const unsigned long long (&T)[8],
+                                             const unsigned long long (&TC)[4], const unsigned long long (&TS)[4],
+                                             float (&part)[U]) {
+    unsigned long long BR[4], BI[4];
+    {
+        float cs[8], sn[8];
+        phasors(T, c.p_now - (int64_t)kpos[0], cs, sn);
+        rotate_coef(c, cs, sn, BR, BI);
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+        if (u > 0) {
+            if (kpos[u] == kpos[u - 1] + NG) {
+                advance_coef(BR, BI, TC, TS);
+            } else {
+                float cs[8], sn[8];
+                phasors(T, c.p_now - (int64_t)kpos[u], cs, sn);
+                rotate_coef(c, cs, sn, BR, BI);
+            }
+        }
+        float x[8], y[8];
+        key(u, x, y);
+        part[u] = ok[u] ? partial_rotated(x, y, BR, BI, c) : 0.f;
+    }
+}
+
+// Partials of one lane's U keys of a whole batch (keys NG slots apart); pre-RoPE
+// keys through pre_partials.  Invalid (unplaceable) keys give 0.
 template <bool PRE, int U, int NG, typename Chunk>
 __device__ __forceinline__ void batch_partials(const Chunk (&kc)[U], const int32_t (&kpos)[U], const bool (&ok)[U],
                                                const RowCtx &c, const unsigned long long (&T)[8],
-                                               const float (&stc)[8], const float (&sts)[8], float (&part)[U]) {
+                                               const unsigned long long (&TC)[4], const unsigned long long (&TS)[4],
+                                               float (&part)[U]) {
     if (!PRE) {
 #pragma unroll
         for (int u = 0; u < U; u++) {
@@ -180,18 +267,8 @@ __device__ __forceinline__ void batch_partials(const Chunk (&kc)[U], const int32
         }
         return;
     }
-    float cs[8], sn[8];
-    phasors(T, c.p_now - (int64_t)kpos[0], cs, sn);
-#pragma unroll
-    for (int u = 0; u < U; u++) {
-        if (u > 0) {
-            if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
-            else phasors(T, c.p_now - (int64_t)kpos[u], cs, sn);
-        }
-        float x[8], y[8];
-        kc[u].unpack(x, y);
-        part[u] = ok[u] ? partial_pre_rot(x, y, c, cs, sn) : 0.f;
-    }
+    pre_partials<U, NG>([&](int u, float(&x)[8], float(&y)[8]) { kc[u].unpack(x, y); }, kpos, ok, c, T, TC, TS,
+                        part);
 }
 
 // batch_partials for keys read as they are scored (from shared memory, where a
@@ -199,9 +276,10 @@ __device__ __forceinline__ void batch_partials(const Chunk (&kc)[U], const int32
 // fetches key u.  The same arithmetic in the same order, so the same bits.
 template <bool PRE, int U, int NG, typename Chunk, typename Load>
 __device__ __forceinline__ void batch_partials_lazy(Load &&load, const int32_t (&kpos)[U], const RowCtx &c,
-                                                    const unsigned long long (&T)[8], const float (&stc)[8],
-                                                    const float (&sts)[8], float (&part)[U]) {
-    if (!PRE) {
+                                                    const unsigned long long (&T)[8],
+                                                    const unsigned long long (&TC)[4],
+                                                    const unsigned long long (&TS)[4], float (&part)[U]) {
+    if constexpr (!PRE) {
 #pragma unroll
         for (int u = 0; u < U; u++) {
             Chunk kc;
@@ -210,21 +288,17 @@ __device__ __forceinline__ void batch_partials_lazy(Load &&load, const int32_t (
             kc.unpack(x, y);
             part[u] = partial_post(x, y, c);
         }
-        return;
-    }
-    float cs[8], sn[8];
-    phasors(T, c.p_now - (int64_t)kpos[0], cs, sn);
+    } else {
+        bool ok[U];
 #pragma unroll
-    for (int u = 0; u < U; u++) {
-        if (u > 0) {
-            if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
-            else phasors(T, c.p_now - (int64_t)kpos[u], cs, sn);
-        }
-        Chunk kc;
-        load(u, kc);
-        float x[8], y[8];
-        kc.unpack(x, y);
-        part[u] = partial_pre_rot(x, y, c, cs, sn);
+        for (int u = 0; u < U; u++) ok[u] = true;
+        pre_partials<U, NG>(
+            [&](int u, float(&x)[8], float(&y)[8]) {
+                Chunk kc;
+                load(u, kc);
+                kc.unpack(x, y);
+            },
+            kpos, ok, c, T, TC, TS, part);
     }
 }
 

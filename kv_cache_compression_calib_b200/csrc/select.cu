@@ -512,7 +512,11 @@ __device__ __forceinline__ bool one_pass_select(const float *sc, int M, uint32_t
     return true;
 }
 
-template <bool GATHER>
+// LONG: rows average more than one chunk.  Then multi-chunk rows try the single
+// pass (its 96 KB of dynamic shared memory are reserved) and the kernel copies
+// its row's records; otherwise neither, and the launch reserves no dynamic shared
+// memory, leaving the L1 its passes' re-reads use.
+template <bool LONG>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectParams p, const GatherParams g) {
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t bmw[kWords];  // keep-bitmap of the current chunk
@@ -558,7 +562,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
         const float *sc = p.scores + row_lo;
         const bool vec = (((uintptr_t)sc) & 15) == 0;
         const int nchunks = (int)((M + kChunk - 1) / kChunk);
-        if (M >= kOpMinRow && M <= kOpMaxRow) {
+        if (LONG && M >= kOpMinRow && M <= kOpMaxRow) {
             extern __shared__ uint32_t sel_dyn[];
             if (one_pass_select(sc, (int)M, K, vec, out, p.flags, sel_dyn, hist, scan_sm, &sh_bin, &sh_above, &sh_count,
                                 red_fa, red_fb, red_a, red_b))
@@ -788,7 +792,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
             emit_bitmap(bmw, c0, out, K, out_base, scan_sm);
         }
     } while (0);
-    if (!GATHER || !row_ok) return;
+    if (!LONG || !row_ok) return;
     __syncthreads();  // out[] of this row is complete and visible to the block
     const int cnt = (int)(N < (int64_t)B ? N : (int64_t)B);
     switch (g.geo.D * g.geo.elem_bytes) {
@@ -799,27 +803,29 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
     }
 }
 
-template <bool GATHER>
+template <bool LONG>
 static cudaError_t launch_select_t(const SelectParams &p, const GatherParams &g, cudaStream_t s) {
     const int64_t R = (int64_t)p.geo.L * p.geo.S * p.geo.H;
     if (R <= 0) return cudaSuccess;
+    const size_t dyn = LONG ? kSelDynSmem : 0;
     static bool attr[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!attr[dev & 63]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(select_kernel<GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
+    if (LONG && !attr[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kSelDynSmem);
         if (e != cudaSuccess) return e;
         attr[dev & 63] = true;
     }
-    return launch_pdl(select_kernel<GATHER>, dim3((unsigned)R), dim3(kSelThreads), kSelDynSmem, s, p, g);
+    return launch_pdl(select_kernel<LONG>, dim3((unsigned)R), dim3(kSelThreads), dyn, s, p, g);
 }
 
-// Rows longer than one selection chunk on average: the selection kernel copies
-// its row's records itself (rows still selecting overlap rows already copying,
-// over several waves).  Shorter rows all select in one wave, where the gather
-// kernel, with more bytes in flight per thread, moves the records faster.  The
-// results are identical either way.
+// Rows longer than one selection chunk on average: the single pass for
+// multi-chunk rows, and the selection kernel copies its row's records itself
+// (rows still selecting overlap rows already copying, over several waves).
+// Shorter rows all select in one wave, where the gather kernel, with more bytes
+// in flight per thread, moves the records faster.  The results are identical
+// either way.
 cudaError_t launch_select_gather(const SelectParams &p, const GatherParams &g, cudaStream_t s) {
     const int rb = g.geo.D * g.geo.elem_bytes;
     if (rb != 64 && rb != 128 && rb != 256 && rb != 512) return cudaErrorInvalidValue;

@@ -154,6 +154,7 @@ struct FusedParams {
 cudaError_t launch_calib(const CalibParams &p, cudaStream_t s);
 cudaError_t launch_fused(const FusedParams &p, int pre_rope, cudaStream_t s);
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t s);
+cudaError_t launch_attention_tc(const AttnParams &p, int64_t R, cudaStream_t s);  // cudaErrorNotSupported outside its case
 cudaError_t launch_calib_update(const CalibUpdateParams &p, cudaStream_t s);
 cudaError_t launch_stats(const StatsParams &p, cudaStream_t s);
 cudaError_t launch_key_centres(const KeyCentreParams &p, cudaStream_t s);

@@ -20,12 +20,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def run_attention(m, kv, K, V, q, scale, n_seqs):
+def run_attention(m, kv, K, V, q, scale, n_seqs, fn=None):
     L, S, Hq, d = q.shape
     out = torch.full((L, S, Hq, d), float("nan"), device=DEV)
     lse = torch.full((L, S, Hq), float("nan"), device=DEV)
     ws = tri.alloc_attention_workspace(m, n_seqs)
-    tri.tri_decode_attention(m, kv, K, V, q, scale, out, lse, ws)
+    (fn or tri.tri_decode_attention)(m, kv, K, V, q, scale, out, lse, ws)
     st, flags = tri.tri_status_check(ws)
     assert st == 0, flags
     return out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
@@ -197,3 +197,43 @@ def test_attention_full_size_after_compaction():
         vals = H.to_f64(cache.V[a + sampled[r]])
         for g in range(G):
             check_row(out[li, s, h * G + g], lse[li, s, h * G + g], qf[s, h * G + g], keys, vals, scale, (r, g))
+
+
+@pytest.mark.parametrize("hq", [8, 32, 64, 128])
+def test_attention_tensor_memory_kernel(hq):
+    """tri_decode_attention_tc (tcgen05, bf16, head dim 128, contiguous): G = 1, 4, 8 and
+    16 queries per KV head; rows empty, of one key, of exact multiples of the 128-key
+    tile and with ragged tails, against the oracle."""
+    wl = synth.WORKLOADS["single_layer_4k"].with_(name=f"atc{hq}", n_q_heads=hq, batch=7, n_calib=8)
+    lens = [4096, 0, 1, 33, 700, 128, 256]
+    host = synth.make_contig(wl, "cpu", lens=lens)
+    q = synth.decode_queries(wl, 0, np.asarray(lens), "cpu")[None]
+    scale = 1.0 / math.sqrt(128)
+    m = model_of(wl, 1)
+    kv = tri.kv_contig(len(lens), host.row_off.to(DEV), host.total)
+    out, lse = run_attention(m, kv, host.K.to(DEV), host.V.to(DEV), q.to(DEV).contiguous(), scale, len(lens),
+                             fn=tri.tri_decode_attention_tc)
+    K, V, qf = H.to_f64(host.K), H.to_f64(host.V), H.to_f64(q)
+    G = wl.group
+    for r in range(host.n_rows):
+        _, s_, h = host.row_lhs(r)
+        a, b = host.row_off_np[r], host.row_off_np[r + 1]
+        for g in range(G):
+            qh = h * G + g
+            check_row(out[0, s_, qh], lse[0, s_, qh], qf[0, s_, qh], K[a:b], V[a:b], scale, (r, g))
+
+
+def test_attention_tensor_memory_kernel_refuses_other_caches():
+    """Head dims other than 128, fp8 elements and paged caches are refused before any launch."""
+    from kv_cache_compression_calib_b200 import _abi
+    for d, elem in ((64, tri.TRI_ELEM_BF16), (128, tri.TRI_ELEM_FP8_E4M3)):
+        m = tri.model(1, 32, 8, 1e6, head_dim=d)
+        ro = torch.zeros(9, dtype=torch.int64, device=DEV)
+        ro[1:] = 16
+        kv = tri.kv_contig(1, ro, 16, elem)
+        buf = torch.zeros(16 * d, dtype=torch.bfloat16, device=DEV)
+        out = torch.zeros(32 * d, device=DEV)
+        ws = tri.alloc_attention_workspace(m, 1)
+        with pytest.raises(tri.TriError) as e:
+            tri.tri_decode_attention_tc(m, kv, buf, buf, buf, 0.1, out, None, ws)
+        assert e.value.status == _abi.TRI_ERR_UNSUPPORTED
