@@ -304,9 +304,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_simt(const AttnPara
 // ------------------------------------------------ tensor-core slice kernel
 //
 // For d <= 128: warp-level MMAs (mma.sync m16n8k16, fp32 accumulation) with the
-// G <= 16 queries as the 16 rows of the A operand - below the 64-row minimum
-// of tcgen05, and the op is HBM-bound, so the tensor pipe only takes the
-// multiply-adds off the CUDA cores.  bf16 caches use bf16 MMAs (the q and key
+// G <= 16 queries as the 16 rows of the A operand.  The op is HBM-bound, so the
+// tensor pipe only takes the multiply-adds off the CUDA cores.  (The transposed
+// form, keys on the 128-row M side of tcgen05.mma and the queries on N, is the
+// kernel of attention_tc.cu; on the same caches it is slower than this one,
+// because each 128-key tile's softmax sits between its two MMAs in one
+// warpgroup's chain.)  bf16 caches use bf16 MMAs (the q and key
 // products are exact in fp32); fp8 caches use f16 MMAs with e4m3 converted to
 // f16 exactly and q rounded to f16 (exact for |q| in [2^-14, 65504]).  A
 // persistent grid of the resident CTAs (4 warps each): every warp is a worker

@@ -14,7 +14,16 @@
 // sum |k|) per pair.  Pass 2: one CTA per row adds its
 // chunks' partials in chunk order and divides.  Both passes sum in a fixed order,
 // so results are deterministic.  It reads every key once: an HBM-bound pass like
-// the scoring one (plus one sin/cos per (key, pair) for a RoPE cache).
+// the scoring one.
+//
+// RoPE caches: the de-rotated sum of a lane's keys is accumulated in Horner form
+// along the lane's keys, H = sum_i k_i e^{i w (p - p_i)} with p the position of
+// the lane's last key, so a key whose position is a fixed step D past the last
+// one costs H <- H e^{i w D} + k: one complex multiply-add per pair, with two
+// constant steps (the next key of a lane's batch, NG positions on, and the first
+// key of the lane's next batch).  Any other key, and the end of every run of
+// kFlush batches, first settles H into the run sums as H e^{-i w p} (one sin/cos
+// per pair of the exactly reduced phase) and restarts it.
 #include "score_common.cuh"
 #include "stage.cuh"
 
@@ -25,9 +34,59 @@ constexpr double kKcTurnScale = 2.9358905032820014e+18;  // 2^64 / (2 pi)
 
 constexpr int kFlush = 8;  // batches summed in fp32 before folding into fp64
 
-// Each thread folds its fp32 runs into its own fp64 column of `acc` (element-major,
-// so a warp's 8-byte accesses are consecutive); after the loop the CTA adds the
-// columns of every pair in a fixed order.
+// Turn rates T_f = w_f / 2 pi in 0.64 fixed point, w_f = theta^(-2f/d), of the F
+// pairs into t[f]: one fp64 power per pair, by the block's first F threads.
+template <int F>
+__device__ __forceinline__ void kc_turns(double theta, unsigned long long *t) {
+    for (int f = threadIdx.x; f < F; f += blockDim.x)
+        t[f] = __double2ull_rn(pow(theta, -2.0 * (double)f / (double)(2 * F)) * kKcTurnScale);
+}
+
+// e^{i w delta} of the lane's 8 pairs, two pairs per register: C = cos, S = sin, NS = -sin.
+__device__ __forceinline__ void kc_step(const unsigned long long (&T)[8], int64_t delta, unsigned long long (&C)[4],
+                                        unsigned long long (&S)[4], unsigned long long (&NS)[4]) {
+    float cs[8], sn[8];
+    phasors(T, delta, cs, sn);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        C[k] = f2(cs[2 * k], cs[2 * k + 1]);
+        S[k] = f2(sn[2 * k], sn[2 * k + 1]);
+        NS[k] = neg2(S[k]);
+    }
+}
+
+// Settles the Horner sum H (relative to position p) into the run sums,
+// fr + i fi += H e^{-i w p}, and clears it.  Tg: the lane group's 8 turn rates in
+// shared memory (read only here, so they hold no registers in the key loop).
+__device__ __forceinline__ void kc_settle(const unsigned long long *Tg, int32_t p, unsigned long long (&HR)[4],
+                                          unsigned long long (&HI)[4], unsigned long long (&fr)[4],
+                                          unsigned long long (&fi)[4]) {
+    unsigned long long T[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) T[i] = Tg[i];
+    float cs[8], sn[8];
+    phasors(T, (int64_t)p, cs, sn);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const unsigned long long CS = f2(cs[2 * k], cs[2 * k + 1]), SN = f2(sn[2 * k], sn[2 * k + 1]);
+        fr[k] = add2(fr[k], fma2(HR[k], CS, mul2(HI[k], SN)));        // HR cos + HI sin
+        fi[k] = add2(fi[k], fma2(HI[k], CS, mul2(neg2(HR[k]), SN)));  // HI cos - HR sin
+        HR[k] = HI[k] = 0ull;
+    }
+}
+
+// H <- H e^{i w D} + (X + i Y) for the step (C, S, NS) of D, two pairs per register.
+__device__ __forceinline__ void kc_horner(unsigned long long (&HR)[4], unsigned long long (&HI)[4], int k,
+                                          unsigned long long X, unsigned long long Y, const unsigned long long (&C)[4],
+                                          const unsigned long long (&S)[4], const unsigned long long (&NS)[4]) {
+    const unsigned long long re = fma2(HR[k], C[k], fma2(HI[k], NS[k], X));
+    HI[k] = fma2(HR[k], S[k], fma2(HI[k], C[k], Y));
+    HR[k] = re;
+}
+
+// Each run of kFlush batches is folded in fp64 across the lanes of a warp that
+// hold the same pairs (a fixed shuffle tree) into one column per (warp, lane
+// group); after the loop the CTA adds the columns of every pair in warp order.
 template <bool PAGED, bool POST, int ELEM, bool IL, int LPK>
 __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCentreParams p) {
     constexpr int NG = 32 / LPK;
@@ -35,7 +94,8 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
     constexpr int F = 8 * LPK;
     constexpr int RB = 2 * F * ELEM;
     constexpr int W = kKcThreads / 32;
-    __shared__ double acc[24][kKcThreads];
+    __shared__ double acc[24 * W * LPK];          // [24][W * LPK]: one column per (warp, lane group)
+    __shared__ unsigned long long t_sm[8 * LPK];  // turn rates of the pairs, [gl][i]
     const Geometry &geo = p.geo;
     const int64_t r = blockIdx.x / kKeyCentreChunks;
     const int chunk = (int)(blockIdx.x % kKeyCentreChunks);
@@ -53,22 +113,45 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
     const int64_t beg = lo + n * chunk / kKeyCentreChunks;
     const int64_t end = lo + n * (chunk + 1) / kKeyCentreChunks;
 
-    unsigned long long T[8];
+    if (POST) kc_turns<F>(p.theta, t_sm);
+    for (int e = threadIdx.x; e < 24 * W * LPK; e += kKcThreads) acc[e] = 0.0;
+    __syncthreads();  // t_sm and acc written
+    const unsigned long long *Tg = t_sm + 8 * gl;
+    // Horner steps: the lane's next key in a batch (NG positions on) and the first
+    // key of its next batch (W KB - (U - 1) NG positions after the batch's last).
+    constexpr int DB = W * NG * U - (U - 1) * NG;
+    unsigned long long ZC[4], ZS[4], ZN[4], BC[4], BS[4], BN[4];
+    if (POST) {
+        unsigned long long T[8];
 #pragma unroll
-    for (int i = 0; i < 8; i++)
-        T[i] = POST ? __double2ull_rn(pow(p.theta, -2.0 * (double)(8 * gl + i) / (double)(2 * F)) * kKcTurnScale)
-                    : 0ull;
-    float stc[8], sts[8];  // e^{+i w NG}: from one key's rotation to the next one's in a batch
-    if (POST) phasors(T, (int64_t)NG, stc, sts);
+        for (int i = 0; i < 8; i++) T[i] = Tg[i];
+        kc_step(T, NG, ZC, ZS, ZN);
+        kc_step(T, DB, BC, BS, BN);
+    }
     const unsigned long long pol = policy_evict_first();
     const int32_t *table = geo.block_table + (int64_t)s * geo.max_blocks;
     const int64_t layer_blk = (int64_t)l * geo.n_blocks;
-
+    unsigned long long fr2[4], fi2[4], fn2[4], HR[4], HI[4];  // pairs (2k, 2k+1) packed
 #pragma unroll
-    for (int i = 0; i < 24; i++) acc[i][threadIdx.x] = 0.0;
-    float fr[8], fi[8], fn[8];
+    for (int i = 0; i < 4; i++) fr2[i] = fi2[i] = fn2[i] = HR[i] = HI[i] = 0ull;
+    int32_t plast = 0;  // position of the lane's last key (H is relative to it)
+    // Adds the lanes' runs into this warp's columns: fp64 tree over the NG lanes
+    // of each lane group, then lane group gl's column.
+    auto flush = [&]() {
+        if (POST) kc_settle(Tg, plast, HR, HI, fr2, fi2);
 #pragma unroll
-    for (int i = 0; i < 8; i++) fr[i] = fi[i] = fn[i] = 0.f;
+        for (int c3 = 0; c3 < 3; c3++)
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float2 pr = f2split(c3 == 0 ? fr2[i >> 1] : c3 == 1 ? fi2[i >> 1] : fn2[i >> 1]);
+                double v = (double)((i & 1) ? pr.y : pr.x);
+#pragma unroll
+                for (int o = LPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (q == 0) acc[(c3 * 8 + i) * (W * LPK) + warp * LPK + gl] += v;
+            }
+#pragma unroll
+        for (int i = 0; i < 4; i++) fr2[i] = fi2[i] = fn2[i] = 0ull;
+    };
 
     int run = 0;
     for (int64_t b0 = beg + (int64_t)warp * NG * U; b0 < end; b0 += (int64_t)W * NG * U) {
@@ -100,56 +183,41 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_kernel(const KeyCent
                 kc[u].zero();
             }
         }
-        // Rotation phasors e^{i w pos} of the lane's keys: the first from its reduced
-        // phase, each next one by one complex step when positions advance by NG.
-        float cs[8], sn[8];
-        if (POST) phasors(T, (int64_t)kpos[0], cs, sn);
 #pragma unroll
         for (int u = 0; u < U; u++) {
-            if (POST && u > 0) {
-                if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
-                else phasors(T, (int64_t)kpos[u], cs, sn);
-            }
             if (slot[u] < 0) continue;
             float x[8], y[8];
             kc[u].unpack(x, y);
+            if (POST && !pos_follows(kpos[u], plast, u == 0 ? DB : NG)) kc_settle(Tg, plast, HR, HI, fr2, fi2);
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                float xr = x[i], xi = y[i];
+            for (int k2 = 0; k2 < 4; k2++) {
+                const unsigned long long X = f2(x[2 * k2], x[2 * k2 + 1]), Y = f2(y[2 * k2], y[2 * k2 + 1]);
                 if (POST) {
-                    xr = x[i] * cs[i] + y[i] * sn[i];
-                    xi = y[i] * cs[i] - x[i] * sn[i];
+                    if (u == 0) kc_horner(HR, HI, k2, X, Y, BC, BS, BN);
+                    else kc_horner(HR, HI, k2, X, Y, ZC, ZS, ZN);
+                } else {
+                    fr2[k2] = add2(fr2[k2], X);
+                    fi2[k2] = add2(fi2[k2], Y);
                 }
-                fr[i] += xr;
-                fi[i] += xi;
-                fn[i] += sqrt_approx(fmaf(x[i], x[i], y[i] * y[i]));
+                const float2 qq = f2split(fma2(X, X, mul2(Y, Y)));
+                fn2[k2] = add2(fn2[k2], f2(sqrt_approx(qq.x), sqrt_approx(qq.y)));
             }
+            if (POST) plast = kpos[u];
         }
         if (++run == kFlush) {
             run = 0;
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                acc[i][threadIdx.x] += (double)fr[i];
-                acc[8 + i][threadIdx.x] += (double)fi[i];
-                acc[16 + i][threadIdx.x] += (double)fn[i];
-                fr[i] = fi[i] = fn[i] = 0.f;
-            }
+            flush();
         }
     }
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        acc[i][threadIdx.x] += (double)fr[i];
-        acc[8 + i][threadIdx.x] += (double)fi[i];
-        acc[16 + i][threadIdx.x] += (double)fn[i];
-    }
+    flush();
     __syncthreads();
-    // Pair f = 8 gl + i lives in the columns of the threads with that gl (every warp,
-    // every key group): add them in thread order.
+    // Pair f = 8 gl + i lives in the column of lane group gl of every warp: add
+    // them in warp order.
     for (int e = threadIdx.x; e < 3 * F; e += kKcThreads) {
         const int f = e % F, comp = e / F;
         const int g = f >> 3, i = f & 7;
         double v = 0.0;
-        for (int t = g; t < kKcThreads; t += LPK) v += acc[comp * 8 + i][t];
+        for (int w = 0; w < W; w++) v += acc[(comp * 8 + i) * (W * LPK) + w * LPK + g];
         p.partial[((r * kKeyCentreChunks + chunk) * F + f) * 3 + comp] = v;
     }
 }
@@ -179,7 +247,7 @@ struct KcStaging {
     static constexpr size_t SMEM = (size_t)HEADER + ACC_BYTES + (size_t)kWarps * STAGES * SLOT;
     static_assert(KB % 4 == 0 && SLOT % 16 == 0 && KEY_BYTES % 16 == 0 && ACC_BYTES % 16 == 0, "16-byte units");
     static_assert(kWarps * STAGES * 8 <= HEADER, "barriers fit the header");
-    static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+    static_assert(2 * (SMEM + 8 * 8 * LPK + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 // Issues batch t of a warp (keys b0 .. b0 + n - 1) into slot t % STAGES: its
@@ -209,6 +277,7 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
     constexpr int NG = St::NG, U = St::U, KB = St::KB, F = St::F, RB = St::RB, W = St::kWarps;
     constexpr int STAGES = St::STAGES;
     extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ unsigned long long t_sm[8 * LPK];  // turn rates of the pairs, [gl][i]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
     double *acc = reinterpret_cast<double *>(smem + St::HEADER);  // [24][W * LPK]
     unsigned char *rings = smem + St::HEADER + St::ACC_BYTES;
@@ -229,36 +298,42 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
     const int64_t first0 = beg + (int64_t)warp * KB;
     const int nbw = first0 < end ? (int)((end - first0 + (int64_t)W * KB - 1) / ((int64_t)W * KB)) : 0;
 
-    unsigned long long T[8];
-#pragma unroll
-    for (int i = 0; i < 8; i++)
-        T[i] = POST ? __double2ull_rn(pow(p.theta, -2.0 * (double)(8 * gl + i) / (double)(2 * F)) * kKcTurnScale)
-                    : 0ull;
-    float stc[8], sts[8];
-    if (POST) phasors(T, (int64_t)NG, stc, sts);
     const unsigned long long pol = policy_evict_first();
     uint64_t *bar = bars + warp * STAGES;
     unsigned char *ring = rings + (size_t)warp * STAGES * St::SLOT;
 
+    if (POST) kc_turns<F>(p.theta, t_sm);
     for (int e = threadIdx.x; e < 24 * W * LPK; e += kKcThreads) acc[e] = 0.0;
     if (lane == 0) {
 #pragma unroll
         for (int k = 0; k < STAGES; k++) mbar_init(&bar[k], 1);
         mbar_init_fence();
     }
-    __syncthreads();
+    __syncthreads();  // t_sm, acc and the barriers are ready
+    const unsigned long long *Tg = t_sm + 8 * gl;
+    constexpr int DB = W * KB - (U - 1) * NG;  // a lane's last key of a batch -> its first of the next
+    unsigned long long ZC[4], ZS[4], ZN[4], BC[4], BS[4], BN[4];
+    if (POST) {
+        unsigned long long T[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) T[i] = Tg[i];
+        kc_step(T, NG, ZC, ZS, ZN);
+        kc_step(T, DB, BC, BS, BN);
+    }
     if (lane == 0)
         for (int t = 0; t < min(nbw, STAGES); t++) {
             const int64_t b0 = first0 + (int64_t)t * W * KB;
             kc_stage_batch<St>(p, b0, (int)min((int64_t)KB, end - b0), ring, bar, t, pol);
         }
 
-    unsigned long long fr2[4], fi2[4], fn2[4];  // fp32 runs, pairs (2k, 2k+1) packed
+    unsigned long long fr2[4], fi2[4], fn2[4], HR[4], HI[4];  // fp32 runs, pairs (2k, 2k+1) packed
 #pragma unroll
-    for (int i = 0; i < 4; i++) fr2[i] = fi2[i] = fn2[i] = 0ull;
+    for (int i = 0; i < 4; i++) fr2[i] = fi2[i] = fn2[i] = HR[i] = HI[i] = 0ull;
+    int32_t plast = 0;  // position of the lane's last key (H is relative to it)
     // Adds the lanes' runs into this warp's columns: fp64 tree over the NG lanes
     // of each lane group, then lane group gl's column.
     auto fold = [&]() {
+        if (POST) kc_settle(Tg, plast, HR, HI, fr2, fi2);
 #pragma unroll
         for (int c3 = 0; c3 < 3; c3++)
 #pragma unroll
@@ -298,36 +373,30 @@ __global__ void __launch_bounds__(kKcThreads, 2) key_centre_staged_kernel(const 
             kpos[u] = 0;
             if (valid[u] && POST) kpos[u] = k < a1 ? spos[k - a0] : __ldg(p.pos + k);
         }
-        float cs[8], sn[8];
-        if (POST) phasors(T, (int64_t)kpos[0], cs, sn);
 #pragma unroll
         for (int u = 0; u < U; u++) {
-            if (POST && u > 0) {
-                if (kpos[u] == kpos[u - 1] + NG) advance_phasors(cs, sn, stc, sts);
-                else phasors(T, (int64_t)kpos[u], cs, sn);
-            }
             if (!valid[u]) continue;
             KeyChunk<ELEM, IL, F> kc;  // read from the slot as it is used
             kc.lds(slot + (NG * u + q) * RB, gl);
             float x[8], y[8];
             kc.unpack(x, y);
-            // Two pairs per packed instruction: the de-rotation by e^{-i w pos},
-            // the sums and the magnitudes.
+            if (POST && !pos_follows(kpos[u], plast, u == 0 ? DB : NG)) kc_settle(Tg, plast, HR, HI, fr2, fi2);
+            // Two pairs per packed instruction: the Horner step (RoPE caches) or
+            // the plain sums, and the magnitudes.
 #pragma unroll
             for (int k2 = 0; k2 < 4; k2++) {
                 const unsigned long long X = f2(x[2 * k2], x[2 * k2 + 1]), Y = f2(y[2 * k2], y[2 * k2 + 1]);
-                unsigned long long XR = X, XI = Y;
                 if (POST) {
-                    const unsigned long long CS = f2(cs[2 * k2], cs[2 * k2 + 1]);
-                    const unsigned long long SN = f2(sn[2 * k2], sn[2 * k2 + 1]);
-                    XR = fma2(X, CS, mul2(Y, SN));   // x cs + y sn
-                    XI = fma2(Y, CS, mul2(X, neg2(SN)));  // y cs - x sn
+                    if (u == 0) kc_horner(HR, HI, k2, X, Y, BC, BS, BN);
+                    else kc_horner(HR, HI, k2, X, Y, ZC, ZS, ZN);
+                } else {
+                    fr2[k2] = add2(fr2[k2], X);
+                    fi2[k2] = add2(fi2[k2], Y);
                 }
-                fr2[k2] = add2(fr2[k2], XR);
-                fi2[k2] = add2(fi2[k2], XI);
                 const float2 qq = f2split(fma2(X, X, mul2(Y, Y)));
                 fn2[k2] = add2(fn2[k2], f2(sqrt_approx(qq.x), sqrt_approx(qq.y)));
             }
+            if (POST) plast = kpos[u];
         }
         if (t + STAGES < nbw) {  // the slot's bytes are consumed: refill it
             fence_async_smem();

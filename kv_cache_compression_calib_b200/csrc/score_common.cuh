@@ -118,23 +118,6 @@ __device__ __forceinline__ void phasors(const unsigned long long (&T)[8], int64_
         __sincosf(turn_units23((unsigned long long)delta * T[i]) * kTurn23ToRad, &sn[i], &cs[i]);
 }
 
-// (cs, sn) <- (cs, sn) * (stc, sts) for the 8 pairs: the phasors of a key NG
-// slots further on, from those of this one (consecutive positions).
-__device__ __forceinline__ void advance_phasors(float (&cs)[8], float (&sn)[8], const float (&stc)[8],
-                                                const float (&sts)[8]) {
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-        const unsigned long long C = f2(cs[2 * k], cs[2 * k + 1]), S = f2(sn[2 * k], sn[2 * k + 1]);
-        const unsigned long long TC = f2(stc[2 * k], stc[2 * k + 1]), TS = f2(sts[2 * k], sts[2 * k + 1]);
-        const float2 nc = f2split(fma2(C, TC, mul2(f2(-sn[2 * k], -sn[2 * k + 1]), TS)));
-        const float2 ns = f2split(fma2(C, TS, mul2(S, TC)));
-        cs[2 * k] = nc.x;
-        cs[2 * k + 1] = nc.y;
-        sn[2 * k] = ns.x;
-        sn[2 * k + 1] = ns.y;
-    }
-}
-
 // Partial score of a pre-RoPE key given its rotation phasors e^{i w_i delta}: the
 // rotation, the dot product and the squared norms two pairs per packed instruction.
 __device__ __forceinline__ float partial_pre_rot(const float (&x)[8], const float (&y)[8], const RowCtx &c,
@@ -219,6 +202,12 @@ __device__ __forceinline__ float partial_rotated(const float (&x)[8], const floa
     return (dd.x + dd.y) + (ee.x + ee.y);
 }
 
+// True when position `pos` lies exactly `step` past `last` (positions are int32:
+// no wrap-around across the int32 range counts as a step).
+__device__ __forceinline__ bool pos_follows(int32_t pos, int32_t last, int step) {
+    return pos > last && (uint32_t)pos - (uint32_t)last == (uint32_t)step;
+}
+
 // Pre-RoPE partials of a lane's U keys (NG slots apart): the first key's rotated
 // coefficients from its exactly reduced phase, each next key's by one complex
 // step of the coefficients themselves when the positions advance by NG (any
@@ -237,7 +226,7 @@ __device__ __forceinline__ void pre_partials(Key &&key, const int32_t (&kpos)[U]
 #pragma unroll
     for (int u = 0; u < U; u++) {
         if (u > 0) {
-            if (kpos[u] == kpos[u - 1] + NG) {
+            if (pos_follows(kpos[u], kpos[u - 1], NG)) {
                 advance_coef(BR, BI, TC, TS);
             } else {
                 float cs[8], sn[8];
