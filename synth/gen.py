@@ -289,9 +289,15 @@ def decode_keys(wl: Workload, layer: int, round_idx: int, start: np.ndarray, cou
 FP8_MAX = 448.0  # largest finite OCP e4m3 value
 
 
-def to_fp8(t: torch.Tensor) -> torch.Tensor:
-    """The cache as an fp8 e4m3 cache would store it: clamp to +-448, round to nearest."""
-    return t.float().clamp_(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn)
+def to_fp8(t: torch.Tensor, chunk: int = 1 << 28) -> torch.Tensor:
+    """The cache as an fp8 e4m3 cache would store it: clamp to +-448, round to nearest.
+    Converted `chunk` elements at a time, so a cache near the device's size needs no
+    full-size fp32 copy."""
+    out = torch.empty(t.shape, dtype=torch.float8_e4m3fn, device=t.device)
+    src, dst = t.reshape(-1), out.view(-1)
+    for i in range(0, src.numel(), chunk):
+        dst[i:i + chunk] = src[i:i + chunk].float().clamp_(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn)
+    return out
 
 
 def decode_queries(wl: Workload, layer: int, p_now: np.ndarray, device, heads: LayerHeads = None) -> torch.Tensor:
