@@ -6,19 +6,9 @@
 //
 // A batched GEMV with G = Hq/H queries per KV head: 4 G flops per 2 d bytes of
 // K and V, bound by HBM.  Pass 1 cuts every row into slices and writes each
-// slice's unnormalised output, running maximum and sum to the workspace; pass 2
-// (attn_combine_kernel) merges a row's slices.  Pass 1 has two kernels:
-// attn_partial_mma (d <= 128, warp-level tensor-core MMAs, below) and
-// attn_partial_simt (d = 256, CUDA cores), described here.  `chunks` CTAs per
-// row (about one wave over the SMs), each over a contiguous slice of the row's
-// keys in tiles of TK keys (64, or 32 for 512-byte records).  K and V tiles are
-// staged in shared memory with cp.async (16-byte copies, double-buffered, rows
-// padded by 16 bytes so lane-per-key reads hit distinct banks).  QK: lane =
-// key, warps split the tile's keys into 32-key halves and the head dims into
-// slices, partial dot products for all G queries (q pre-scaled by scale * log2
-// e, broadcast from shared memory), added over the dim slices in a fixed order.
-// Online softmax in base 2, one warp per query.  PV: each thread owns a pair of
-// dims for all G queries over a group of the tile's keys.
+// slice's unnormalised output, running maximum and sum to the workspace
+// (attn_partial_mma, warp-level tensor-core MMAs, below; head dims 64, 128 and
+// 256); pass 2 (attn_combine_kernel) merges a row's slices.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -26,8 +16,6 @@
 #include "keys.cuh"
 
 namespace tri {
-
-constexpr int kAttnThreads = 256;
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
@@ -47,264 +35,11 @@ __device__ __forceinline__ int64_t paged_record(const Geometry &geo, const int32
     return ((((layer_blk + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) * geo.H) + h;
 }
 
-// 8 elements of a record (bf16: 16 bytes, fp8: 8 bytes) from shared memory, as floats.
-template <int ELEM>
-__device__ __forceinline__ void smem_elems8(const char *p, float (&x)[8]) {
-    if (ELEM == 2) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(p);
-        unpack_bf16x8(v, x);
-    } else {
-        const uint2 v = *reinterpret_cast<const uint2 *>(p);
-        unpack_e4m3x8(v, x);
-    }
-}
-
-// Two adjacent elements (dims 2i, 2i+1) of a record in shared memory.
-template <int ELEM>
-__device__ __forceinline__ float2 smem_elems2(const char *p) {
-    if (ELEM == 2) {
-        const uint32_t w = *reinterpret_cast<const uint32_t *>(p);
-        return make_float2(bf16lo(w), bf16hi(w));
-    }
-    return e4m3x2_to_float2(*reinterpret_cast<const uint16_t *>(p));
-}
-
-template <int ELEM, int D, int GB>
-struct AttnSmem {
-    static constexpr int RB = D * ELEM;           // record bytes
-    static constexpr int RS = RB + 16;            // padded row stride
-    static constexpr int TK = RB <= 256 ? 64 : 32;  // keys per tile
-    static constexpr int NKH = TK / 32;           // 32-key halves of a tile (QK)
-    static constexpr int NDQ = 8 / NKH;           // head-dim slices (QK)
-    static constexpr int KV = TK * RS;            // one tile of K or V
-    static constexpr int off_k = 0;               // [2][KV]
-    static constexpr int off_v = 2 * KV;          // [2][KV]
-    static constexpr int off_q = 4 * KV;          // float [GB][D]
-    static constexpr int off_red = off_q + GB * D * 4;            // float [NDQ][GB][TK] (also [G][D] at the end)
-    static constexpr int off_sc = off_red + NDQ * GB * TK * 4;    // float [GB][TK]
-    static constexpr int off_alpha = off_sc + GB * TK * 4;        // float [GB]
-    static constexpr int bytes = off_alpha + GB * 4;
-    static_assert(NDQ * GB * TK >= GB * D, "the final [G][D] sum reuses the QK partial buffer");
-};
-
-template <int ELEM, int D, int GB, bool PAGED>
-__global__ void __launch_bounds__(kAttnThreads) attn_partial_simt(const AttnParams p) {
-    using SM = AttnSmem<ELEM, D, GB>;
-    constexpr int RB = SM::RB, RS = SM::RS, TK = SM::TK, NDQ = SM::NDQ;
-    constexpr int CPR = RB / 16;              // 16-byte chunks per record
-    constexpr int DW = D / NDQ;               // dims per warp in QK
-    constexpr int NDP = D / 2;                // dim pairs
-    constexpr int NKG = kAttnThreads / NDP;   // key groups in PV
-    constexpr int KPG = TK / NKG;             // keys per group per tile
-    extern __shared__ __align__(16) char smem[];
-    char *sK = smem + SM::off_k;
-    char *sV = smem + SM::off_v;
-    float *qs = reinterpret_cast<float *>(smem + SM::off_q);
-    float *red = reinterpret_cast<float *>(smem + SM::off_red);
-    float *sc = reinterpret_cast<float *>(smem + SM::off_sc);
-    float *alpha = reinterpret_cast<float *>(smem + SM::off_alpha);
-
-    const Geometry &geo = p.geo;
-    const int G = geo.G;
-    const int nc = p.chunks;
-    const int64_t r = blockIdx.x / nc;
-    const int chunk = (int)(blockIdx.x % nc);
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int h = (int)(r % geo.H);
-    const int s = (int)((r / geo.H) % geo.S);
-    const int l = (int)(r / ((int64_t)geo.H * geo.S));
-    int64_t lo = geo.row_off[r], hi = geo.row_off[r + 1];
-    if (lo < 0 || hi < lo || hi > geo.total) {
-        if (t == 0 && chunk == 0) atomicOr(p.flags, TRI_FLAG_ROW_OFFSETS);
-        lo = hi = 0;
-    }
-    const int64_t n = hi - lo;
-    const int64_t beg = n * chunk / nc, end = n * (chunk + 1) / nc;  // slots in the row
-    const int32_t *table = geo.block_table + (int64_t)s * geo.max_blocks;
-    const int64_t layer_blk = (int64_t)l * geo.n_blocks;
-
-    // Scaled queries of this KV head's G query heads.
-    const uint16_t *qrow = p.q + (((int64_t)l * geo.S + s) * geo.Hq + (int64_t)h * G) * D;
-    for (int i = t; i < G * D; i += kAttnThreads)
-        qs[i] = __uint_as_float((uint32_t)qrow[i] << 16) * p.scale_log2;
-
-    // Issue the cp.async copies of the tile starting at slot j0 into buffer b.
-    auto load_tile = [&](int64_t j0, int b) {
-        const int cnt = (int)min((int64_t)TK, end - j0);
-        for (int i = t; i < 2 * TK * CPR; i += kAttnThreads) {
-            const int rec = i / CPR, part = i % CPR;
-            const int key = rec % TK;
-            const bool isv = rec >= TK;
-            if (key >= cnt) continue;
-            const int64_t j = j0 + key;
-            int64_t src = PAGED ? paged_record(geo, table, layer_blk, h, j) : lo + j;
-            if (src < 0) {
-                if (part == 0 && !isv) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
-                src = -1;
-            }
-            char *dst = (isv ? sV : sK) + b * SM::KV + key * RS + 16 * part;
-            if (src >= 0) cp_async16(dst, (isv ? p.V : p.K) + src * RB + 16 * part);
-            else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        cp_async_commit();
-    };
-
-    float acc[GB][2];
-#pragma unroll
-    for (int g = 0; g < GB; g++) acc[g][0] = acc[g][1] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f;  // of query `warp` (and warp + 8), kept by that warp
-    float m_run2 = -INFINITY, l_run2 = 0.f;
-
-    const int ntiles = (int)((end - beg + TK - 1) / TK);
-    if (ntiles > 0) load_tile(beg, 0);
-    for (int it = 0; it < ntiles; it++) {
-        const int b = it & 1;
-        const int64_t j0 = beg + (int64_t)it * TK;
-        const int cnt = (int)min((int64_t)TK, end - j0);
-        if (it + 1 < ntiles) {
-            load_tile(j0 + TK, b ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        // QK partials: key = 32 * (warp % NKH) + lane, dims [dq * DW, (dq + 1) * DW).
-        {
-            const int key = 32 * (warp % SM::NKH) + lane, dq = warp / SM::NKH;
-            float sp[GB];
-#pragma unroll
-            for (int g = 0; g < GB; g++) sp[g] = 0.f;
-            const char *krow = sK + b * SM::KV + key * RS;
-#pragma unroll
-            for (int c = 0; c < DW / 8; c++) {
-                const int d0 = dq * DW + 8 * c;
-                float x[8];
-                smem_elems8<ELEM>(krow + d0 * ELEM, x);
-#pragma unroll
-                for (int g = 0; g < GB; g++) {
-                    if (g < G) {
-                        const float4 qa = *reinterpret_cast<const float4 *>(qs + g * D + d0);
-                        const float4 qb = *reinterpret_cast<const float4 *>(qs + g * D + d0 + 4);
-                        float a = sp[g];
-                        a = fmaf(x[0], qa.x, a); a = fmaf(x[1], qa.y, a); a = fmaf(x[2], qa.z, a); a = fmaf(x[3], qa.w, a);
-                        a = fmaf(x[4], qb.x, a); a = fmaf(x[5], qb.y, a); a = fmaf(x[6], qb.z, a); a = fmaf(x[7], qb.w, a);
-                        sp[g] = a;
-                    }
-                }
-            }
-#pragma unroll
-            for (int g = 0; g < GB; g++)
-                if (g < G) red[(dq * GB + g) * TK + key] = sp[g];
-        }
-        __syncthreads();
-        for (int i = t; i < G * TK; i += kAttnThreads) {
-            const int g = i / TK, key = i % TK;
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < NDQ; w++) v += red[(w * GB + g) * TK + key];
-            sc[g * TK + key] = key < cnt ? v : -INFINITY;
-        }
-        __syncthreads();
-        // Online softmax, base 2: warp w handles queries w and w + 8.
-#pragma unroll
-        for (int rep = 0; rep < 2; rep++) {
-            const int g = warp + 8 * rep;
-            if (g < G) {
-                float v[SM::NKH];
-                float mt = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < SM::NKH; k++) {
-                    v[k] = sc[g * TK + 32 * k + lane];
-                    mt = fmaxf(mt, v[k]);
-                }
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
-                float &mr = rep ? m_run2 : m_run;
-                float &lr = rep ? l_run2 : l_run;
-                const float mn = fmaxf(mr, mt);
-                float ps = 0.f;
-#pragma unroll
-                for (int k = 0; k < SM::NKH; k++) {
-                    const float pv = exp2f(v[k] - mn);
-                    sc[g * TK + 32 * k + lane] = pv;
-                    ps += pv;
-                }
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-                const float a = exp2f(mr - mn);
-                lr = lr * a + ps;
-                mr = mn;
-                if (lane == 0) alpha[g] = a;
-            }
-        }
-        __syncthreads();
-        // PV: thread = (key group kg, dim pair dp) over the group's keys of the tile.
-        {
-            const int dp = t % NDP, kg = t / NDP;
-#pragma unroll
-            for (int g = 0; g < GB; g++) {
-                if (g < G) {
-                    const float a = alpha[g];
-                    acc[g][0] *= a;
-                    acc[g][1] *= a;
-                }
-            }
-            const char *vb = sV + b * SM::KV + 2 * dp * ELEM;
-            for (int kk = 0; kk < KPG; kk++) {
-                const int key = kg * KPG + kk;
-                if (key >= cnt) break;
-                const float2 v2 = smem_elems2<ELEM>(vb + key * RS);
-#pragma unroll
-                for (int g = 0; g < GB; g++) {
-                    if (g < G) {
-                        const float pr = sc[g * TK + key];
-                        acc[g][0] = fmaf(pr, v2.x, acc[g][0]);
-                        acc[g][1] = fmaf(pr, v2.y, acc[g][1]);
-                    }
-                }
-            }
-        }
-        __syncthreads();  // buffer b is refilled by the load issued in the next iteration
-    }
-
-    // Add the key groups' accumulators in order (group 0 first), then write the slice.
-    {
-        const int dp = t % NDP, kg = t / NDP;
-        float *buf = red;  // [G][D]
-        for (int k = 0; k < NKG; k++) {
-            if (kg == k) {
-#pragma unroll
-                for (int g = 0; g < GB; g++) {
-                    if (g < G) {
-                        if (k == 0) {
-                            buf[g * D + 2 * dp] = acc[g][0];
-                            buf[g * D + 2 * dp + 1] = acc[g][1];
-                        } else {
-                            buf[g * D + 2 * dp] += acc[g][0];
-                            buf[g * D + 2 * dp + 1] += acc[g][1];
-                        }
-                    }
-                }
-            }
-            __syncthreads();
-        }
-        float *out = p.part + ((r * nc + chunk) * (int64_t)G) * (D + 2);
-        for (int i = t; i < G * D; i += kAttnThreads) out[(i / D) * (D + 2) + (i % D)] = buf[i];
-#pragma unroll
-        for (int rep = 0; rep < 2; rep++) {
-            const int g = warp + 8 * rep;
-            if (g < G && lane == 0) {
-                out[g * (D + 2) + D] = rep ? m_run2 : m_run;
-                out[g * (D + 2) + D + 1] = rep ? l_run2 : l_run;
-            }
-        }
-    }
-}
-
 // ------------------------------------------------ tensor-core slice kernel
 //
-// For d <= 128: warp-level MMAs (mma.sync m16n8k16, fp32 accumulation) with the
-// G <= 16 queries as the 16 rows of the A operand.  The op is HBM-bound, so the
+// Warp-level MMAs (mma.sync m16n8k16, fp32 accumulation) with the G <= 16
+// queries as the 16 rows of the A operand (head dim 256: a warp pair per item,
+// see MmaSmem).  The op is HBM-bound, so the
 // tensor pipe only takes the multiply-adds off the CUDA cores.  (The transposed
 // form, keys on the 128-row M side of tcgen05.mma and the queries on N, is the
 // kernel of attention_tc.cu; on the same caches it is slower than this one,
@@ -377,13 +112,22 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
     return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
+// Head dim 256: a pair of warps shares each work item, warp h of the pair
+// holding dims [128 h, 128 h + 128) of Q, K, V and O (so its fragments are those
+// of a d = 128 warp); the two halves of every S tile are added through shared
+// memory (a 64-thread named barrier per tile) before the softmax, which both
+// warps then run on the same values.
 template <int ELEM, int D>
 struct MmaSmem {
-    static constexpr int RB = D * ELEM;                  // record bytes
+    static constexpr bool PAIR = D > 128;                // two warps per item
+    static constexpr int DW = PAIR ? D / 2 : D;          // dims per warp
+    static constexpr int RB = DW * ELEM;                 // a warp's bytes of a record
     static constexpr int RS = RB + 16;                   // padded row stride of a K/V tile
     static constexpr int TILE = kMmaKeys * RS;           // one 16-key tile of K or V
     static constexpr int WARP = 2 * 2 * TILE;            // per warp: 2 stages x (K, V)
-    static constexpr int bytes = kMmaWarps * WARP;
+    static constexpr int XCH = PAIR ? 2 * 32 * 8 * 4 : 0;  // per warp: S halves [2 tiles][32 lanes][8]
+    static constexpr int WPI = PAIR ? 2 : 1;             // warps per work item
+    static constexpr int bytes = kMmaWarps * (WARP + XCH);
 };
 
 // One work item: slice `c` of row `r`, keys [beg, end) of the row.
@@ -418,17 +162,23 @@ template <int ELEM, int D, bool PAGED>
 __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams p) {
     using SM = MmaSmem<ELEM, D>;
     constexpr bool F16 = ELEM == 1;
+    constexpr bool PAIR = SM::PAIR;
+    constexpr int DW = SM::DW, WPI = SM::WPI;
     constexpr int RB = SM::RB, RS = SM::RS, CPR = RB / 16;
-    constexpr int KS = D / 16;  // k-steps of QK
-    constexpr int NT = D / 8;   // output n-tiles of PV
-    constexpr int KPI = 16 / CPR;  // keys per copy instruction (K and V of each)
+    constexpr int RBG = D * ELEM;   // record bytes in the cache
+    constexpr int KS = DW / 16;     // k-steps of QK (this warp's dims)
+    constexpr int NT = DW / 8;      // output n-tiles of PV (this warp's dims)
+    constexpr int KPI = 16 / CPR;   // keys per copy instruction (K and V of each)
     extern __shared__ __align__(16) char smem[];
     const Geometry &geo = p.geo;
     const int G = geo.G;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t nwork = (int64_t)gridDim.x * kMmaWarps;
+    const int half = PAIR ? (warp & 1) : 0;  // which dims of the item this warp holds
+    const int dw0 = half * DW;               // its first dim
+    const int64_t nwork = (int64_t)gridDim.x * (kMmaWarps / WPI);
     const int64_t items = (int64_t)geo.L * geo.S * geo.H * p.chunks;
     char *wbuf = smem + warp * SM::WARP;  // [stage][K, V][16 keys][RS]
+    float *xch = reinterpret_cast<float *>(smem + kMmaWarps * SM::WARP);  // [warp][2][32][8]
     const float sl2 = p.scale_log2;
 
     // Copy tile `ti` of item `a` into stage `st`: lane i < 16 finds the record of
@@ -447,22 +197,23 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
                 my_rec = a.lo + j0 + lane;
             }
         }
-        const int half = lane >> 4, c16 = lane & 15;
+        const int kv = lane >> 4, c16 = lane & 15;
         const int sub = c16 / CPR, part = c16 % CPR;
-        const char *base = half ? p.V : p.K;
+        const char *base = (kv ? p.V : p.K) + dw0 * ELEM;
 #pragma unroll
         for (int i = 0; i < kMmaKeys / KPI; i++) {
             const int key = i * KPI + sub;
             const int64_t rec = __shfl_sync(0xffffffffu, my_rec, key);
-            char *dst = wbuf + (st * 2 + half) * SM::TILE + key * RS + 16 * part;
-            if (rec >= 0) cp_async16(dst, base + rec * RB + 16 * part);
+            char *dst = wbuf + (st * 2 + kv) * SM::TILE + key * RS + 16 * part;
+            if (rec >= 0) cp_async16(dst, base + rec * RBG + 16 * part);
             else *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);  // finite zeros past the end
         }
         cp_async_commit();
     };
 
-    // The warp's stream of (item, tile) pairs: items wid, wid + nwork, ...
-    int64_t item = (int64_t)blockIdx.x * kMmaWarps + warp;
+    // The warp's stream of (item, tile) pairs: items wid, wid + nwork, ... (both
+    // warps of a pair take the same stream, so their control flow is the same).
+    int64_t item = (int64_t)blockIdx.x * (kMmaWarps / WPI) + warp / WPI;
     AttnItem cur;
     cur.ntiles = 0;
     // Advance `item` to the next one with tiles, writing empty results for empty items.
@@ -471,7 +222,8 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
             a = attn_item(p, i, p.flags, lane == 0 && (i % p.chunks) == 0);
             if (a.ntiles > 0) return i;
             float *out = p.part + (i * (int64_t)G) * (D + 2);  // an empty slice: m = -inf, l = 0, O = 0
-            for (int k = lane; k < G * (D + 2); k += 32) out[k] = (k % (D + 2)) == D ? -INFINITY : 0.f;
+            if (half == 0)
+                for (int k = lane; k < G * (D + 2); k += 32) out[k] = (k % (D + 2)) == D ? -INFINITY : 0.f;
         }
         return items;
     };
@@ -494,7 +246,7 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
                     const int g = (e & 1) ? g1 : g0;
-                    const int dim = ks * 16 + kc + ((e & 2) ? 8 : 0);
+                    const int dim = dw0 + ks * 16 + kc + ((e & 2) ? 8 : 0);
                     uint32_t w = 0u;
                     if (g < G) {
                         const uint32_t raw = (uint32_t)qrow[(int64_t)g * D + dim] | ((uint32_t)qrow[(int64_t)g * D + dim + 1] << 16);
@@ -545,6 +297,22 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
             }
             mma16816<F16>(sc[0], qf[ks], b[0], b[1]);
             mma16816<F16>(sc[1], qf[ks], b[2], b[3]);
+        }
+        if constexpr (PAIR) {
+            // S = (dims 0-127 part) + (dims 128-255 part), added in that order by both
+            // warps of the pair: the halves meet in shared memory (double-buffered by
+            // tile parity, so one barrier per tile keeps a buffer from being rewritten
+            // before the partner has read it).
+            float *mine = xch + ((warp * 2 + st) * 32 + lane) * 8;
+            const float *other = xch + (((warp ^ 1) * 2 + st) * 32 + lane) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; e++) mine[e] = sc[e >> 2][e & 3];
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp >> 1)) : "memory");
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                const float ov = other[e];
+                sc[e >> 2][e & 3] = half == 0 ? sc[e >> 2][e & 3] + ov : ov + sc[e >> 2][e & 3];
+            }
         }
         // ---- scale to base 2, mask keys past the slice (partial tiles only), online softmax per row
         const int kc = 2 * (lane & 3);
@@ -638,15 +406,15 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
 #pragma unroll
             for (int i = 0; i < NT; i++) {
                 if (g0 < G) {
-                    out[g0 * (D + 2) + i * 8 + c0] = o[i][0];
-                    out[g0 * (D + 2) + i * 8 + c0 + 1] = o[i][1];
+                    out[g0 * (D + 2) + dw0 + i * 8 + c0] = o[i][0];
+                    out[g0 * (D + 2) + dw0 + i * 8 + c0 + 1] = o[i][1];
                 }
                 if (g1 < G) {
-                    out[g1 * (D + 2) + i * 8 + c0] = o[i][2];
-                    out[g1 * (D + 2) + i * 8 + c0 + 1] = o[i][3];
+                    out[g1 * (D + 2) + dw0 + i * 8 + c0] = o[i][2];
+                    out[g1 * (D + 2) + dw0 + i * 8 + c0 + 1] = o[i][3];
                 }
             }
-            if ((lane & 3) == 0) {
+            if ((lane & 3) == 0 && half == 0) {
                 if (g0 < G) {
                     out[g0 * (D + 2) + D] = m0;
                     out[g0 * (D + 2) + D + 1] = s0;
@@ -697,32 +465,6 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const AttnParams p) {
     if (p.lse && dim == 0) p.lse[qi] = den > 0.f ? (m + log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int ELEM, int D, int GB, bool PAGED>
-static cudaError_t launch_attn_t(const AttnParams &p0, int64_t R, cudaStream_t s) {
-    using SM = AttnSmem<ELEM, D, GB>;
-    auto kern = attn_partial_simt<ELEM, D, GB, PAGED>;
-    static int occ[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    int &o = occ[dev & 63];
-    if (o == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::bytes);
-        if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kAttnThreads, SM::bytes);
-        if (e != cudaSuccess) return e;
-        if (o < 1) o = 1;
-    }
-    // About one wave: enough slices per row to give every SM its resident CTAs.
-    AttnParams p = p0;
-    const int64_t slots = (int64_t)sm_count() * o;
-    p.chunks = (int)std::min<int64_t>(kAttnMaxChunks, std::max<int64_t>(1, (slots + R - 1) / R));
-    kern<<<(unsigned)(R * p.chunks), kAttnThreads, SM::bytes, s>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    attn_combine_kernel<D><<<(unsigned)(R * p.geo.G), D, 0, s>>>(p);
-    return cudaGetLastError();
-}
-
 template <int ELEM, int D, bool PAGED>
 static cudaError_t launch_attn_mma(const AttnParams &p0, int64_t R, cudaStream_t s) {
     using SM = MmaSmem<ELEM, D>;
@@ -743,9 +485,10 @@ static cudaError_t launch_attn_mma(const AttnParams &p0, int64_t R, cudaStream_t
     // and read back, so more slices than that only add traffic).
     AttnParams p = p0;
     const int64_t ctas = (int64_t)sm_count() * o;
-    const int64_t workers = ctas * kMmaWarps;
+    const int64_t per_cta = kMmaWarps / SM::WPI;  // workers per CTA (a warp, or a warp pair)
+    const int64_t workers = ctas * per_cta;
     p.chunks = (int)std::min<int64_t>(kAttnMaxChunks, std::max<int64_t>(1, (2 * workers + R - 1) / R));
-    const int64_t grid = std::min<int64_t>(ctas, (R * p.chunks + kMmaWarps - 1) / kMmaWarps);
+    const int64_t grid = std::min<int64_t>(ctas, (R * p.chunks + per_cta - 1) / per_cta);
     kern<<<(unsigned)grid, kMmaThreads, SM::bytes, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -755,10 +498,7 @@ static cudaError_t launch_attn_mma(const AttnParams &p0, int64_t R, cudaStream_t
 
 template <int ELEM, int D, bool PAGED>
 static cudaError_t launch_attn_g(const AttnParams &p, int64_t R, cudaStream_t s) {
-    if (D <= 128) return launch_attn_mma<ELEM, (D <= 128 ? D : 128), PAGED>(p, R, s);
-    if (p.geo.G <= 4) return launch_attn_t<ELEM, D, 4, PAGED>(p, R, s);
-    if (p.geo.G <= 8) return launch_attn_t<ELEM, D, 8, PAGED>(p, R, s);
-    return launch_attn_t<ELEM, D, 16, PAGED>(p, R, s);
+    return launch_attn_mma<ELEM, D, PAGED>(p, R, s);
 }
 
 template <int ELEM, bool PAGED>

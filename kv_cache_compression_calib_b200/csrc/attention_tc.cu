@@ -2,7 +2,8 @@
 // KV 压缩的高效长推理", 流程详解 step 5: later attention steps read only the
 // compressed cache).  For bf16 caches of head dim 128 in the contiguous layout
 // (the [R][B] output of tri_compact, or any contiguous cache) and G <= 16
-// queries per KV head; the other cases take attn_partial_mma / _simt.
+// queries per KV head (tri_decode_attention_tc); tri_decode_attention runs
+// attn_partial_mma, which serves every case and measured faster on these.
 //
 // The contraction is transposed so the keys, not the few queries, fill the
 // 128-row tile of tcgen05.mma:
