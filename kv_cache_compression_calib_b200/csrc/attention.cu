@@ -180,6 +180,8 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
     char *wbuf = smem + warp * SM::WARP;  // [stage][K, V][16 keys][RS]
     float *xch = reinterpret_cast<float *>(smem + kMmaWarps * SM::WARP);  // [warp][2][32][8]
     const float sl2 = p.scale_log2;
+    grid_dependency_wait();  // the cache may come from the compaction just before
+    grid_dependents_launch();
 
     // Copy tile `ti` of item `a` into stage `st`: lane i < 16 finds the record of
     // key i once; every instruction then moves whole records, half the warp on K
@@ -246,7 +248,10 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
                     const int g = (e & 1) ? g1 : g0;
-                    const int dim = dw0 + ks * 16 + kc + ((e & 2) ? 8 : 0);
+                    // fp8 caches: k index 2c + e' (+8) of k-step ks holds dim
+                    // c DW/4 + 4 ks + e' (+2), c = lane % 4 (see the fp8 fragments below)
+                    const int dim = F16 ? dw0 + (lane & 3) * (DW / 4) + 4 * ks + ((e & 2) ? 2 : 0)
+                                        : dw0 + ks * 16 + kc + ((e & 2) ? 8 : 0);
                     uint32_t w = 0u;
                     if (g < G) {
                         const uint32_t raw = (uint32_t)qrow[(int64_t)g * D + dim] | ((uint32_t)qrow[(int64_t)g * D + dim + 1] << 16);
@@ -280,20 +285,37 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
         const char *kt = wbuf + (st * 2) * SM::TILE;
         const char *vt = wbuf + (st * 2 + 1) * SM::TILE;
         // ---- S = Q K^T for keys 0-7 (sc[0]) and 8-15 (sc[1])
+        // fp8 caches take the dims of the contraction in a permuted order (the sum
+        // is the same for any order that Q and K share): lane c = lane % 4 holds,
+        // over all k-steps, the DW/4 consecutive dims c DW/4 .. of its keys, so it
+        // reads them with 16-byte loads; k-step ks uses the key's bytes 4 ks .. 4 ks + 3.
+        uint32_t kw[2][F16 ? DW / 16 : 1];
+        if constexpr (F16) {
+            const char *k0p = kt + (lane >> 2) * RS + (lane & 3) * (DW / 4);
+#pragma unroll
+            for (int kk = 0; kk < 2; kk++)
+#pragma unroll
+                for (int v = 0; v < DW / 64; v++) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(k0p + kk * 8 * RS + 16 * v);
+                    kw[kk][4 * v] = w.x;
+                    kw[kk][4 * v + 1] = w.y;
+                    kw[kk][4 * v + 2] = w.z;
+                    kw[kk][4 * v + 3] = w.w;
+                }
+        }
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int ks = 0; ks < KS; ks++) {
             uint32_t b[4];  // b0, b1 of keys 0-7, then of keys 8-15
-            if (!F16) {
+            if constexpr (!F16) {
                 const int mi = lane >> 3, i = lane & 7;
                 const int key = i + 8 * (mi >> 1), dim = ks * 16 + 8 * (mi & 1);
                 ldsm_x4(b, kt + key * RS + dim * 2);
             } else {
-                const int key = lane >> 2, dim = ks * 16 + 2 * (lane & 3);
-                b[0] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t *>(kt + key * RS + dim));
-                b[1] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t *>(kt + key * RS + dim + 8));
-                b[2] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t *>(kt + (key + 8) * RS + dim));
-                b[3] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t *>(kt + (key + 8) * RS + dim + 8));
+                b[0] = e4m3x2_to_f16x2(kw[0][ks]);
+                b[1] = e4m3x2_to_f16x2(kw[0][ks] >> 16);
+                b[2] = e4m3x2_to_f16x2(kw[1][ks]);
+                b[3] = e4m3x2_to_f16x2(kw[1][ks] >> 16);
             }
             mma16816<F16>(sc[0], qf[ks], b[0], b[1]);
             mma16816<F16>(sc[1], qf[ks], b[2], b[3]);
@@ -370,29 +392,50 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
                 pl[i] = pack2<F16>(src[i][0] - back.x, src[i][1] - back.y);
             }
         }
-        // ---- O += P V, two n-tiles of 8 dims per step
+        // ---- O += P V
+        if constexpr (!F16) {
+            // two n-tiles of 8 dims per step
 #pragma unroll
-        for (int dt = 0; dt < NT; dt += 2) {
-            uint32_t b[4];  // b0, b1 of dims dt*8.., then of dims (dt+1)*8..
-            if (!F16) {
+            for (int dt = 0; dt < NT; dt += 2) {
+                uint32_t b[4];  // b0, b1 of dims dt*8.., then of dims (dt+1)*8..
                 const int mi = lane >> 3, i = lane & 7;
                 const int key = i + 8 * (mi & 1), dim = (dt + (mi >> 1)) * 8;
                 ldsm_x4_t(b, vt + key * RS + dim * 2);
-            } else {
-                const int key = 2 * (lane & 3), dim = lane >> 2;
+                mma16816<F16>(o[dt], ph, b[0], b[1]);
+                mma16816<F16>(o[dt], pl, b[0], b[1]);
+                mma16816<F16>(o[dt + 1], ph, b[2], b[3]);
+                mma16816<F16>(o[dt + 1], pl, b[2], b[3]);
+            }
+        } else {
+            // fp8: column n of n-tile j is dim n NT + j, so lane (n = lane / 4) reads
+            // the NT consecutive bytes n NT .. of each of its keys 2c, 2c+1, 2c+8,
+            // 2c+9 once, and pairs the keys' bytes of dim n NT + j with a byte permute.
+            uint32_t vw[4][NT / 4];
+            const int key = 2 * (lane & 3);
+            const char *vp = vt + key * RS + (lane >> 2) * NT;
 #pragma unroll
-                for (int hh = 0; hh < 2; hh++) {
-                    const int dd = (dt + hh) * 8 + dim;
-                    const uint32_t k0 = (uint8_t)vt[key * RS + dd], k1 = (uint8_t)vt[(key + 1) * RS + dd];
-                    const uint32_t k8 = (uint8_t)vt[(key + 8) * RS + dd], k9 = (uint8_t)vt[(key + 9) * RS + dd];
-                    b[2 * hh] = e4m3x2_to_f16x2(k0 | (k1 << 8));
-                    b[2 * hh + 1] = e4m3x2_to_f16x2(k8 | (k9 << 8));
+            for (int r = 0; r < 4; r++) {
+                const char *row = vp + ((r & 1) + 8 * (r >> 1)) * RS;
+                if constexpr (NT == 16) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(row);
+                    vw[r][0] = w.x;
+                    vw[r][1] = w.y;
+                    vw[r][2] = w.z;
+                    vw[r][3] = w.w;
+                } else {
+                    const uint2 w = *reinterpret_cast<const uint2 *>(row);
+                    vw[r][0] = w.x;
+                    vw[r][1] = w.y;
                 }
             }
-            mma16816<F16>(o[dt], ph, b[0], b[1]);
-            mma16816<F16>(o[dt], pl, b[0], b[1]);
-            mma16816<F16>(o[dt + 1], ph, b[2], b[3]);
-            mma16816<F16>(o[dt + 1], pl, b[2], b[3]);
+#pragma unroll
+            for (int j = 0; j < NT; j++) {
+                const uint32_t sel = (uint32_t)(j & 3) | ((uint32_t)(4 + (j & 3)) << 4);
+                const uint32_t b0 = e4m3x2_to_f16x2(__byte_perm(vw[0][j >> 2], vw[1][j >> 2], sel));
+                const uint32_t b1 = e4m3x2_to_f16x2(__byte_perm(vw[2][j >> 2], vw[3][j >> 2], sel));
+                mma16816<F16>(o[j], ph, b0, b1);
+                mma16816<F16>(o[j], pl, b0, b1);
+            }
         }
         __syncwarp();  // this stage is refilled by the prefetch after next
         if (tile + 1 == cur.ntiles) {
@@ -405,13 +448,16 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
             const int g0 = lane >> 2, g1 = g0 + 8, c0 = 2 * (lane & 3);
 #pragma unroll
             for (int i = 0; i < NT; i++) {
+                // column c of n-tile i: dim i 8 + c (bf16), dim c NT + i (fp8, permuted)
+                const int d0 = dw0 + (F16 ? c0 * NT + i : i * 8 + c0);
+                const int d1 = dw0 + (F16 ? (c0 + 1) * NT + i : i * 8 + c0 + 1);
                 if (g0 < G) {
-                    out[g0 * (D + 2) + dw0 + i * 8 + c0] = o[i][0];
-                    out[g0 * (D + 2) + dw0 + i * 8 + c0 + 1] = o[i][1];
+                    out[g0 * (D + 2) + d0] = o[i][0];
+                    out[g0 * (D + 2) + d1] = o[i][1];
                 }
                 if (g1 < G) {
-                    out[g1 * (D + 2) + dw0 + i * 8 + c0] = o[i][2];
-                    out[g1 * (D + 2) + dw0 + i * 8 + c0 + 1] = o[i][3];
+                    out[g1 * (D + 2) + d0] = o[i][2];
+                    out[g1 * (D + 2) + d1] = o[i][3];
                 }
             }
             if ((lane & 3) == 0 && half == 0) {
@@ -437,6 +483,7 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
 // Merge a row's slices: one CTA of D threads per (row, query of the group).
 template <int D>
 __global__ void __launch_bounds__(D) attn_combine_kernel(const AttnParams p) {
+    grid_dependency_wait();
     const Geometry &geo = p.geo;
     const int G = geo.G;
     const int nc = p.chunks;
@@ -480,20 +527,33 @@ static cudaError_t launch_attn_mma(const AttnParams &p0, int64_t R, cudaStream_t
         if (e != cudaSuccess) return e;
         if (o < 1) o = 1;
     }
-    // Persistent grid of the resident CTAs; rows cut into enough slices that every
-    // warp gets about two work items (each slice costs (d + 2) G floats written
-    // and read back, so more slices than that only add traffic).
+    // Persistent grid of the resident CTAs; rows cut into c slices, the workers
+    // taking items round-robin.  At most about two items per worker (each slice
+    // adds (d + 2) G floats written and read back, and a few dependent loads per
+    // item); within that, the slowest worker streams ceil(R c / workers) items of
+    // about keys/(R c) keys each plus a fixed cost per item, and c minimises that
+    // (the smallest such c): a last round that keeps few workers busy is avoided.
     AttnParams p = p0;
     const int64_t ctas = (int64_t)sm_count() * o;
     const int64_t per_cta = kMmaWarps / SM::WPI;  // workers per CTA (a warp, or a warp pair)
     const int64_t workers = ctas * per_cta;
-    p.chunks = (int)std::min<int64_t>(kAttnMaxChunks, std::max<int64_t>(1, (2 * workers + R - 1) / R));
+    const int64_t keys_per_row = std::max<int64_t>(1, p.geo.total / R);
+    const int c_max = (int)std::min<int64_t>(kAttnMaxChunks, std::max<int64_t>(1, (2 * workers + R - 1) / R));
+    int64_t best = -1;
+    p.chunks = 1;
+    for (int c = 1; c <= c_max; c++) {
+        const int64_t rounds = (R * c + workers - 1) / workers;
+        const int64_t tiles = (keys_per_row + (int64_t)c * kMmaKeys - 1) / ((int64_t)c * kMmaKeys);
+        const int64_t cost = rounds * (tiles + 2);
+        if (best < 0 || cost < best) {
+            best = cost;
+            p.chunks = c;
+        }
+    }
     const int64_t grid = std::min<int64_t>(ctas, (R * p.chunks + per_cta - 1) / per_cta);
-    kern<<<(unsigned)grid, kMmaThreads, SM::bytes, s>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(kern, dim3((unsigned)grid), dim3(kMmaThreads), SM::bytes, s, p);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<D><<<(unsigned)(R * p.geo.G), D, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(attn_combine_kernel<D>, dim3((unsigned)(R * p.geo.G)), dim3(D), 0, s, p);
 }
 
 template <int ELEM, int D, bool PAGED>

@@ -69,15 +69,21 @@ def test_attention_contig(d, style, elem, hq):
             check_row(out[0, s, qh], lse[0, s, qh], qf[0, s, qh], K[a:b], V[a:b], scale, (r, g))
 
 
-def test_attention_paged():
-    wl = synth.WORKLOADS["paged_16seq"].with_(name="attp", batch=3, n_calib=8)
+@pytest.mark.parametrize("d,elem", [(128, "bf16"), (256, "bf16"), (64, "fp8"), (256, "fp8")])
+def test_attention_paged(d, elem):
+    """Paged caches (shuffled block table), ragged rows; head dim 256 runs the
+    warp-pair form of the MMA kernel, fp8 its permuted-dim fragments."""
+    wl = synth.WORKLOADS["paged_16seq"].with_(name=f"attp{d}{elem}", batch=3, n_calib=8, head_dim=d,
+                                             theta=1e6 if d == 128 else 1e4)
     lens = np.array([300, 2100, 17])
     p = synth.make_paged(wl, "cpu", lens=lens)
-    S, Hh, bs, d = len(lens), wl.n_kv_heads, wl.block_size, 128
+    if elem == "fp8":
+        p.K, p.V = synth.to_fp8(p.K), synth.to_fp8(p.V)
+    S, Hh, bs = len(lens), wl.n_kv_heads, wl.block_size
     row_off = synth.paged_row_offsets(lens, Hh)
     m = model_of(wl, 1)
     kv = tri.kv_paged(S, torch.as_tensor(row_off, device=DEV), int(row_off[-1]), p.block_table.to(DEV), bs,
-                      p.K.shape[0])
+                      p.K.shape[0], tri.elem_type_of(p.K))
     q = synth.decode_queries(wl, 0, lens, "cpu")[None]
     scale = 1.0 / math.sqrt(d)
     out, lse = run_attention(m, kv, p.K.to(DEV), p.V.to(DEV), q.to(DEV).contiguous(), scale, S)
