@@ -124,7 +124,11 @@ struct MmaSmem {
     static constexpr int RB = DW * ELEM;                 // a warp's bytes of a record
     static constexpr int RS = RB + 16;                   // padded row stride of a K/V tile
     static constexpr int TILE = kMmaKeys * RS;           // one 16-key tile of K or V
-    static constexpr int WARP = 2 * 2 * TILE;            // per warp: 2 stages x (K, V)
+    // Tiles in flight per warp (one computed, STAGES - 1 loading).  Deeper rings
+    // measured no faster, for fp8 too (its tiles are half as long, but its time
+    // goes to the per-tile arithmetic, which is the same as for bf16).
+    static constexpr int STAGES = 2;
+    static constexpr int WARP = STAGES * 2 * TILE;       // per warp: STAGES x (K, V)
     static constexpr int XCH = PAIR ? 2 * 32 * 8 * 4 : 0;  // per warp: S halves [2 tiles][32 lanes][8]
     static constexpr int WPI = PAIR ? 2 : 1;             // warps per work item
     static constexpr int bytes = kMmaWarps * (WARP + XCH);
@@ -159,7 +163,7 @@ __device__ __forceinline__ AttnItem attn_item(const AttnParams &p, int64_t item,
 }
 
 template <int ELEM, int D, bool PAGED>
-__global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams p) {
+__global__ void __launch_bounds__(kMmaThreads, 3) attn_partial_mma(const AttnParams p) {
     using SM = MmaSmem<ELEM, D>;
     constexpr bool F16 = ELEM == 1;
     constexpr bool PAIR = SM::PAIR;
@@ -218,21 +222,49 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
     int64_t item = (int64_t)blockIdx.x * (kMmaWarps / WPI) + warp / WPI;
     AttnItem cur;
     cur.ntiles = 0;
-    // Advance `item` to the next one with tiles, writing empty results for empty items.
-    auto next_nonempty = [&](int64_t from, AttnItem &a) -> int64_t {
+    // Advance `item` to the next one with tiles; the prefetch cursor (first) writes
+    // the empty results of empty items on the way.
+    auto next_nonempty = [&](int64_t from, AttnItem &a, bool write_empty) -> int64_t {
         for (int64_t i = from; i < items; i += nwork) {
-            a = attn_item(p, i, p.flags, lane == 0 && (i % p.chunks) == 0);
+            a = attn_item(p, i, p.flags, write_empty && lane == 0 && (i % p.chunks) == 0);
             if (a.ntiles > 0) return i;
             float *out = p.part + (i * (int64_t)G) * (D + 2);  // an empty slice: m = -inf, l = 0, O = 0
-            if (half == 0)
+            if (write_empty && half == 0)
                 for (int k = lane; k < G * (D + 2); k += 32) out[k] = (k % (D + 2)) == D ? -INFINITY : 0.f;
         }
         return items;
     };
-    item = next_nonempty(item, cur);
+    // The next (item, tile) of the stream; false at its end.
+    auto advance = [&](int64_t &it, AttnItem &a, int &t, bool write_empty) -> bool {
+        if (t + 1 < a.ntiles) {
+            t++;
+            return true;
+        }
+        it = next_nonempty(it + nwork, a, write_empty);
+        t = 0;
+        return it < items;
+    };
+    item = next_nonempty(item, cur, true);
     if (item >= items) return;
-    int tile = 0, st = 0;
-    load_tile(cur, 0, 0);
+    int tile = 0;
+    // The prefetch cursor runs NS - 1 tiles ahead of the compute cursor, one
+    // cp.async group per tile (an empty group past the stream's end, so that
+    // waiting for all but the newest NS - 1 groups always means "this tile").
+    constexpr int NS = SM::STAGES;
+    int64_t pitem = item;
+    AttnItem pcur = cur;
+    int ptile = 0;
+    bool pmore = true;
+#pragma unroll
+    for (int k = 0; k < NS - 1; k++) {
+        if (pmore) {
+            load_tile(pcur, ptile, k);
+            pmore = advance(pitem, pcur, ptile, true);
+        } else {
+            cp_async_commit();
+        }
+    }
+    int ci = 0;  // tiles computed so far
 
     uint32_t qf[KS][4];
     float o[NT][4];
@@ -265,21 +297,15 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
             m0 = m1 = -INFINITY;
             l0 = l1 = 0.f;
         }
-        // Prefetch the next tile of the stream (this item's next, or the next item's first).
-        AttnItem nxt = cur;
-        int64_t nitem = item;
-        int ntile = tile + 1;
-        if (ntile >= cur.ntiles) {
-            nitem = next_nonempty(item + nwork, nxt);
-            ntile = 0;
-        }
-        const bool more = nitem < items;
-        if (more) {
-            load_tile(nxt, ntile, st ^ 1);
-            cp_async_wait<1>();
+        // Prefetch NS - 1 tiles ahead, into the stage computed in the previous step.
+        const int st = ci % NS;
+        if (pmore) {
+            load_tile(pcur, ptile, (ci + NS - 1) % NS);
+            pmore = advance(pitem, pcur, ptile, true);
         } else {
-            cp_async_wait<0>();
+            cp_async_commit();
         }
+        cp_async_wait<NS - 1>();
         __syncwarp();
         const int cnt = (int)min((int64_t)kMmaKeys, cur.end - (cur.beg + (int64_t)tile * kMmaKeys));
         const char *kt = wbuf + (st * 2) * SM::TILE;
@@ -325,8 +351,8 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
             // warps of the pair: the halves meet in shared memory (double-buffered by
             // tile parity, so one barrier per tile keeps a buffer from being rewritten
             // before the partner has read it).
-            float *mine = xch + ((warp * 2 + st) * 32 + lane) * 8;
-            const float *other = xch + (((warp ^ 1) * 2 + st) * 32 + lane) * 8;
+            float *mine = xch + ((warp * 2 + (ci & 1)) * 32 + lane) * 8;
+            const float *other = xch + (((warp ^ 1) * 2 + (ci & 1)) * 32 + lane) * 8;
 #pragma unroll
             for (int e = 0; e < 8; e++) mine[e] = sc[e >> 2][e & 3];
             asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp >> 1)) : "memory");
@@ -437,7 +463,7 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
                 mma16816<F16>(o[j], pl, b0, b1);
             }
         }
-        __syncwarp();  // this stage is refilled by the prefetch after next
+        __syncwarp();  // this stage is refilled by the next step's prefetch
         if (tile + 1 == cur.ntiles) {
             // Item done: row sums over the 4 lanes of each row, then (O, m, l) of rows < G.
             float s0 = l0 + __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -471,11 +497,8 @@ __global__ void __launch_bounds__(kMmaThreads) attn_partial_mma(const AttnParams
                 }
             }
         }
-        if (!more) break;
-        item = nitem;
-        cur = nxt;
-        tile = ntile;
-        st ^= 1;
+        if (!advance(item, cur, tile, false)) break;
+        ci++;
     }
     cp_async_wait<0>();
 }

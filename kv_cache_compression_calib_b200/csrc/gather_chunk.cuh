@@ -8,6 +8,45 @@
 
 namespace tri {
 
+// Source and destination records of kept slot i of row r (layer l, sequence
+// s, KV head h).  False for an entry the fused kernel emptied (-1) and for a
+// slot a block table cannot place (flagged by the lane with c == 0).
+__device__ __forceinline__ bool kept_record(const GatherParams &p, int64_t r, int64_t row_lo, int64_t N, int i, int h,
+                                            int s, int l, int c, int64_t &src, int64_t &dst) {
+    const Geometry &geo = p.geo;
+    const int64_t j = p.kept[r * p.B + i];
+    if (j == -1) return false;  // an entry the fused kernel emptied (its row was flagged there)
+    src = -1;
+    if (j >= 0 && j < N) {
+        if (geo.layout == TRI_KV_PAGED) {
+            const int64_t bi = j >> geo.block_shift;
+            const int32_t blk = bi < geo.max_blocks ? __ldg(geo.block_table + (int64_t)s * geo.max_blocks + bi) : -1;
+            if (blk >= 0 && blk < geo.n_blocks)
+                src = ((((int64_t)l * geo.n_blocks + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) *
+                          geo.H +
+                      h;
+        } else {
+            src = row_lo + j;
+        }
+    }
+    dst = -1;
+    if (p.out_layout == TRI_KV_PAGED) {
+        const int64_t bi = (int64_t)i >> p.out_block_shift;
+        const int32_t blk = bi < p.out_max_blocks ? __ldg(p.out_table + (int64_t)s * p.out_max_blocks + bi) : -1;
+        if (blk >= 0 && blk < p.out_n_blocks)
+            dst = ((((int64_t)l * p.out_n_blocks + blk) << p.out_block_shift) | (i & ((1 << p.out_block_shift) - 1))) *
+                      geo.H +
+                  h;
+    } else {
+        dst = r * p.B + i;
+    }
+    if (src < 0 || dst < 0) {
+        if (c == 0) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
+        return false;
+    }
+    return true;
+}
+
 // THREADS threads move CHUNK consecutive kept slots, base .. base + kSlots - 1
 // (those below cnt): a record of RB bytes is RB/16 16-byte vectors, one per
 // lane, so a warp instruction moves 32/(RB/16) whole records; each thread keeps
@@ -35,37 +74,8 @@ struct GatherChunk {
             const int i = base + (warp * ITERS + it) * kPerWarp + sub;
             dst[it] = -1;
             pv[it] = 0;
-            if (i >= cnt) continue;
-            const int64_t j = p.kept[r * p.B + i];
-            if (j == -1) continue;  // an entry the fused kernel emptied (its row was flagged there)
-            int64_t src = -1;
-            if (j >= 0 && j < N) {
-                if (geo.layout == TRI_KV_PAGED) {
-                    const int64_t bi = j >> geo.block_shift;
-                    const int32_t blk =
-                        bi < geo.max_blocks ? __ldg(geo.block_table + (int64_t)s * geo.max_blocks + bi) : -1;
-                    if (blk >= 0 && blk < geo.n_blocks)
-                        src = ((((int64_t)l * geo.n_blocks + blk) << geo.block_shift) |
-                               (j & ((1 << geo.block_shift) - 1))) * geo.H + h;
-                } else {
-                    src = row_lo + j;
-                }
-            }
-            int64_t d = -1;
-            if (p.out_layout == TRI_KV_PAGED) {
-                const int64_t bi = (int64_t)i >> p.out_block_shift;
-                const int32_t blk =
-                    bi < p.out_max_blocks ? __ldg(p.out_table + (int64_t)s * p.out_max_blocks + bi) : -1;
-                if (blk >= 0 && blk < p.out_n_blocks)
-                    d = ((((int64_t)l * p.out_n_blocks + blk) << p.out_block_shift) |
-                         (i & ((1 << p.out_block_shift) - 1))) * geo.H + h;
-            } else {
-                d = r * p.B + i;
-            }
-            if (src < 0 || d < 0) {
-                if (c == 0) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
-                continue;
-            }
+            int64_t src, d;
+            if (i >= cnt || !kept_record(p, r, row_lo, N, i, h, s, l, c, src, d)) continue;
             dst[it] = d;
             kv[it] = ld_nc16(p.K + src * RB + 16 * c);
             vv[it] = ld_nc16(p.V + src * RB + 16 * c);
@@ -78,6 +88,89 @@ struct GatherChunk {
             st_stream16(p.V_out + dst[it] * RB + 16 * c, vv[it]);
             if (p.pos_out && c == 0) p.pos_out[dst[it]] = pv[it];
         }
+    }
+};
+
+__device__ __forceinline__ void gc_cp_async16(void *smem, const void *gmem) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void gc_cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void gc_cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// A whole row's kept records through shared memory: the records are moved in
+// groups of kSlots (K and V of each, ITERS vectors of each per thread) with
+// asynchronous 16-byte copies into one half of `stage` while the other half,
+// which the same threads filled before, is written out.  No register holds a
+// record while it is in flight, so a group's 2 kSlots RB bytes are all in
+// flight at once; every thread stores exactly the vectors it copied, so no
+// barrier is needed.  `stage`: kStageBytes of shared memory, 16-byte aligned.
+template <int RB, int THREADS, int ITERS>
+struct GatherStaged {
+    static constexpr int kLanes = RB / 16;
+    static constexpr int kPerWarp = 32 / kLanes;
+    static constexpr int kSlots = (THREADS / 32) * ITERS * kPerWarp;  // records per half
+    static constexpr int kHalfBytes = kSlots * 2 * RB;
+    static constexpr int kStageBytes = 2 * kHalfBytes;
+
+    __device__ __forceinline__ static void copy(const GatherParams &p, int64_t r, int64_t row_lo, int64_t N, int cnt,
+                                                unsigned char *stage) {
+        const Geometry &geo = p.geo;
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int sub = lane / kLanes, c = lane % kLanes;
+        const int h = (int)(r % geo.H);
+        const int s = (int)((r / geo.H) % geo.S);
+        const int l = (int)(r / ((int64_t)geo.H * geo.S));
+        int64_t dst0[ITERS], dst1[ITERS];
+        int32_t pv0[ITERS], pv1[ITERS];
+        // Records base .. base + kSlots - 1 into half `hf` (one commit group).
+        auto issue = [&](unsigned char *buf, int base, int64_t (&dst)[ITERS], int32_t (&pv)[ITERS]) {
+#pragma unroll
+            for (int it = 0; it < ITERS; it++) {
+                const int k = (warp * ITERS + it) * kPerWarp + sub;
+                const int i = base + k;
+                dst[it] = -1;
+                pv[it] = 0;
+                int64_t src, d;
+                if (i >= cnt || !kept_record(p, r, row_lo, N, i, h, s, l, c, src, d)) continue;
+                dst[it] = d;
+                gc_cp_async16(buf + k * 2 * RB + 16 * c, p.K + src * RB + 16 * c);
+                gc_cp_async16(buf + k * 2 * RB + RB + 16 * c, p.V + src * RB + 16 * c);
+                if (p.pos && c == 0) pv[it] = __ldg(p.pos + src);
+            }
+            gc_cp_async_commit();
+        };
+        auto drain = [&](const unsigned char *buf, const int64_t (&dst)[ITERS], const int32_t (&pv)[ITERS]) {
+#pragma unroll
+            for (int it = 0; it < ITERS; it++) {
+                if (dst[it] < 0) continue;
+                const int k = (warp * ITERS + it) * kPerWarp + sub;
+                const uint4 a = *reinterpret_cast<const uint4 *>(buf + k * 2 * RB + 16 * c);
+                const uint4 b = *reinterpret_cast<const uint4 *>(buf + k * 2 * RB + RB + 16 * c);
+                st_stream16(p.K_out + dst[it] * RB + 16 * c, a);
+                st_stream16(p.V_out + dst[it] * RB + 16 * c, b);
+                if (p.pos_out && c == 0) p.pos_out[dst[it]] = pv[it];
+            }
+        };
+        if (cnt <= 0) return;
+        unsigned char *b0 = stage, *b1 = stage + kHalfBytes;
+        issue(b0, 0, dst0, pv0);
+        for (int base = 0;;) {
+            if (base + kSlots < cnt) issue(b1, base + kSlots, dst1, pv1);
+            else gc_cp_async_commit();
+            gc_cp_async_wait<1>();
+            drain(b0, dst0, pv0);
+            base += kSlots;
+            if (base >= cnt) break;
+            if (base + kSlots < cnt) issue(b0, base + kSlots, dst0, pv0);
+            else gc_cp_async_commit();
+            gc_cp_async_wait<1>();
+            drain(b1, dst1, pv1);
+            base += kSlots;
+            if (base >= cnt) break;
+        }
+        gc_cp_async_wait<0>();
     }
 };
 

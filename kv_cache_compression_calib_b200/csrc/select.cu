@@ -248,9 +248,9 @@ __device__ __forceinline__ void emit_bitmap(const uint32_t *bm_words, int64_t c0
 // GatherChunk<RB, kSelThreads, 2>::kSlots slots (two K and two V vectors in flight per
 // thread: 64 KB per SM with two CTAs, within the select path's registers).
 template <int RB>
-__device__ __forceinline__ void gather_row(const GatherParams &g, int64_t r, int64_t row_lo, int64_t N, int cnt) {
-    using Chunk = GatherChunk<RB, kSelThreads, 2>;
-    for (int base = 0; base < cnt; base += Chunk::kSlots) Chunk::move(g, r, row_lo, N, cnt, base);
+__device__ __forceinline__ void gather_row(const GatherParams &g, int64_t r, int64_t row_lo, int64_t N, int cnt,
+                                           unsigned char *stage) {
+    GatherStaged<RB, kSelThreads, 3>::copy(g, r, row_lo, N, cnt, stage);
 }
 
 // ------------------------------------------------------------------ one pass
@@ -284,6 +284,11 @@ constexpr int kOpCand = 8192;                    // band keys held on chip
 constexpr float kOpZ = 5.f;                      // band half-width in binomial standard deviations
 constexpr int kOpUnroll = 4;                     // 16-byte loads in flight per thread
 constexpr size_t kSelDynSmem = (size_t)(2 * kOpWords + 2 * kOpCand) * sizeof(uint32_t);
+static_assert(GatherStaged<64, kSelThreads, 3>::kStageBytes <= (int)kSelDynSmem &&
+                  GatherStaged<128, kSelThreads, 3>::kStageBytes <= (int)kSelDynSmem &&
+                  GatherStaged<256, kSelThreads, 3>::kStageBytes <= (int)kSelDynSmem &&
+                  GatherStaged<512, kSelThreads, 3>::kStageBytes <= (int)kSelDynSmem,
+              "the copy stages fit the selection's dynamic shared memory");
 
 __device__ __forceinline__ bool one_pass_select(const float *sc, int M, uint32_t K, bool vec, int32_t *out,
                                                 unsigned *flags, uint32_t *dyn, uint32_t *hist, uint32_t *scan_sm,
@@ -793,13 +798,16 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelectPara
         }
     } while (0);
     if (!LONG || !row_ok) return;
-    __syncthreads();  // out[] of this row is complete and visible to the block
+    __syncthreads();  // out[] of this row is complete and visible to the block; the
+                      // selection's dynamic shared memory is free for the copy stages
     const int cnt = (int)(N < (int64_t)B ? N : (int64_t)B);
+    extern __shared__ __align__(16) uint32_t sel_dyn[];
+    unsigned char *stage = reinterpret_cast<unsigned char *>(sel_dyn);
     switch (g.geo.D * g.geo.elem_bytes) {
-        case 64: gather_row<64>(g, r, row_lo, N, cnt); break;
-        case 128: gather_row<128>(g, r, row_lo, N, cnt); break;
-        case 256: gather_row<256>(g, r, row_lo, N, cnt); break;
-        case 512: gather_row<512>(g, r, row_lo, N, cnt); break;
+        case 64: gather_row<64>(g, r, row_lo, N, cnt, stage); break;
+        case 128: gather_row<128>(g, r, row_lo, N, cnt, stage); break;
+        case 256: gather_row<256>(g, r, row_lo, N, cnt, stage); break;
+        case 512: gather_row<512>(g, r, row_lo, N, cnt, stage); break;
     }
 }
 

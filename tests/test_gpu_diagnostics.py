@@ -1,7 +1,8 @@
 """Online centre update, concentration/drift statistics and pre-RoPE key centres
 against the oracle.  Calibration statistics to 1e-6 of the mean norm (fp64 on
-both sides, fp32 outputs); key centres to 2e-5 of the mean norm (fp32 key
-de-rotation with an exactly reduced phase, fp64 sums)."""
+both sides, fp32 outputs); key centres to 2e-5 of the mean norm (fp32 Horner sums
+along a lane's keys, settled with an exactly reduced phase every 8 batches and
+at every irregular position step; fp64 sums across runs)."""
 import numpy as np
 import pytest
 import torch
@@ -157,6 +158,27 @@ def test_key_centres_short_rows_ragged_total(elem, mode):
             continue
         rc, rm = oracle.key_centres(wl.theta, K[a:b], pos[a:b], post, wl.interleaved)
         check_centres(c[r], n[r], rc, rm)
+
+def test_key_centres_irregular_positions():
+    """RoPE caches with positions that break the regular stride (gaps, descending,
+    repeated, across the int32 range's end): every such key settles the lane's
+    Horner sum and restarts it."""
+    from tests.test_gpu_parity import irregular_positions
+    wl = synth.WORKLOADS["single_layer_4k"].with_(name="kcirr", batch=1, n_calib=8)
+    host = synth.make_contig(wl, "cpu", rotate=True)
+    for r in range(host.n_rows):
+        a, b = host.row_off_np[r], host.row_off_np[r + 1]
+        host.pos[a:b] = torch.as_tensor(irregular_positions(b - a, r).astype(np.int32))
+    m = model_of(wl, 1)
+    kv = tri.kv_contig(1, host.row_off.to(DEV), host.total)
+    c, n = run_key_centres(m, kv, host.K.to(DEV), host.pos.to(DEV), tri.TRI_KEYS_POST_ROPE, host.n_rows, 64, 1)
+    K = H.to_f64(host.K)
+    pos = host.pos.numpy().astype(np.int64)
+    for r in range(host.n_rows):
+        a, b = host.row_off_np[r], host.row_off_np[r + 1]
+        rc, rm = oracle.key_centres(wl.theta, K[a:b], pos[a:b], True, wl.interleaved)
+        check_centres(c[r], n[r], rc, rm)
+
 
 def test_key_centres_paged():
     wl = synth.WORKLOADS["paged_16seq"].with_(name="kcp", batch=3, n_calib=8)

@@ -297,6 +297,46 @@ def test_pre_rope_shifted_positions():
         assert H.score_error(got[a:b], ref, bd) <= 1e-4
 
 
+def irregular_positions(n, r):
+    """Position patterns per row that break the regular stride: gaps (a compacted
+    cache), a descending run, repeats, a run across the end of the int32 range,
+    and runs of 16 with gaps between them."""
+    rng = np.random.default_rng(1000 + r)
+    kind = r % 5
+    if kind == 0:
+        return np.sort(rng.choice(50000, n, replace=False))
+    if kind == 1:
+        return np.arange(n)[::-1].copy()
+    if kind == 2:
+        return np.arange(n) // 2
+    if kind == 3:
+        top = np.iinfo(np.int32).max
+        return np.concatenate([np.arange(top - n // 2 + 1, top + 1), np.iinfo(np.int32).min + np.arange(n - n // 2)])
+    return (np.arange(n) // 16) * 100 + np.arange(n) % 16
+
+
+def test_pre_rope_irregular_positions():
+    """The pre-RoPE kernels chain a lane's rotated coefficients only where a key sits
+    exactly NG positions after the last one; every other key (gaps, descending or
+    repeated positions, a run across the int32 range's end) takes its own phase."""
+    wl = synth.WORKLOADS["single_layer_4k"].with_(name="preirr", n_calib=64)
+    host = synth.make_contig(wl, "cpu", rotate=False)
+    for r in range(host.n_rows):
+        a, b = host.row_off_np[r], host.row_off_np[r + 1]
+        host.pos[a:b] = torch.as_tensor(irregular_positions(b - a, r).astype(np.int32))
+    cs, ms = oracle_centres(host)
+    K = H.to_f64(host.K)
+    pos = host.pos.numpy().astype(np.int64)
+    got = gpu_score(to_dev(host), cs, ms, key_mode=PRE).cpu().numpy().astype(np.float64)
+    for r in range(host.n_rows):
+        li, s, h = host.row_lhs(r)
+        a, b = host.row_off_np[r], host.row_off_np[r + 1]
+        ref = oracle.row_scores(wl.theta, cs[li], ms[li], h, wl.group, K[a:b], pos[a:b], False,
+                                int(host.p_now[s]), wl.offsets, "collapsed")
+        bd = H.series_bound(wl.theta, cs[li], ms[li], h, wl.group, K[a:b], wl.offsets)
+        assert H.score_error(got[a:b], ref, bd) <= 1e-4, r
+
+
 # ------------------------------------------------------ GQA 8, 17 offsets
 
 def test_group_of_eight_seventeen_offsets():
