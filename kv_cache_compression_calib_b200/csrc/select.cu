@@ -282,7 +282,7 @@ constexpr int64_t kOpMaxRow = 4 * kChunk;        // 131072 slots: the bitmaps' c
 constexpr int kOpWords = (int)(kOpMaxRow / 32);  // words per bitmap
 constexpr int kOpCand = 8192;                    // band keys held on chip
 constexpr float kOpZ = 5.f;                      // band half-width in binomial standard deviations
-constexpr int kOpUnroll = 4;                     // 16-byte loads in flight per thread
+constexpr int kOpUnroll = 8;                     // 16-byte loads in flight per thread
 constexpr size_t kSelDynSmem = (size_t)(2 * kOpWords + 2 * kOpCand) * sizeof(uint32_t);
 static_assert(GatherStaged<64, kSelThreads, 3>::kStageBytes <= (int)kSelDynSmem &&
                   GatherStaged<128, kSelThreads, 3>::kStageBytes <= (int)kSelDynSmem &&
