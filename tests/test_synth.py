@@ -102,3 +102,17 @@ def test_fp8_conversion_is_nearest_e4m3_of_the_clamped_value():
         assert gv in near, (xi, gi, near)
         if len(near) == 2:  # an exact tie between two values: the even mantissa wins
             assert gi & 1 == 0, (xi, gi, near)
+
+
+def test_fp8_conversion_in_chunks_is_the_one_shot_conversion():
+    """The chunked conversion (bounded temporary memory for caches near the device's
+    size) gives the same bytes as converting the whole tensor at once, including
+    values beyond the e4m3 range (clamped to +-448) and a ragged last chunk."""
+    import torch
+    g = torch.Generator().manual_seed(7)
+    t = (torch.randn(1001, 37, generator=g) * 200).to(torch.bfloat16)
+    t[0, :4] = torch.tensor([1e4, -1e4, 448.0, -0.0], dtype=torch.bfloat16)
+    whole = t.float().clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    got = synth.to_fp8(t, chunk=1000)
+    assert got.shape == t.shape and got.dtype == torch.float8_e4m3fn
+    assert torch.equal(got.view(torch.uint8), whole.view(torch.uint8))
