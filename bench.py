@@ -8,7 +8,10 @@ offline and timed separately.  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload qwen3_32b_128k] [--also qwen3_8b_32k|none] [--budget B] [--key-mode post|pre]
-                  [--elem bf16|fp8] [--head-dim 64|128|256] [--rope half|interleaved]
+                  [--elem bf16|fp8] [--head-dim 64|128|256] [--rope half|interleaved] [--no-variants]
+
+The default line also carries the 32K workload's step ('also') and the same step
+over a pre-RoPE cache and over an fp8 e4m3 cache ('variants'), step timings only.
 
 N > 1 (under torchrun): every rank compacts its own cache of the same shape
 (independent sequences; no collective on the data path), timing is the max
@@ -78,6 +81,8 @@ def parse():
                          "fused: one tri_score_compact call per step (rows up to TRI_FUSED_MAX_ROW keys, scores "
                          "kept on chip, no score buffer)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the 32K workload's pre-RoPE and fp8 step timings reported under 'variants'")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     a = ap.parse_args()
@@ -869,6 +874,21 @@ def main():
             gc.collect()
             torch.cuda.empty_cache()
             line["also"] = also_summary(run_ours(a, rank, world, local_rank, workload=a.also, light=True))
+        if not a.no_variants and a.key_mode == "post" and a.elem == "bf16" and a.path == "split" \
+                and not a.layers and not a.budget and a.head_dim is None and a.rope is None:
+            # the same 32K step with a pre-RoPE cache and with an fp8 e4m3 cache
+            import copy
+            import gc
+
+            variants = {}
+            for name, field, val in (("pre_rope", "key_mode", "pre"), ("fp8", "elem", "fp8")):
+                gc.collect()
+                torch.cuda.empty_cache()
+                b = copy.copy(a)
+                setattr(b, field, val)
+                variants[name] = also_summary(run_ours(b, rank, world, local_rank, workload="qwen3_8b_32k",
+                                                       light=True))
+            line["variants"] = variants
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
