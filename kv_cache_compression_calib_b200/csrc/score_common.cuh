@@ -91,6 +91,19 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
     return d;
 }
 
+// The same two-lane operations as scalar fp32 instructions on the register pair's
+// halves (each rounds exactly as the packed form, so the results are the same
+// bits), for the pre-RoPE steps, where the compiler can then fold sign flips
+// into the multiply-adds.
+__device__ __forceinline__ unsigned long long fma2s(unsigned long long a, unsigned long long b, unsigned long long c) {
+    const float2 A = f2split(a), B = f2split(b), C = f2split(c);
+    return f2(__fmaf_rn(A.x, B.x, C.x), __fmaf_rn(A.y, B.y, C.y));
+}
+__device__ __forceinline__ unsigned long long mul2s(unsigned long long a, unsigned long long b) {
+    const float2 A = f2split(a), B = f2split(b);
+    return f2(__fmul_rn(A.x, B.x), __fmul_rn(A.y, B.y));
+}
+
 // Partial score of 8 pairs: sum_i Re(A_i conj k_i) + c_i |k_i|, two pairs (i, i+1)
 // per packed instruction: the dot product and the squared norms in f32x2, one
 // square root per pair.
@@ -167,8 +180,8 @@ __device__ __forceinline__ void rotate_coef(const RowCtx &c, const float (&cs)[8
     for (int k = 0; k < 4; k++) {
         const unsigned long long AR = f2(c.ar[2 * k], c.ar[2 * k + 1]), AI = f2(c.ai[2 * k], c.ai[2 * k + 1]);
         const unsigned long long CS = f2(cs[2 * k], cs[2 * k + 1]), SN = f2(sn[2 * k], sn[2 * k + 1]);
-        BR[k] = fma2(AR, CS, mul2(neg2(AI), SN));
-        BI[k] = fma2(AR, SN, mul2(AI, CS));
+        BR[k] = fma2s(AR, CS, mul2s(neg2(AI), SN));
+        BI[k] = fma2s(AR, SN, mul2s(AI, CS));
     }
 }
 
@@ -178,8 +191,8 @@ __device__ __forceinline__ void advance_coef(unsigned long long (&BR)[4], unsign
                                              const unsigned long long (&TC)[4], const unsigned long long (&TS)[4]) {
 #pragma unroll
     for (int k = 0; k < 4; k++) {
-        const unsigned long long r = fma2(BR[k], TC[k], mul2(BI[k], neg2(TS[k])));
-        BI[k] = fma2(BR[k], TS[k], mul2(BI[k], TC[k]));
+        const unsigned long long r = fma2s(BR[k], TC[k], mul2s(BI[k], neg2(TS[k])));
+        BI[k] = fma2s(BR[k], TS[k], mul2s(BI[k], TC[k]));
         BR[k] = r;
     }
 }
@@ -193,10 +206,10 @@ __device__ __forceinline__ float partial_rotated(const float (&x)[8], const floa
 #pragma unroll
     for (int k = 0; k < 4; k++) {
         const unsigned long long X = f2(x[2 * k], x[2 * k + 1]), Y = f2(y[2 * k], y[2 * k + 1]);
-        d = fma2(BR[k], X, d);
-        d = fma2(BI[k], Y, d);
-        const float2 q = f2split(fma2(X, X, mul2(Y, Y)));
-        e = fma2(f2(c.cc[2 * k], c.cc[2 * k + 1]), f2(sqrt_approx(q.x), sqrt_approx(q.y)), e);
+        d = fma2s(BR[k], X, d);
+        d = fma2s(BI[k], Y, d);
+        const float2 q = f2split(fma2s(X, X, mul2s(Y, Y)));
+        e = fma2s(f2(c.cc[2 * k], c.cc[2 * k + 1]), f2(sqrt_approx(q.x), sqrt_approx(q.y)), e);
     }
     const float2 dd = f2split(d), ee = f2split(e);
     return (dd.x + dd.y) + (ee.x + ee.y);
