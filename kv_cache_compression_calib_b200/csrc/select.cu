@@ -40,7 +40,6 @@ namespace tri {
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kItems = 64;  // slots per thread per chunk
-constexpr int kLoadsInFlight = 4;  // 16-byte score loads a thread issues before using them (chunk passes)
 constexpr int64_t kChunk = (int64_t)kSelThreads * kItems;
 constexpr int kWords = (int)(kChunk / 32);  // bitmap words per chunk
 constexpr int kBins = 2048;
@@ -140,23 +139,15 @@ __device__ __forceinline__ void for_each_score(const float *base, int n, bool ve
     if (vec) {
         const float4 *q = reinterpret_cast<const float4 *>(base);
         const int nvec = n >> 2;
-        // kLoadsInFlight 16-byte loads issued before any is used
-        for (int k0 = 0; k0 < kItems / 4; k0 += kLoadsInFlight) {
-            float4 x[kLoadsInFlight];
-#pragma unroll
-            for (int u = 0; u < kLoadsInFlight; u++) {
-                const int v = (k0 + u) * kSelThreads + t;
-                x[u] = v < nvec ? __ldg(q + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < kLoadsInFlight; u++) {
-                const int v = (k0 + u) * kSelThreads + t;
-                if (v < nvec) {
-                    fn(4 * v + 0, x[u].x);
-                    fn(4 * v + 1, x[u].y);
-                    fn(4 * v + 2, x[u].z);
-                    fn(4 * v + 3, x[u].w);
-                }
+#pragma unroll 4
+        for (int k = 0; k < kItems / 4; k++) {
+            const int v = k * kSelThreads + t;
+            if (v < nvec) {
+                const float4 x = __ldg(q + v);
+                fn(4 * v + 0, x.x);
+                fn(4 * v + 1, x.y);
+                fn(4 * v + 2, x.z);
+                fn(4 * v + 3, x.w);
             }
         }
         const int j = 4 * nvec + t;  // ragged tail: at most 3 slots
@@ -179,31 +170,24 @@ __device__ __forceinline__ void build_bitmap(const float *base, int n, bool vec,
     const int t = threadIdx.x, lane = t & 31;
     if (vec) {
         const float4 *q = reinterpret_cast<const float4 *>(base);
-        for (int k0 = 0; k0 < kItems / 4; k0 += kLoadsInFlight) {
-            float4 x[kLoadsInFlight];
+#pragma unroll 4
+        for (int k = 0; k < kItems / 4; k++) {
+            const int v = k * kSelThreads + t;
+            uint32_t nib = 0;
+            if (4 * v + 3 < n) {
+                const float4 x = __ldg(q + v);
+                nib = (uint32_t)pred(4 * v, x.x) | ((uint32_t)pred(4 * v + 1, x.y) << 1) |
+                      ((uint32_t)pred(4 * v + 2, x.z) << 2) | ((uint32_t)pred(4 * v + 3, x.w) << 3);
+            } else {
 #pragma unroll
-            for (int u = 0; u < kLoadsInFlight; u++) {
-                const int v = (k0 + u) * kSelThreads + t;
-                x[u] = 4 * v + 3 < n ? __ldg(q + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int i = 0; i < 4; i++)
+                    if (4 * v + i < n) nib |= (uint32_t)pred(4 * v + i, __ldg(base + 4 * v + i)) << i;
             }
-#pragma unroll
-            for (int u = 0; u < kLoadsInFlight; u++) {
-                const int v = (k0 + u) * kSelThreads + t;
-                uint32_t nib = 0;
-                if (4 * v + 3 < n) {
-                    nib = (uint32_t)pred(4 * v, x[u].x) | ((uint32_t)pred(4 * v + 1, x[u].y) << 1) |
-                          ((uint32_t)pred(4 * v + 2, x[u].z) << 2) | ((uint32_t)pred(4 * v + 3, x[u].w) << 3);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 4; i++)
-                        if (4 * v + i < n) nib |= (uint32_t)pred(4 * v + i, __ldg(base + 4 * v + i)) << i;
-                }
-                uint32_t w = nib << (4 * (lane & 7));
-                w |= __shfl_xor_sync(0xffffffffu, w, 1);
-                w |= __shfl_xor_sync(0xffffffffu, w, 2);
-                w |= __shfl_xor_sync(0xffffffffu, w, 4);
-                if ((lane & 7) == 0) bm_words[(4 * v) >> 5] = w;
-            }
+            uint32_t w = nib << (4 * (lane & 7));
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            w |= __shfl_xor_sync(0xffffffffu, w, 4);
+            if ((lane & 7) == 0) bm_words[(4 * v) >> 5] = w;
         }
     } else {
 #pragma unroll 4
