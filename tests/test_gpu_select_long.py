@@ -199,3 +199,61 @@ def test_band_cases_on_long_rows(long_rows, case):
             assert res["flags"] == tri.TRI_FLAG_NONFINITE
         else:
             assert res["status"] == 0
+
+
+@pytest.mark.parametrize("d,elem", [(64, "fp8"), (128, "fp8"), (256, "bf16")])
+@pytest.mark.parametrize("paged_out", [False, True])
+def test_long_row_copy_record_sizes_and_paged_output(d, elem, paged_out):
+    """The select-and-gather kernel copies a long row's kept records through its
+    shared memory in groups whose size depends on the record (64, 128 and 512
+    bytes here; 128 above): K, V and positions bit for bit, into [R][B] or into a
+    fresh, shuffled paged block table."""
+    lens = np.array([CHUNK + 4000, 90000])
+    R, B, W, bs = len(lens), 4096, 256, 16
+    row_off_np = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    total = int(row_off_np[-1])
+    g = torch.Generator().manual_seed(23)
+    if elem == "fp8":
+        K = torch.randint(0, 256, (total, d), dtype=torch.uint8, generator=g).view(torch.float8_e4m3fn)
+        V = torch.randint(0, 256, (total, d), dtype=torch.uint8, generator=g).view(torch.float8_e4m3fn)
+    else:
+        K = torch.randint(-32768, 32767, (total, d), dtype=torch.int16, generator=g).view(torch.bfloat16)
+        V = torch.randint(-32768, 32767, (total, d), dtype=torch.int16, generator=g).view(torch.bfloat16)
+    pos = torch.cat([torch.arange(int(n), dtype=torch.int32) for n in lens])
+    rng = np.random.default_rng(29)
+    s32 = H.as_f32_exact(rng.standard_normal(total))
+    m = tri.model(1, R, R, 1e6, head_dim=d)  # one sequence, R KV heads
+    kv = tri.kv_contig(1, torch.as_tensor(row_off_np, device=DEV), total, tri.elem_type_of(K))
+    ws = tri.alloc_workspace(m, 1, B)
+    kept = torch.full((R, B), -1, dtype=torch.int32, device=DEV)
+    if paged_out:
+        n_out = B // bs
+        out_tbl = rng.permutation(n_out).reshape(1, n_out).astype(np.int32)
+        Ko = torch.zeros(1, n_out, bs, R, d, dtype=K.dtype, device=DEV)
+        po = torch.full((1, n_out, bs, R), -7, dtype=torch.int32, device=DEV)
+        out = tri.out_paged(torch.as_tensor(out_tbl, device=DEV), bs, n_out)
+    else:
+        Ko = torch.zeros(R, B, d, dtype=K.dtype, device=DEV)
+        po = torch.full((R, B), -7, dtype=torch.int32, device=DEV)
+        out = tri.out_contig()
+    Vo = torch.zeros_like(Ko)
+    tri.tri_compact(m, kv, torch.tensor(s32, dtype=torch.float32, device=DEV), B, W, K.to(DEV), V.to(DEV),
+                    pos.to(DEV), out, Ko, Vo, po, kept, None, ws)
+    st, flags = tri.tri_status_check(ws)
+    assert st == 0, flags
+    Kb, Vb = H.raw_bits(K), H.raw_bits(V)
+    Kob, Vob, pob = H.raw_bits(Ko.cpu()), H.raw_bits(Vo.cpu()), po.cpu().numpy()
+    kept = kept.cpu().numpy()
+    for r in range(R):
+        a, b = row_off_np[r], row_off_np[r + 1]
+        ref = oracle.select(s32[a:b], B, W)
+        np.testing.assert_array_equal(kept[r], ref)
+        i = np.arange(B)
+        if paged_out:
+            blk = out_tbl[0, i // bs]
+            got_k, got_v, got_p = Kob[0, blk, i % bs, r], Vob[0, blk, i % bs, r], pob[0, blk, i % bs, r]
+        else:
+            got_k, got_v, got_p = Kob[r], Vob[r], pob[r]
+        np.testing.assert_array_equal(got_k, oracle.gather(Kb[a:b], ref))
+        np.testing.assert_array_equal(got_v, oracle.gather(Vb[a:b], ref))
+        np.testing.assert_array_equal(got_p, oracle.gather(pos.numpy()[a:b], ref))
