@@ -136,6 +136,108 @@ def test_fused_fallback_and_long_rows():
     np.testing.assert_array_equal(kept[8:].cpu().numpy(), plain["kept"][8:])
 
 
+@pytest.mark.parametrize("d,elem", [(128, "bf16"), (256, "bf16"), (128, "fp8")])
+def test_fused_rows_beyond_the_stated_bound(d, elem):
+    """max_row_len 4096 against rows of 100 to 32768 keys: the call takes the fused
+    kernel and every row up to TRI_FUSED_MAX_ROW is processed normally, equal to
+    tri_score + tri_compact bit for bit."""
+    wl = synth.WORKLOADS["single_layer_4k"].with_(name=f"fzbound{d}{elem}", head_dim=d, batch=6, n_calib=16,
+                                                  theta=1e6 if d == 128 else 1e4)
+    host = synth.make_contig(wl, "cpu", lens=[20480, 20481, 24000, 32768, 2176, 100])
+    if elem == "fp8":
+        host.K, host.V = synth.to_fp8(host.K), synth.to_fp8(host.V)
+    from tests.test_gpu_parity import to_dev
+    cs, ms = oracle_centres(host)
+    dev = to_dev(host)
+    fused, plain = run_both(wl, dev, cs, ms, 2048, 128, max_row_len=4096)
+    assert_identical(fused, plain)
+
+
+def paged_both(wl, lens, B, W, elem="bf16", edit_table=None):
+    """(fused, unfused) results of one paged re-score round (post-RoPE keys,
+    contiguous [R][B] outputs): (status, flags, scores, kept, K, V, pos) each, and
+    the row offsets."""
+    p = synth.make_paged(wl, "cpu", lens=lens)
+    if elem == "fp8":
+        p.K, p.V = synth.to_fp8(p.K), synth.to_fp8(p.V)
+    qcal = synth.calib_queries(wl, 0, "cpu")[None]
+    cs, ms = H.oracle_calibration(qcal)
+    cs, ms = H.as_f32_exact(cs), H.as_f32_exact(ms)
+    S, Hh, bs, d = len(lens), wl.n_kv_heads, wl.block_size, wl.head_dim
+    row_off = synth.paged_row_offsets(np.asarray(lens), Hh)
+    total = int(row_off[-1])
+    m = model_of(wl, 1)
+    tbl = p.block_table.clone()
+    if edit_table:
+        edit_table(tbl)
+    kv = tri.kv_paged(S, torch.as_tensor(row_off, device=DEV), total, tbl.to(DEV), bs, p.K.shape[0],
+                      tri.elem_type_of(p.K))
+    Kd, Vd, pd = p.K.to(DEV), p.V.to(DEV), p.pos.to(DEV)
+    c32 = torch.tensor(cs, dtype=torch.float32, device=DEV)
+    m32 = torch.tensor(ms, dtype=torch.float32, device=DEV)
+    res = []
+    for fused in (True, False):
+        ws = tri.alloc_workspace(m, S, B)
+        scores = torch.full((total,), float("nan"), device=DEV)
+        Ko = torch.zeros(S * Hh, B, d, dtype=Kd.dtype, device=DEV)
+        Vo = torch.zeros_like(Ko)
+        po = torch.full((S * Hh, B), -1, dtype=torch.int32, device=DEV)
+        kept = torch.full((S * Hh, B), -1, dtype=torch.int32, device=DEV)
+        if fused:
+            tri.tri_score_compact(m, kv, Kd, Vd, pd, c32, m32, p.p_now.to(DEV), wl.offsets, POST, B, W,
+                                  int(max(lens)), tri.out_contig(), Ko, Vo, po, kept, None, scores, ws)
+        else:
+            tri.tri_score(m, kv, Kd, pd, c32, m32, p.p_now.to(DEV), wl.offsets, POST, scores, ws)
+            tri.tri_compact(m, kv, scores, B, W, Kd, Vd, pd, tri.out_contig(), Ko, Vo, po, kept, None, ws)
+        st, flags = tri.tri_status_check(ws)
+        res.append((st, flags, scores.cpu(), kept.cpu(), H.torch_bits(Ko.cpu()), H.torch_bits(Vo.cpu()), po.cpu()))
+    return res, row_off
+
+
+def assert_same_round(a, b):
+    for x, y in zip(a, b):
+        if isinstance(x, torch.Tensor):
+            assert torch.equal(x.view(torch.int32) if x.dtype == torch.float32 else x,
+                               y.view(torch.int32) if y.dtype == torch.float32 else y)
+        else:
+            assert x == y
+
+
+@pytest.mark.parametrize("d,style,elem", [(128, "half", "bf16"), (64, "interleaved", "bf16"), (256, "half", "bf16"),
+                                          (128, "half", "fp8"), (128, "interleaved", "fp8"), (256, "interleaved", "bf16")])
+def test_fused_paged_rounds_equal_two_calls(d, style, elem):
+    """Paged re-score rounds (rows of a few thousand keys: several batches per warp,
+    partial batches at the row ends) at every head dim, pairing and element type:
+    fused equals tri_score + tri_compact bit for bit."""
+    wl = synth.WORKLOADS["paged_16seq"].with_(name=f"fzpr{d}{style}{elem}", batch=3, n_calib=16, head_dim=d,
+                                              rope_style=style, theta=1e6 if d == 128 else 1e4)
+    (f, u), _ = paged_both(wl, [2176, 3000, 700], 2048, 128, elem)
+    assert f[0] == u[0] == 0, (f[1], u[1])
+    assert_same_round(f, u)
+
+
+def test_fused_paged_unplaceable_block():
+    """Block ids outside the pool inside whole batches: the fused kernel scores
+    those keys 0 and raises the same flag as the score kernel; results equal
+    tri_score + tri_compact."""
+    wl = synth.WORKLOADS["paged_16seq"].with_(name="fzpb", batch=2, n_calib=16)
+    bs = wl.block_size
+
+    def edit(tbl):
+        tbl[0, 5] = 10 ** 6  # keys 80 .. 95 of sequence 0: out of the pool
+        tbl[1, 63] = -3      # the last block of sequence 1
+
+    (f, u), row_off = paged_both(wl, [2176, 1024], 1024, 64, edit_table=edit)
+    assert f[1] == u[1] == tri.TRI_FLAG_BLOCK_TABLE and f[0] == u[0] == tri._abi.TRI_ERR_DEVICE_FLAG
+    bad = np.zeros(int(row_off[-1]), dtype=bool)
+    for s, blk in ((0, 5), (1, 63)):
+        for h in range(wl.n_kv_heads):
+            r0 = int(row_off[s * wl.n_kv_heads + h])
+            bad[r0 + blk * bs: r0 + (blk + 1) * bs] = True
+    assert torch.all(f[2][torch.as_tensor(bad)] == 0)  # unplaceable keys score 0 on both paths
+    assert_same_round(f, u)
+
+
 def plain_rows(res, r0):
     return H.raw_bits(res["K"][r0:])
 
