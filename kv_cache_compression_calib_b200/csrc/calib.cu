@@ -6,9 +6,11 @@
 // Thread (grp, f) walks queries t = grp, grp+4, ... reading the two dims of
 // pair f - (f, f+F) with rotate-half RoPE, (2f, 2f+1) with interleaved RoPE,
 // coalesced across the warp either way - and accumulates in fp64 (x^2 + y^2 of
-// two bf16 values is exact in fp64).  The four partial sums are combined in a
-// fixed order, so results are deterministic.  Runs once, offline; it is not on
-// the per-token path.
+// two bf16 values is exact in fp64).  The loads of 8 consecutive queries of a
+// thread are issued before their sums (the sums still run in query order), so
+// each thread keeps 16 loads in flight.  The four partial sums are combined in
+// a fixed order, so results are deterministic.  Runs once, offline; it is not
+// on the per-token path.
 #include "tri_internal.cuh"
 
 namespace tri {
@@ -23,9 +25,27 @@ __global__ void __launch_bounds__(4 * F) calib_kernel(const CalibParams p) {
     const uint16_t *base = p.q + (int64_t)head * p.nq * D;
     const int ia = IL ? 2 * f : f, ib = IL ? 2 * f + 1 : f + F;
     double sr = 0.0, si = 0.0, sn = 0.0;
-    for (int64_t t = grp; t < p.nq; t += 4) {
-        const double x = (double)__uint_as_float((uint32_t)base[t * D + ia] << 16);
-        const double y = (double)__uint_as_float((uint32_t)base[t * D + ib] << 16);
+    constexpr int kBatch = 8;  // queries per thread whose loads are in flight together
+    int64_t t = grp;
+    for (; t + 4 * (kBatch - 1) < p.nq; t += 4 * kBatch) {
+        uint16_t xa[kBatch], ya[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; k++) {
+            xa[k] = __ldg(base + (t + 4 * k) * D + ia);
+            ya[k] = __ldg(base + (t + 4 * k) * D + ib);
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; k++) {
+            const double x = (double)__uint_as_float((uint32_t)xa[k] << 16);
+            const double y = (double)__uint_as_float((uint32_t)ya[k] << 16);
+            sr += x;
+            si += y;
+            sn += sqrt(x * x + y * y);
+        }
+    }
+    for (; t < p.nq; t += 4) {
+        const double x = (double)__uint_as_float((uint32_t)__ldg(base + t * D + ia) << 16);
+        const double y = (double)__uint_as_float((uint32_t)__ldg(base + t * D + ib) << 16);
         sr += x;
         si += y;
         sn += sqrt(x * x + y * y);
