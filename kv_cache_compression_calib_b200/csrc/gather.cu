@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     grid_dependency_wait();
     grid_dependents_launch();
     const Geometry &geo = p.geo;
-    const int64_t chunks = (p.B + kSlotsPerCta - 1) / kSlotsPerCta;
+    const uint32_t chunks = (uint32_t)((p.B + kSlotsPerCta - 1) / kSlotsPerCta);  // grid = rows x chunks < 2^31
     const int64_t r = blockIdx.x / chunks;
     const int base = (int)(blockIdx.x % chunks) * kSlotsPerCta;
     const int64_t row_lo = geo.row_off[r];

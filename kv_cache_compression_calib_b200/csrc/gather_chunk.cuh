@@ -8,6 +8,18 @@
 
 namespace tri {
 
+// Layer l, sequence s and KV head h of row r = (l S + s) H + h, in 32-bit
+// arithmetic (a 64-bit division is a long instruction sequence, paid by every
+// thread of every gather CTA): r < 2^31, since every launch over rows keeps its
+// grid within one grid dimension.
+__device__ __forceinline__ void row_lsh(const Geometry &geo, int64_t r, int &l, int &s, int &h) {
+    const uint32_t ru = (uint32_t)r, H = (uint32_t)geo.H, S = (uint32_t)geo.S;
+    const uint32_t q = ru / H;
+    h = (int)(ru - q * H);
+    l = (int)(q / S);
+    s = (int)(q - (uint32_t)l * S);
+}
+
 // Source and destination records of kept slot i of row r (layer l, sequence
 // s, KV head h).  False for an entry the fused kernel emptied (-1) and for a
 // slot a block table cannot place (flagged by the lane with c == 0).
@@ -63,9 +75,8 @@ struct GatherChunk {
         const Geometry &geo = p.geo;
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
         const int sub = lane / kLanes, c = lane % kLanes;
-        const int h = (int)(r % geo.H);
-        const int s = (int)((r / geo.H) % geo.S);
-        const int l = (int)(r / ((int64_t)geo.H * geo.S));
+        int l, s, h;
+        row_lsh(geo, r, l, s, h);
         uint4 kv[ITERS], vv[ITERS];
         int64_t dst[ITERS];
         int32_t pv[ITERS];
@@ -119,9 +130,8 @@ struct GatherStaged {
         const Geometry &geo = p.geo;
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
         const int sub = lane / kLanes, c = lane % kLanes;
-        const int h = (int)(r % geo.H);
-        const int s = (int)((r / geo.H) % geo.S);
-        const int l = (int)(r / ((int64_t)geo.H * geo.S));
+        int l, s, h;
+        row_lsh(geo, r, l, s, h);
         int64_t dst0[ITERS], dst1[ITERS];
         int32_t pv0[ITERS], pv1[ITERS];
         // Records base .. base + kSlots - 1 into half `hf` (one commit group).
