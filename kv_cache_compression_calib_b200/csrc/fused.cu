@@ -151,25 +151,47 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_kernel(const FusedParams f
         float part[U];
         if (b0 >= lo && b0 + KB <= hi) {
             KeyChunk<ELEM, IL, F> kc[U];
-            int64_t slot[U];
             int32_t kpos[U];
-#pragma unroll
-            for (int u = 0; u < U; u++) {
-                slot[u] = key_slot<PAGED>(p, c, b0 + NG * u + q);
-                if (slot[u] >= 0) {
-                    kc[u].load(p.K + slot[u] * RB, gl, pol);
-                    kpos[u] = PRE ? __ldg(p.pos + slot[u]) : 0;
-                } else {
-                    kc[u].zero();
-                    kpos[u] = 0;
-                }
-            }
             bool ok[U];
+            if constexpr (PAGED && !PRE) {
+                // key_slot's address in 32-bit steps where they fit: the row has at
+                // most kFusedMaxRow keys, so a key's place in the row and its block
+                // index are small; only the block's byte offset needs 64 bits.
+                // Byte address: the layer's head-h record of block 0, plus blk blocks,
+                // plus the slot within the block.
+                const int j0 = (int)(b0 - lo) + q;
+                const char *kb = p.K + (((c.layer_blk << geo.block_shift) * geo.H) + c.h) * RB;
+                const int64_t blk_bytes = ((int64_t)geo.H * RB) << geo.block_shift;
+                const int64_t slot_bytes = (int64_t)geo.H * RB;
 #pragma unroll
-            for (int u = 0; u < U; u++) {
-                ok[u] = !PAGED || slot[u] >= 0;
-                if (!ok[u]) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
+                for (int u = 0; u < U; u++) {
+                    const int j = j0 + NG * u;
+                    const int bi = j >> geo.block_shift;
+                    const int32_t blk = bi < geo.max_blocks ? __ldg(c.table + bi) : -1;
+                    ok[u] = blk >= 0 && blk < geo.n_blocks;
+                    kpos[u] = 0;
+                    if (ok[u]) kc[u].load(kb + blk * blk_bytes + (j & ((1 << geo.block_shift) - 1)) * slot_bytes, gl, pol);
+                    else kc[u].zero();
+                }
+            } else {
+                int64_t slot[U];
+#pragma unroll
+                for (int u = 0; u < U; u++) {
+                    slot[u] = key_slot<PAGED>(p, c, b0 + NG * u + q);
+                    if (slot[u] >= 0) {
+                        kc[u].load(p.K + slot[u] * RB, gl, pol);
+                        kpos[u] = PRE ? __ldg(p.pos + slot[u]) : 0;
+                    } else {
+                        kc[u].zero();
+                        kpos[u] = 0;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; u++) ok[u] = !PAGED || slot[u] >= 0;
             }
+#pragma unroll
+            for (int u = 0; u < U; u++)
+                if (!ok[u]) atomicOr(p.flags, TRI_FLAG_BLOCK_TABLE);
             batch_partials<PRE, U, NG>(kc, kpos, ok, c, T, TC, TS, part);
         } else {
 #pragma unroll
