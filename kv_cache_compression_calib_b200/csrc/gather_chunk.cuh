@@ -28,27 +28,29 @@ __device__ __forceinline__ bool kept_record(const GatherParams &p, int64_t r, in
     const Geometry &geo = p.geo;
     const int64_t j = p.kept[r * p.B + i];
     if (j == -1) return false;  // an entry the fused kernel emptied (its row was flagged there)
+    // Paged records: (layer l, block blk, slot t, head h) is record
+    // (l n_blocks + blk) bs H + t H + h; j < N < 2^31 and i < B, so a slot's place
+    // and block index are 32-bit and only the block term needs 64 bits.
     src = -1;
     if (j >= 0 && j < N) {
         if (geo.layout == TRI_KV_PAGED) {
-            const int64_t bi = j >> geo.block_shift;
+            const int jj = (int)j;
+            const int bi = jj >> geo.block_shift;
             const int32_t blk = bi < geo.max_blocks ? __ldg(geo.block_table + (int64_t)s * geo.max_blocks + bi) : -1;
             if (blk >= 0 && blk < geo.n_blocks)
-                src = ((((int64_t)l * geo.n_blocks + blk) << geo.block_shift) | (j & ((1 << geo.block_shift) - 1))) *
-                          geo.H +
-                      h;
+                src = ((int64_t)l * geo.n_blocks + blk) * ((int64_t)geo.H << geo.block_shift) +
+                      (int64_t)(jj & ((1 << geo.block_shift) - 1)) * geo.H + h;
         } else {
             src = row_lo + j;
         }
     }
     dst = -1;
     if (p.out_layout == TRI_KV_PAGED) {
-        const int64_t bi = (int64_t)i >> p.out_block_shift;
+        const int bi = i >> p.out_block_shift;
         const int32_t blk = bi < p.out_max_blocks ? __ldg(p.out_table + (int64_t)s * p.out_max_blocks + bi) : -1;
         if (blk >= 0 && blk < p.out_n_blocks)
-            dst = ((((int64_t)l * p.out_n_blocks + blk) << p.out_block_shift) | (i & ((1 << p.out_block_shift) - 1))) *
-                      geo.H +
-                  h;
+            dst = ((int64_t)l * p.out_n_blocks + blk) * ((int64_t)geo.H << p.out_block_shift) +
+                  (int64_t)(i & ((1 << p.out_block_shift) - 1)) * geo.H + h;
     } else {
         dst = r * p.B + i;
     }
